@@ -1,0 +1,446 @@
+#!/usr/bin/env python
+"""Benchmark of the grouped 4-bit MoE GEMM (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the hot path over one routed batch: for every token count
+of the workload, the gate_up projection (reads token rows, writes sorted rows)
+and the down projection (reads sorted rows, weights them, scatters to t*k+slot),
+each one grouped GEMM call through the C ABI. Inputs are synthetic (seeded);
+the weights are N(0, 0.02) quantized on the device by the library's quantizer.
+
+Metric: packed-weight GB/s = nibble + scale bytes of the experts each call
+touches, divided by device time (decode workloads); TFLOP/s = 2*R*N*K / time
+for the prefill workload. L2: the timed steps rotate over enough copies of the
+weight stacks that the bytes between two uses of one copy exceed twice the L2
+size. Multi-GPU: one independent replica per rank (the path has no exchange
+step), value = all ranks' work / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+from synth.workloads import WORKLOADS, expert_bytes  # noqa: E402
+
+METRIC = "grouped 4-bit MoE GEMM: packed-weight GB/s (decode), TFLOP/s (prefill)"
+DEFAULT_WORKLOAD = "olmoe_decode_nf4"
+PREFILL_WORKLOADS = {"qwen3_prefill_nf4"}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--top-k", type=int, default=None, help="sweep workload: top_k (default first)")
+    ap.add_argument("--tokens", type=str, default=None, help="comma list overriding the token counts")
+    return ap.parse_args()
+
+
+def workload_calls(wl, seed, top_k=None, tokens=None):
+    """The grouped GEMM calls of one step: (T, projection, routed batch)."""
+    k = top_k if top_k is not None else wl.top_k[-1 if wl.name != "olmoe_sweep_nf4" else 0]
+    Ts = tokens if tokens is not None else wl.T
+    calls = []
+    for T in Ts:
+        b = synth.make_routed_batch(seed, T, wl.E, k, routing=wl.routing)
+        for proj in wl.projections:
+            calls.append((T, proj, b))
+    return calls, k
+
+
+def call_bytes(fmt, proj, b):
+    pb = expert_bytes(fmt, proj.N, proj.K)
+    n_act = int((np.diff(b.offsets) > 0).sum())
+    return n_act * (pb["nibbles"] + pb["scales"]), n_act * pb["nibbles"]
+
+
+def describe(wl, k):
+    projs = ", ".join(f"{p.name} K={p.K} N={p.N}" for p in wl.projections)
+    return (f"{wl.name}: {wl.note}; E={wl.E}, top_k={k}, {projs}, T in {list(wl.T)}, "
+            f"{wl.fmt}, routing {wl.routing}")
+
+
+# --------------------------------------------------------------------------
+# clocks sampled during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), \
+            d.get("bf16_tflops_sustained", 1400.0), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def kernel_source_hash(names):
+    h = hashlib.sha256()
+    for n in names:
+        h.update(open(os.path.join(ROOT, "bit_grouped_moe_gnf4_b200", "csrc", n), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the
+    current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(f"{kernel}:{workload}")
+    if not d:
+        return None
+    if d.get("source_hash") != kernel_source_hash(d.get("sources", [])):
+        return None
+    return d.get("bytes_per_launch")
+
+
+# --------------------------------------------------------------------------
+# the oracle on the host cores (CPU baseline and the reference arm)
+# --------------------------------------------------------------------------
+def oracle_sample(wl, calls, budget_s=15.0, seed=0):
+    """Run the oracle's grouped GEMM over whole calls of the step (smallest token
+    counts first) until ~budget_s of host time. The oracle's own quantization of
+    the inputs is untimed. Returns (bytes, flops, calls, gemm_seconds, cores)."""
+    from oracle import gnf4_oracle as O
+    from synth import generators as G
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    done_bytes = done_flop = gemm_s = 0.0
+    ncalls = 0
+    t_begin = time.perf_counter()
+    sdiv = 64 if wl.fmt == "nf4" else 32
+    q = O.quantize_nf4 if wl.fmt == "nf4" else O.quantize_mxfp4
+    for T, proj, b in sorted(calls, key=lambda c: c[0]):
+        Wh = np.zeros((wl.E, proj.N, proj.K // 2), np.uint8)
+        Sh = np.zeros((wl.E, proj.N, proj.K // sdiv), np.float32 if wl.fmt == "nf4" else np.uint8)
+        for e in b.active_experts():
+            Wh[e], Sh[e] = q(G.expert_weights(seed, int(e), proj.N, proj.K))
+        if proj.name == "gate_up":
+            x = synth.activations_bf16(seed, T, proj.K)
+            t1 = time.perf_counter()
+            O.grouped_gemm(wl.fmt, x, Wh, Sh, b.offsets, b.row_token, None, None, T_out=b.R)
+        else:
+            x = synth.activations_bf16(seed, b.R, proj.K, tag="x_down")
+            t1 = time.perf_counter()
+            O.grouped_gemm(wl.fmt, x, Wh, Sh, b.offsets, None, b.row_weight, b.row_dest, T_out=T * b.k)
+        gemm_s += time.perf_counter() - t1
+        nb, _ = call_bytes(wl.fmt, proj, b)
+        done_bytes += nb
+        done_flop += 2.0 * b.R * proj.N * proj.K
+        ncalls += 1
+        if time.perf_counter() - t_begin > budget_s:
+            break
+    return done_bytes, done_flop, ncalls, gemm_s, cores
+
+
+def run_reference(args, wl):
+    """The reference arm: the oracle as it stands, timed on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    calls, k = workload_calls(wl, args.seed, args.top_k, _tokens(args))
+    prefill = wl.name in PREFILL_WORKLOADS
+    from oracle import gnf4_oracle as O  # noqa: F401
+    times, vals = [], []
+    cores = 1
+    for i in range(args.warmup + args.steps):
+        nb, nf, nc, dt, cores = oracle_sample(wl, calls, budget_s=4.0, seed=args.seed)
+        if i >= args.warmup:
+            times.append(dt)
+            vals.append((nf / dt / 1e12) if prefill else (nb / dt / 1e9))
+    v = float(np.median(vals))
+    unit = "TFLOP/s" if prefill else "GB/s"
+    line = {"metric": METRIC, "value": v, "unit": unit, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * float(np.median(times)),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": describe(wl, k), "l2": "n/a (host)"},
+            "cpu_baseline": {"value": v, "unit": unit, "cores": cores, "kind": "oracle",
+                             "sample": "per step: whole grouped GEMM calls of the workload, smallest "
+                                       "token counts first, until ~4 s of host work; the rate counts "
+                                       "the oracle's grouped GEMM time only (its input quantization "
+                                       "is untimed)"},
+            "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def _tokens(args):
+    return [int(t) for t in args.tokens.split(",")] if args.tokens else None
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+    import bit_grouped_moe_gnf4_b200 as g
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    prefill = wl.name in PREFILL_WORKLOADS
+
+    calls, k = workload_calls(wl, args.seed, args.top_k, _tokens(args))
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
+
+    # weight stacks per projection, drawn on the device, quantized by the library
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(args.seed + 1000 * rank)
+    stacks = {}
+    stack_bytes = 0
+    for proj in wl.projections:
+        Wl, Sl = [], []
+        for e in range(wl.E):
+            w = torch.randn((proj.N, proj.K), generator=gen, device=dev, dtype=torch.float32) * 0.02
+            if wl.fmt == "nf4":
+                p, s = g.quantize_nf4(w)
+            else:
+                p, s = g.quantize_mxfp4(w)
+            Wl.append(p)
+            Sl.append(s)
+        W = torch.stack(Wl)
+        S = torch.stack(Sl)
+        del Wl, Sl
+        stacks[proj.name] = [(W, S)]
+        stack_bytes += W.numel() + S.numel() * S.element_size()
+    # copies so that two uses of one copy are > 2 x L2 apart
+    step_bytes = sum(call_bytes(wl.fmt, p, b)[0] for _, p, b in calls)
+    ncopies = max(1, min(8, int(np.ceil(2.0 * l2 / max(1, step_bytes))) + 1))
+    free = torch.cuda.mem_get_info(dev)[0]
+    while ncopies > 1 and (ncopies - 1) * stack_bytes > 0.5 * free:
+        ncopies -= 1
+    for proj in wl.projections:
+        W, S = stacks[proj.name][0]
+        for _ in range(ncopies - 1):
+            stacks[proj.name].append((W.clone(), S.clone()))
+
+    # per-call device inputs, outputs and pinned host mirrors (end-to-end leg)
+    prepared = []
+    for T, proj, b in calls:
+        if proj.name == "gate_up":
+            xb = synth.activations_bf16(args.seed, T, proj.K)
+            tok, wt, dst, T_out = b.row_token, None, None, b.R
+        else:
+            xb = synth.activations_bf16(args.seed, b.R, proj.K, tag="x_down")
+            tok, wt, dst, T_out = None, b.row_weight, b.row_dest, T * b.k
+        xh = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).pin_memory()
+        h = {"x": xh, "off": torch.from_numpy(b.offsets).pin_memory()}
+        for nm, a in (("tok", tok), ("wt", wt), ("dst", dst)):
+            h[nm] = None if a is None else torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+        d = {nm: (None if t is None else t.to(dev)) for nm, t in h.items()}
+        out = torch.zeros((T_out, proj.N), dtype=torch.bfloat16, device=dev)
+        outh = torch.empty((T_out, proj.N), dtype=torch.bfloat16).pin_memory()
+        nb, nn = call_bytes(wl.fmt, proj, b)
+        prepared.append(dict(T=T, proj=proj, b=b, h=h, d=d, out=out, outh=outh, bytes=nb, nib=nn,
+                             flop=2.0 * b.R * proj.N * proj.K))
+
+    fn = g.grouped_gemm
+
+    def one_call(c, copy, ev=None):
+        W, S = stacks[c["proj"].name][copy]
+        d = c["d"]
+        if ev is not None:
+            ev[0].record(stream)
+        fn(wl.fmt, d["x"], W, S, d["off"], row_token=d["tok"], row_weight=d["wt"], row_dest=d["dst"],
+           out=c["out"], R=c["b"].R, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    def step(i, evs=None):
+        copy = i % ncopies
+        for j, c in enumerate(prepared):
+            one_call(c, copy, None if evs is None else evs[j])
+
+    # warm-up
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    launches_per_step = sum(g.launches_per_call(c["b"].R) for c in prepared)
+    ev_calls = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in prepared] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, ev_calls[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    call_ms = np.array([[s.elapsed_time(e) for (s, e) in row] for row in ev_calls])  # [steps, calls]
+
+    # end-to-end: host buffers in, result back, through the same public call
+    e2e_steps = max(3, min(args.steps, 10))
+    h2d = sum(sum(t.numel() * t.element_size() for t in c["h"].values() if t is not None) for c in prepared)
+    d2h = sum(c["outh"].numel() * 2 for c in prepared)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(e2e_steps):
+        copy = i % ncopies
+        for c in prepared:
+            for nm, t in c["h"].items():
+                if t is not None:
+                    c["d"][nm].copy_(t, non_blocking=True)
+            one_call(c, copy)
+            c["outh"].copy_(c["out"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    # max over ranks
+    ms_step = total_ms / args.steps
+    if world > 1:
+        t = torch.tensor([ms_step, e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step, e2e_ms = float(t[0]), float(t[1])
+
+    work_bytes = sum(c["bytes"] for c in prepared)
+    work_flop = sum(c["flop"] for c in prepared)
+    if prefill:
+        value = world * work_flop / (ms_step * 1e-3) / 1e12
+        e2e_v = world * work_flop / (e2e_ms * 1e-3) / 1e12
+        unit = "TFLOP/s"
+    else:
+        value = world * work_bytes / (ms_step * 1e-3) / 1e9
+        e2e_v = world * work_bytes / (e2e_ms * 1e-3) / 1e9
+        unit = "GB/s"
+
+    hbm, tc_burst, tc_sust, src = measured_peaks()
+    mean_call_ms = call_ms.mean(axis=0)
+    if prefill:
+        achieved = work_flop / (call_ms.sum(axis=1).mean() * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_sust, "unit": "TFLOP/s",
+                "frac": achieved / tc_sust, "peak_source": f"{src} bf16 sustained (kernel inside a step)"}
+    else:
+        achieved = work_bytes / (call_ms.sum(axis=1).mean() * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "peak_source": f"{src} HBM copy"}
+    roof["traffic"] = recorded_traffic("decode_band" if not prefill else "prefill_band", wl.name)
+    roof["kernel"] = "prefill_band_kernel" if prefill else "decode_band_kernel"
+    roof["per_call_ms"] = [round(float(x), 5) for x in mean_call_ms]
+    roof["per_call"] = [f"T={c['T']} {c['proj'].name}" for c in prepared]
+
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": describe(wl, k), "format": wl.fmt,
+                   "algorithmic_bytes_per_step": work_bytes, "flop_per_step": work_flop,
+                   "l2": f"rotating {ncopies} weight-stack copies ({ncopies * stack_bytes / 1e6:.0f} MB; "
+                         f"step reads {step_bytes / 1e6:.0f} MB; L2 {l2 / 1e6:.0f} MB)",
+                   "parallelism": f"replicas x{world}"},
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": {"value": e2e_v, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "roofline": roof,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nb, nf, nc, dt, cores = oracle_sample(wl, [(c["T"], c["proj"], c["b"]) for c in prepared],
+                                              budget_s=12.0, seed=args.seed)
+        v = (nf / dt / 1e12) if prefill else (nb / dt / 1e9)
+        line["cpu_baseline"] = {"value": v, "unit": unit, "cores": cores, "kind": "oracle",
+                                "sample": f"{nc} whole grouped GEMM calls of the step (smallest token "
+                                          f"counts first); {dt:.1f} s in the oracle's grouped GEMM, "
+                                          f"its quantization of the inputs untimed"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

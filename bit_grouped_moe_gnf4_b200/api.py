@@ -1,0 +1,121 @@
+"""Thin torch-facing wrappers over the C ABI (argument marshalling only).
+
+Every step of the computation runs in the CUDA kernels of libgnf4.so; these
+functions only pass device pointers, sizes and the current stream.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import lib, check
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, name: str) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def quantize_nf4(w: torch.Tensor, packed: Optional[torch.Tensor] = None,
+                 absmax: Optional[torch.Tensor] = None, stream=None):
+    """fp32 ``[..., K]`` device tensor -> (packed uint8 ``[..., K//2]``, absmax fp32 ``[..., K//64]``)."""
+    _need(w, torch.float32, "w")
+    K = w.shape[-1]
+    rows = w.numel() // K if K else 0
+    lead = tuple(w.shape[:-1])
+    if packed is None:
+        packed = torch.empty(lead + (K // 2,), dtype=torch.uint8, device=w.device)
+    if absmax is None:
+        absmax = torch.empty(lead + (K // 64,), dtype=torch.float32, device=w.device)
+    check(lib.gnf4_quantize_nf4(_ptr(w), rows, K, _ptr(packed), _ptr(absmax), _stream(stream)),
+          "gnf4_quantize_nf4")
+    return packed, absmax
+
+
+def quantize_mxfp4(w: torch.Tensor, blocks: Optional[torch.Tensor] = None,
+                   scales: Optional[torch.Tensor] = None, stream=None):
+    """fp32 ``[..., K]`` device tensor -> (blocks uint8 ``[..., K//2]``, scales uint8 ``[..., K//32]``)."""
+    _need(w, torch.float32, "w")
+    K = w.shape[-1]
+    rows = w.numel() // K if K else 0
+    lead = tuple(w.shape[:-1])
+    if blocks is None:
+        blocks = torch.empty(lead + (K // 2,), dtype=torch.uint8, device=w.device)
+    if scales is None:
+        scales = torch.empty(lead + (K // 32,), dtype=torch.uint8, device=w.device)
+    check(lib.gnf4_quantize_mxfp4(_ptr(w), rows, K, _ptr(blocks), _ptr(scales), _stream(stream)),
+          "gnf4_quantize_mxfp4")
+    return blocks, scales
+
+
+def grouped_gemm(fmt: str, x: torch.Tensor, W: torch.Tensor, scales: torch.Tensor,
+                 expert_offsets: torch.Tensor, row_token: Optional[torch.Tensor] = None,
+                 row_weight: Optional[torch.Tensor] = None, row_dest: Optional[torch.Tensor] = None,
+                 out: Optional[torch.Tensor] = None, T_out: Optional[int] = None, flags: int = 0,
+                 R: Optional[int] = None, stream=None) -> torch.Tensor:
+    """One grouped GEMM call (see include/gnf4.h). ``R`` (the routed row count) is
+    taken from ``row_token``/``row_weight``/``row_dest`` when one is given, else it
+    must be passed (it is never read back from the device)."""
+    if fmt not in ("nf4", "mxfp4"):
+        raise ValueError("fmt must be 'nf4' or 'mxfp4'")
+    _need(x, torch.bfloat16, "x")
+    _need(W, torch.uint8, "W")
+    _need(scales, torch.float32 if fmt == "nf4" else torch.uint8, "scales")
+    _need(expert_offsets, torch.int64, "expert_offsets")
+    for name, t, dt in (("row_token", row_token, torch.int32), ("row_weight", row_weight, torch.float32),
+                        ("row_dest", row_dest, torch.int32)):
+        if t is not None:
+            _need(t, dt, name)
+    E, N, K2 = W.shape
+    K = x.shape[1]
+    if K2 * 2 != K:
+        raise ValueError(f"W is [E, N, K/2] = {tuple(W.shape)} but x has K = {K}")
+    if R is None:
+        for t in (row_token, row_weight, row_dest):
+            if t is not None:
+                R = t.numel()
+                break
+    if R is None:
+        raise ValueError("pass R (routed rows) when row_token, row_weight and row_dest are all None")
+    if out is None:
+        T_out = R if T_out is None else T_out
+        out = torch.empty((T_out, N), dtype=torch.bfloat16, device=x.device)
+    else:
+        _need(out, torch.bfloat16, "out")
+        T_out = out.shape[0]
+    fn = lib.gnf4_grouped_gemm_nf4 if fmt == "nf4" else lib.gnf4_grouped_gemm_mxfp4
+    check(fn(_ptr(x), _ptr(W), _ptr(scales), _ptr(expert_offsets), _ptr(row_token), _ptr(row_weight),
+             _ptr(row_dest), E, N, K, R, x.shape[0], T_out, _ptr(out), flags, _stream(stream)),
+          f"gnf4_grouped_gemm_{fmt}")
+    return out
+
+
+def grouped_gemm_nf4(x, W, absmax, expert_offsets, **kw):
+    return grouped_gemm("nf4", x, W, absmax, expert_offsets, **kw)
+
+
+def grouped_gemm_mxfp4(x, W, scales, expert_offsets, **kw):
+    return grouped_gemm("mxfp4", x, W, scales, expert_offsets, **kw)
+
+
+def launches_per_call(R: int, flags: int = 0) -> int:
+    return lib.gnf4_grouped_gemm_launches(R, flags)
+
+
+version = lib.gnf4_version

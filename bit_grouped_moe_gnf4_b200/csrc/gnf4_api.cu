@@ -1,0 +1,268 @@
+// The C ABI of include/gnf4.h: argument validation, band selection, launches.
+#include <climits>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <cuda_runtime.h>
+
+#include "../../include/gnf4.h"
+#include "gnf4_common.cuh"
+#include "gnf4_kernels.h"
+
+namespace gnf4 {
+
+// Groups with more than this many routed rows go to the prefill (tensor-core)
+// band; the rest to the decode band.
+constexpr int kDecodeMaxRows = 64;
+
+static thread_local char g_err[512] = "";
+
+static gnf4_status fail(gnf4_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+static gnf4_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(GNF4_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+static bool is_device_ptr(const void* p) {
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int device_sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (cached[dev] == 0) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 1;
+    }
+    return cached[dev];
+}
+
+static uint16_t host_bf16_rne(float f) {
+    uint32_t u;
+    std::memcpy(&u, &f, 4);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+LutPlanes make_lut(int fmt) {
+    // NF4 values (QLoRA / bitsandbytes NF4) and the OCP e2m1 magnitudes
+    static const float nf4[16] = {
+        -1.0f, -0.6961928009986877f, -0.5250730514526367f, -0.39491748809814453f,
+        -0.28444138169288635f, -0.18477343022823334f, -0.09105003625154495f, 0.0f,
+        0.07958029955625534f, 0.16093020141124725f, 0.24611230194568634f,
+        0.33791524171829224f, 0.44070982933044434f, 0.5626170039176941f,
+        0.7229568362236023f, 1.0f};
+    static const float e2m1[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+    LutPlanes L;
+    std::memset(&L, 0, sizeof(L));
+    const int n = (fmt == FMT_NF4) ? 16 : 8;
+    for (int i = 0; i < n; ++i) {
+        const uint16_t b = host_bf16_rne(fmt == FMT_NF4 ? nf4[i] : e2m1[i]);
+        L.lo[i >> 2] |= (uint32_t)(b & 0xFFu) << (8 * (i & 3));
+        L.hi[i >> 2] |= (uint32_t)(b >> 8) << (8 * (i & 3));
+    }
+    return L;
+}
+
+static gnf4_status check_quantize_args(const float* w, int64_t rows, int64_t K, const void* o1,
+                                       const void* o2, int64_t kmul) {
+    if (!w || !o1 || !o2) return fail(GNF4_ERR_INVALID_ARG, "null pointer argument");
+    if (rows < 0 || K <= 0) return fail(GNF4_ERR_INVALID_ARG, "rows must be >= 0 and K > 0");
+    if (K % kmul) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K must be a multiple of %lld", (long long)kmul);
+    if (!aligned16(w)) return fail(GNF4_ERR_MISALIGNED, "w must be 16-byte aligned");
+    if (!is_device_ptr(w) || !is_device_ptr(o1) || !is_device_ptr(o2))
+        return fail(GNF4_ERR_INVALID_ARG, "w and the outputs must be device memory");
+    return GNF4_OK;
+}
+
+// status word of the routing check
+__device__ unsigned g_check_status;
+
+__global__ void check_routing_kernel(const GroupedArgs p, int64_t T_in, int64_t T_out) {
+    unsigned bad = 0;
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t e = tid; e < p.E; e += stride)
+        if (p.offsets[e + 1] < p.offsets[e]) bad |= 1u;
+    if (tid == 0 && (p.offsets[0] != 0 || p.offsets[p.E] != p.R)) bad |= 2u;
+    for (int64_t r = tid; r < p.R; r += stride) {
+        if (p.row_token) {
+            const int32_t v = p.row_token[r];
+            if (v < 0 || v >= T_in) bad |= 4u;
+        }
+        if (p.row_dest) {
+            const int32_t v = p.row_dest[r];
+            if (v < 0 || v >= T_out) bad |= 8u;
+        }
+        if (p.row_weight && !isfinite(p.row_weight[r])) bad |= 16u;
+    }
+    if (bad) atomicOr(&g_check_status, bad);
+}
+
+cudaError_t launch_check_routing(const GroupedArgs& a, int64_t T_in, int64_t T_out,
+                                 unsigned* status_out, cudaStream_t s) {
+    const unsigned zero = 0;
+    cudaError_t e = cudaMemcpyToSymbolAsync(g_check_status, &zero, sizeof(zero), 0,
+                                            cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return e;
+    check_routing_kernel<<<64, 256, 0, s>>>(a, T_in, T_out);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbolAsync(status_out, g_check_status, sizeof(unsigned), 0,
+                                  cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return e;
+    return cudaStreamSynchronize(s);
+}
+
+static gnf4_status grouped(int fmt, const void* x, const uint8_t* W, const void* scales,
+                           const int64_t* offsets, const int32_t* row_token,
+                           const float* row_weight, const int32_t* row_dest, int64_t E,
+                           int64_t N, int64_t K, int64_t R, int64_t T_in, int64_t T_out,
+                           void* out, int flags, void* stream) {
+    const int64_t kmul = (fmt == FMT_NF4) ? 64 : 32;
+    if (!x || !W || !scales || !offsets || !out) return fail(GNF4_ERR_INVALID_ARG, "null pointer argument");
+    if (E < 1 || N < 1 || K < 1 || R < 0 || T_in < 0 || T_out < 0)
+        return fail(GNF4_ERR_INVALID_ARG, "sizes must be E,N,K >= 1 and R,T_in,T_out >= 0");
+    if (flags & ~(GNF4_CHECK | GNF4_FORCE_DECODE | GNF4_FORCE_PREFILL))
+        return fail(GNF4_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+    if ((flags & GNF4_FORCE_DECODE) && (flags & GNF4_FORCE_PREFILL))
+        return fail(GNF4_ERR_INVALID_ARG, "GNF4_FORCE_DECODE and GNF4_FORCE_PREFILL exclude each other");
+    if (K % kmul) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K must be a multiple of %lld", (long long)kmul);
+    if (N % 16) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "N must be a multiple of 16");
+    if (E > 2048) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "at most 2048 experts");
+    if (K > (int64_t)INT_MAX / 2 || N > (int64_t)INT_MAX || T_in > INT_MAX || T_out > INT_MAX)
+        return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K, N, T_in and T_out must fit in int32");
+    if (!row_token && T_in < R) return fail(GNF4_ERR_INVALID_ARG, "row_token is NULL but T_in < R");
+    if (!row_dest && T_out < R) return fail(GNF4_ERR_INVALID_ARG, "row_dest is NULL but T_out < R");
+    if (!aligned16(x) || !aligned16(W) || !aligned16(out))
+        return fail(GNF4_ERR_MISALIGNED, "x, W and out must be 16-byte aligned");
+    if (!is_device_ptr(x) || !is_device_ptr(W) || !is_device_ptr(scales) || !is_device_ptr(offsets) ||
+        !is_device_ptr(out) || (row_token && !is_device_ptr(row_token)) ||
+        (row_weight && !is_device_ptr(row_weight)) || (row_dest && !is_device_ptr(row_dest)))
+        return fail(GNF4_ERR_INVALID_ARG, "every buffer must be device memory of the current device");
+    if (R == 0) return GNF4_OK;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    GroupedArgs a;
+    a.x = reinterpret_cast<const uint16_t*>(x);
+    a.W = W;
+    a.scales = scales;
+    a.offsets = offsets;
+    a.row_token = row_token;
+    a.row_weight = row_weight;
+    a.row_dest = row_dest;
+    a.out = reinterpret_cast<uint16_t*>(out);
+    a.R = R;
+    a.E = (int)E;
+    a.N = (int)N;
+    a.K = (int)K;
+    static const LutPlanes lut_nf4 = make_lut(FMT_NF4);
+    static const LutPlanes lut_mx = make_lut(FMT_MXFP4);
+    a.lut = (fmt == FMT_NF4) ? lut_nf4 : lut_mx;
+
+    if (flags & GNF4_CHECK) {
+        unsigned st = 0;
+        cudaError_t e = launch_check_routing(a, T_in, T_out, &st, s);
+        if (e != cudaSuccess) return cuda_fail(e, "routing check");
+        if (st) return fail(GNF4_ERR_DEVICE_STATUS,
+                            "bad routing metadata (status 0x%x: 1 offsets decrease, 2 offsets[0] != 0 "
+                            "or offsets[E] != R, 4 row_token out of range, 8 row_dest out of range, "
+                            "16 non-finite row_weight)", st);
+    }
+
+    // band split by rows per group; decided on the device from the offsets
+    int split = kDecodeMaxRows;
+    if (flags & GNF4_FORCE_DECODE) split = INT_MAX;
+    if (flags & GNF4_FORCE_PREFILL) split = 0;
+#ifndef GNF4_HAVE_PREFILL
+    split = INT_MAX;
+#endif
+    if (split >= 1) {
+        a.m_lo = 1;
+        a.m_hi = split;
+        cudaError_t e = launch_decode_band(fmt, a, s);
+        if (e != cudaSuccess) return cuda_fail(e, "decode band launch");
+    }
+#ifdef GNF4_HAVE_PREFILL
+    if (split < INT_MAX && R > split) {
+        a.m_lo = split + 1;
+        a.m_hi = INT_MAX;
+        cudaError_t e = launch_prefill_band(fmt, a, s);
+        if (e != cudaSuccess) return cuda_fail(e, "prefill band launch");
+    }
+#endif
+    return GNF4_OK;
+}
+
+}  // namespace gnf4
+
+using namespace gnf4;
+
+extern "C" {
+
+const char* gnf4_last_error(void) { return g_err; }
+
+int gnf4_version(void) { return 100; }
+
+gnf4_status gnf4_quantize_nf4(const float* w, int64_t rows, int64_t K, uint8_t* packed,
+                              float* absmax, void* stream) {
+    gnf4_status st = check_quantize_args(w, rows, K, packed, absmax, 64);
+    if (st != GNF4_OK) return st;
+    cudaError_t e = launch_quantize_nf4(w, rows, K, packed, absmax, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GNF4_OK : cuda_fail(e, "quantize_nf4 launch");
+}
+
+gnf4_status gnf4_quantize_mxfp4(const float* w, int64_t rows, int64_t K, uint8_t* blocks,
+                                uint8_t* scales, void* stream) {
+    gnf4_status st = check_quantize_args(w, rows, K, blocks, scales, 32);
+    if (st != GNF4_OK) return st;
+    cudaError_t e = launch_quantize_mxfp4(w, rows, K, blocks, scales, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GNF4_OK : cuda_fail(e, "quantize_mxfp4 launch");
+}
+
+gnf4_status gnf4_grouped_gemm_nf4(const void* x, const uint8_t* W, const float* absmax,
+                                  const int64_t* expert_offsets, const int32_t* row_token,
+                                  const float* row_weight, const int32_t* row_dest, int64_t E,
+                                  int64_t N, int64_t K, int64_t R, int64_t T_in, int64_t T_out,
+                                  void* out, int flags, void* stream) {
+    return grouped(FMT_NF4, x, W, absmax, expert_offsets, row_token, row_weight, row_dest, E, N,
+                   K, R, T_in, T_out, out, flags, stream);
+}
+
+gnf4_status gnf4_grouped_gemm_mxfp4(const void* x, const uint8_t* W, const uint8_t* scales,
+                                    const int64_t* expert_offsets, const int32_t* row_token,
+                                    const float* row_weight, const int32_t* row_dest, int64_t E,
+                                    int64_t N, int64_t K, int64_t R, int64_t T_in, int64_t T_out,
+                                    void* out, int flags, void* stream) {
+    return grouped(FMT_MXFP4, x, W, scales, expert_offsets, row_token, row_weight, row_dest, E,
+                   N, K, R, T_in, T_out, out, flags, stream);
+}
+
+int gnf4_grouped_gemm_launches(int64_t R, int flags) {
+    if (R <= 0) return 0;
+    int n = (flags & GNF4_CHECK) ? 1 : 0;
+#ifdef GNF4_HAVE_PREFILL
+    if (flags & GNF4_FORCE_DECODE) return n + 1;
+    if (flags & GNF4_FORCE_PREFILL) return n + 1;
+    return n + 1 + (R > kDecodeMaxRows ? 1 : 0);
+#else
+    return n + 1;
+#endif
+}
+
+}  // extern "C"

@@ -1,0 +1,120 @@
+// Shared device-side pieces of the gnf4 kernels: argument block, nibble decode
+// through byte permutes, scale decode, small PTX wrappers.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace gnf4 {
+
+enum Fmt : int { FMT_NF4 = 0, FMT_MXFP4 = 1 };
+
+// Byte planes of a 16-entry bf16 table for the prmt decode: lo[i] holds the low
+// bytes of entries 4i..4i+3 (entry 4i in bits 0..7), hi[i] the high bytes.
+// For MXFP4 only entries 0..7 (the e2m1 magnitudes) are used; bit 3 of a code
+// is its sign.
+struct LutPlanes {
+    uint32_t lo[4];
+    uint32_t hi[4];
+};
+
+struct GroupedArgs {
+    const uint16_t* x;          // bf16 [T_in, K]
+    const uint8_t* W;           // [E, N, K/2]
+    const void* scales;         // NF4: f32 [E, N, K/64]; MXFP4: u8 [E, N, K/32]
+    const int64_t* offsets;     // [E+1]
+    const int32_t* row_token;   // [R] or null
+    const float* row_weight;    // [R] or null
+    const int32_t* row_dest;    // [R] or null
+    uint16_t* out;              // bf16 [T_out, N]
+    int64_t R;
+    int E, N, K;
+    int m_lo, m_hi;             // this band takes groups with m_lo <= rows <= m_hi
+    LutPlanes lut;
+};
+
+// Host-side: the decode tables of each format (bf16 of the codebook values,
+// round to nearest even from the fp32 values).
+LutPlanes make_lut(int fmt);
+
+// ---------------------------------------------------------------------------
+// device helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// Decode the 8 nibbles of one 32-bit word into four bf16x2 words: o[i] holds the
+// two elements of byte i, the lower-k element in the low 16 bits.
+//   NF4 (bitsandbytes order): element 2j is the HIGH nibble of byte j.
+//   MXFP4 (OCP order):        element 2j is the LOW nibble of byte j.
+// Codes are looked up by byte permutes (prmt) from tables held in registers:
+// the low three bits of each nibble select a table byte, bit 3 picks the upper
+// half of the table (NF4) or sets the sign (MXFP4). The result equals a plain
+// 16-entry table lookup bit for bit.
+template <int FMT>
+__device__ __forceinline__ void decode_word(uint32_t w, const LutPlanes& L, uint32_t (&o)[4]) {
+    const uint32_t s_lo = w & 0x77777777u;       // 3-bit selectors, nibbles 0..3 in bits 0..15
+    const uint32_t s_hi = s_lo >> 16;            // nibbles 4..7
+    const uint32_t w4 = w << 4;                  // puts bit 3 of every low nibble at a byte msb
+    // byte i of m = 0xFF when nibble i (of the half) has bit 3 set
+    const uint32_t m_lo = prmt(w, w4, 0x9D8Cu);
+    const uint32_t m_hi = prmt(w, w4, 0xBFAEu);
+    if constexpr (FMT == FMT_NF4) {
+        uint32_t lo = (prmt(L.lo[0], L.lo[1], s_lo) & ~m_lo) | (prmt(L.lo[2], L.lo[3], s_lo) & m_lo);
+        uint32_t hi = (prmt(L.hi[0], L.hi[1], s_lo) & ~m_lo) | (prmt(L.hi[2], L.hi[3], s_lo) & m_lo);
+        o[0] = prmt(lo, hi, 0x4051u);            // byte 0: high nibble first
+        o[1] = prmt(lo, hi, 0x6273u);
+        lo = (prmt(L.lo[0], L.lo[1], s_hi) & ~m_hi) | (prmt(L.lo[2], L.lo[3], s_hi) & m_hi);
+        hi = (prmt(L.hi[0], L.hi[1], s_hi) & ~m_hi) | (prmt(L.hi[2], L.hi[3], s_hi) & m_hi);
+        o[2] = prmt(lo, hi, 0x4051u);
+        o[3] = prmt(lo, hi, 0x6273u);
+    } else {
+        uint32_t lo = prmt(L.lo[0], L.lo[1], s_lo);
+        uint32_t hi = prmt(L.hi[0], L.hi[1], s_lo) | (m_lo & 0x80808080u);
+        o[0] = prmt(lo, hi, 0x5140u);            // byte 0: low nibble first
+        o[1] = prmt(lo, hi, 0x7362u);
+        lo = prmt(L.lo[0], L.lo[1], s_hi);
+        hi = prmt(L.hi[0], L.hi[1], s_hi) | (m_hi & 0x80808080u);
+        o[2] = prmt(lo, hi, 0x5140u);
+        o[3] = prmt(lo, hi, 0x7362u);
+    }
+}
+
+// e8m0 -> fp32: 2^(s-127); s = 0 is the subnormal 2^-127, s = 255 is NaN.
+__device__ __forceinline__ float e8m0_to_f32(uint32_t s) {
+    if (s == 0u) return __uint_as_float(0x00400000u);
+    if (s == 255u) return __uint_as_float(0x7FC00000u);
+    return __uint_as_float(s << 23);
+}
+
+template <int FMT>
+__device__ __forceinline__ float load_scale(const void* scales, int64_t idx) {
+    if constexpr (FMT == FMT_NF4) {
+        return __ldg(reinterpret_cast<const float*>(scales) + idx);
+    } else {
+        return e8m0_to_f32(__ldg(reinterpret_cast<const uint8_t*>(scales) + idx));
+    }
+}
+
+// fp32 -> bf16 bits, round to nearest even (NaN stays NaN).
+__device__ __forceinline__ uint16_t f32_to_bf16_rne(float v) {
+    uint32_t u = __float_as_uint(v);
+    if ((u & 0x7FFFFFFFu) > 0x7F800000u) return (uint16_t)((u >> 16) | 0x40u);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+}  // namespace gnf4

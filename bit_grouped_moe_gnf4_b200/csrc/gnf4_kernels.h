@@ -1,0 +1,30 @@
+// Internal launcher declarations (host side); the public C ABI is include/gnf4.h.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "gnf4_common.cuh"
+
+namespace gnf4 {
+
+cudaError_t launch_quantize_nf4(const float* w, int64_t rows, int64_t K, uint8_t* packed,
+                                float* absmax, cudaStream_t s);
+cudaError_t launch_quantize_mxfp4(const float* w, int64_t rows, int64_t K, uint8_t* blocks,
+                                  uint8_t* scales, cudaStream_t s);
+
+// Decode band: register-decoded warp MMAs, K split across the warps of a CTA.
+// Takes the groups whose row count m satisfies a.m_lo <= m <= a.m_hi.
+cudaError_t launch_decode_band(int fmt, const GroupedArgs& a, cudaStream_t s);
+
+// Prefill band: tcgen05 MMAs into tensor memory with the per-block fp32
+// rescale outside the MMA. Takes the groups with a.m_lo <= m <= a.m_hi.
+cudaError_t launch_prefill_band(int fmt, const GroupedArgs& a, cudaStream_t s);
+
+// Device-side validation of the routing metadata; writes a status word.
+cudaError_t launch_check_routing(const GroupedArgs& a, int64_t T_in, int64_t T_out,
+                                 unsigned* status_out, cudaStream_t s);
+
+int device_sm_count();
+
+}  // namespace gnf4

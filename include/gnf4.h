@@ -1,0 +1,147 @@
+/*
+ * gnf4 -- grouped GEMM for routed Mixture-of-Experts layers computed directly on
+ * 4-bit-packed expert weights (NF4 or MXFP4), for NVIDIA B200 (sm_100a).
+ *
+ * C ABI. Every pointer argument marked "device" must be device (or managed)
+ * memory of the current CUDA device; the library checks this and refuses host
+ * pointers. The caller owns and allocates every buffer; the library allocates
+ * nothing and keeps no per-call state. Every call is asynchronous on `stream`
+ * (a cudaStream_t passed as void*, NULL = the legacy default stream) and does
+ * no host synchronisation unless GNF4_CHECK is set.
+ *
+ * Errors: each entry point returns a gnf4_status; on failure nothing was
+ * launched (argument errors) or the CUDA error is reported (GNF4_ERR_CUDA),
+ * and gnf4_last_error() returns a message for the calling thread.
+ *
+ * Citations name the grouped-nf4-gemm pages by title and section.
+ */
+#ifndef GNF4_H
+#define GNF4_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gnf4_status {
+    GNF4_OK = 0,
+    GNF4_ERR_INVALID_ARG = 1,      /* null pointer, negative size, host pointer, bad flag */
+    GNF4_ERR_UNSUPPORTED_SHAPE = 2,/* K or N not a multiple of what the format needs */
+    GNF4_ERR_MISALIGNED = 3,       /* a buffer that must be 16-byte aligned is not */
+    GNF4_ERR_CUDA = 4,             /* a CUDA runtime call or launch failed */
+    GNF4_ERR_DEVICE_STATUS = 5     /* GNF4_CHECK found bad routing metadata on the device */
+} gnf4_status;
+
+/* flags for the grouped GEMM entry points */
+#define GNF4_CHECK          0x1  /* validate offsets / row_token / row_dest on the device
+                                    first (one extra kernel and a stream sync); a bad
+                                    value returns GNF4_ERR_DEVICE_STATUS, nothing else runs */
+#define GNF4_FORCE_DECODE   0x2  /* run every group through the decode band (testing) */
+#define GNF4_FORCE_PREFILL  0x4  /* run every group through the prefill band (testing) */
+
+/* Message describing the last failure on the calling thread ("" if none). */
+const char* gnf4_last_error(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int gnf4_version(void);
+
+/*
+ * NF4 quantizer (input generation).
+ * Follows the grouped-nf4-gemm README (0.11.0), "Try it on CPU right now", block 1:
+ * a row-major fp32 matrix [rows, K] becomes [rows, K/2] uint8 codes plus one fp32
+ * absmax per 64 consecutive K elements ("Supported scope" on the solution page:
+ * blocksize 64, K % 64 == 0, bitsandbytes gemm_4bit layout).
+ *   absmax[r, b] = max |w[r, 64b .. 64b+63]|
+ *   code = nearest NF4 value to fl32(w / absmax) (ties to the lower code; an
+ *          all-zero block gets code 7, the value 0)
+ *   packed[r, j] = (code[r, 2j] << 4) | code[r, 2j+1]
+ * w      device fp32 [rows, K], finite values (NaN/inf give unspecified codes)
+ * packed device uint8 [rows, K/2]     (written)
+ * absmax device fp32  [rows, K/64]    (written)
+ * Output bytes are bit-identical to the CPU oracle's quantizer.
+ * Errors: INVALID_ARG (null/host pointer, rows < 0, K <= 0), UNSUPPORTED_SHAPE (K % 64).
+ */
+gnf4_status gnf4_quantize_nf4(const float* w, int64_t rows, int64_t K,
+                              uint8_t* packed, float* absmax, void* stream);
+
+/*
+ * MXFP4 quantizer (input generation): OCP e2m1 codes with one e8m0 scale per 32
+ * K elements. README (0.11.0), "Try it on CPU right now", block 2 (blocks
+ * [.., K/32, 16] u8 + scales [.., K/32] u8, the same bytes as the kernel view
+ * [rows, K/2] + [rows, K/32] of "The NVMe tier").
+ *   E = floor(log2 amax) - 2 (from the fp32 exponent field, clamped to [-127,127];
+ *       E = 0 for an all-zero block), scales[r, b] = E + 127
+ *   code = e2m1 nearest to w * 2^-E, ties to the even code, |.| > 6 -> 6,
+ *          sign bit set when w < 0
+ *   blocks[r, j] = code[r, 2j] | (code[r, 2j+1] << 4)
+ * w device fp32 [rows, K]; blocks device uint8 [rows, K/2]; scales device uint8 [rows, K/32].
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (K % 32).
+ */
+gnf4_status gnf4_quantize_mxfp4(const float* w, int64_t rows, int64_t K,
+                                uint8_t* blocks, uint8_t* scales, void* stream);
+
+/*
+ * Grouped GEMM on NF4-packed expert weights.
+ * The op of the solution page "How do I run a grouped GEMM directly on NF4
+ * packed MoE expert weights, without dequantizing to bf16 first?" ("Smallest
+ * correct example", "Supported scope"): every active expert in one call, nibbles
+ * decoded on chip, fp32 block scaling and accumulation, bf16 output, no bf16
+ * copy of any expert in memory. Routed rows r = 0..R-1 are sorted by expert:
+ * expert e owns rows [expert_offsets[e], expert_offsets[e+1]).
+ *
+ *   out[dest(r), n] = bf16_rne( w(r) * sum_k x[tok(r), k] * What[e(r), n, k] )
+ *   What[e, n, k]   = nf4[code(e, n, k)] * absmax[e, n, k/64]
+ *   tok(r)  = row_token ? row_token[r] : r
+ *   w(r)    = row_weight ? row_weight[r] : 1
+ *   dest(r) = row_dest ? row_dest[r] : r
+ *
+ * x              device bf16 [T_in, K], 16-byte aligned
+ * W              device uint8 [E, N, K/2] (NF4 codes as gnf4_quantize_nf4 writes them), 16-byte aligned
+ * absmax         device fp32  [E, N, K/64]
+ * expert_offsets device int64 [E+1]: offsets[0] = 0, non-decreasing, offsets[E] = R;
+ *                empty experts (equal neighbours) are legal and cost nothing
+ * row_token      device int32 [R] in [0, T_in), or NULL (then T_in >= R)
+ * row_weight     device fp32  [R], or NULL
+ * row_dest       device int32 [R] in [0, T_out), pairwise distinct, or NULL (then T_out >= R)
+ * out            device bf16 [T_out, N], 16-byte aligned; rows that no routed row
+ *                names are not written
+ * E >= 1, N % 16 == 0, K % 64 == 0, R >= 0 (R == 0 launches nothing), T_in, T_out < 2^31.
+ * Offsets are 64-bit everywhere inside, so stacks past 2^31 bytes are addressed
+ * correctly (the int64-offset rule under "Supported scope" / "Limitations").
+ * flags: 0, or GNF4_CHECK / GNF4_FORCE_DECODE / GNF4_FORCE_PREFILL (above).
+ * Results are deterministic: the same inputs give the same bits on every call.
+ */
+gnf4_status gnf4_grouped_gemm_nf4(const void* x, const uint8_t* W, const float* absmax,
+                                  const int64_t* expert_offsets, const int32_t* row_token,
+                                  const float* row_weight, const int32_t* row_dest,
+                                  int64_t E, int64_t N, int64_t K, int64_t R,
+                                  int64_t T_in, int64_t T_out, void* out,
+                                  int flags, void* stream);
+
+/*
+ * Grouped GEMM on MXFP4-packed expert weights: identical contract, with
+ *   What[e, n, k] = e2m1[code(e, n, k)] * 2^(scales[e, n, k/32] - 127)
+ * W      device uint8 [E, N, K/2] (element 2j in the low nibble of byte j)
+ * scales device uint8 [E, N, K/32] (e8m0; 255 decodes to NaN)
+ * K % 32 == 0. The README's "MXFP4 native-byte lane": the same mainloop by
+ * table swap, on the released bytes.
+ */
+gnf4_status gnf4_grouped_gemm_mxfp4(const void* x, const uint8_t* W, const uint8_t* scales,
+                                    const int64_t* expert_offsets, const int32_t* row_token,
+                                    const float* row_weight, const int32_t* row_dest,
+                                    int64_t E, int64_t N, int64_t K, int64_t R,
+                                    int64_t T_in, int64_t T_out, void* out,
+                                    int flags, void* stream);
+
+/*
+ * How many kernels one grouped GEMM call with R routed rows and these flags
+ * launches (0 when R == 0; GNF4_CHECK adds one). Host-only, no CUDA call.
+ */
+int gnf4_grouped_gemm_launches(int64_t R, int flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GNF4_H */

@@ -56,3 +56,14 @@ WORKLOADS = {
                      Projection("down", K=1024, N=2048)),
         routing="zipf", note="M-axis sweep, Zipf(1.2)-skewed routing"),
 }
+
+
+def expert_bytes(fmt: str, N: int, K: int) -> dict:
+    """Algorithmic bytes of one packed ``[N, K]`` expert matrix: the 4-bit codes
+    (K/2 bytes per row) plus one fp32 absmax per 64 K (NF4) or one e8m0 byte per
+    32 K (MXFP4)."""
+    if fmt == "nf4":
+        return {"nibbles": N * K // 2, "scales": N * (K // 64) * 4}
+    if fmt == "mxfp4":
+        return {"nibbles": N * K // 2, "scales": N * (K // 32)}
+    raise ValueError(fmt)

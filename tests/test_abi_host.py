@@ -1,0 +1,90 @@
+"""Host-side checks of the C ABI (no GPU needed, no kernel launched).
+
+The library loads, exports every symbol include/gnf4.h declares, and rejects
+bad arguments with the documented status before touching the device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_grouped_moe_gnf4_b200 import _lib
+from bit_grouped_moe_gnf4_b200._lib import lib
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "gnf4.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gnf4_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_four_ops():
+    names = declared_functions()
+    for op in ("gnf4_quantize_nf4", "gnf4_quantize_mxfp4", "gnf4_grouped_gemm_nf4",
+               "gnf4_grouped_gemm_mxfp4"):
+        assert op in names
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert names, "no declarations parsed"
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in gnf4.h but not exported"
+    assert set(_lib.EXPORTED) == set(names)
+
+
+def test_version_and_launch_count():
+    assert lib.gnf4_version() >= 100
+    assert lib.gnf4_grouped_gemm_launches(0, 0) == 0
+    assert lib.gnf4_grouped_gemm_launches(1, 0) == 1
+    assert lib.gnf4_grouped_gemm_launches(1, _lib.GNF4_CHECK) == 2
+
+
+FAKE = 0x7f0000001000          # 16-byte aligned, never dereferenced: validation fails first
+
+
+def _gemm(**kw):
+    a = dict(x=FAKE, W=FAKE, s=FAKE, off=FAKE, tok=None, wt=None, dst=None, E=4, N=128, K=256,
+             R=8, T_in=8, T_out=8, out=FAKE, flags=0)
+    a.update(kw)
+    return lib.gnf4_grouped_gemm_nf4(a["x"], a["W"], a["s"], a["off"], a["tok"], a["wt"], a["dst"],
+                                     a["E"], a["N"], a["K"], a["R"], a["T_in"], a["T_out"],
+                                     a["out"], a["flags"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=None), _lib.GNF4_ERR_INVALID_ARG),
+    (dict(off=None), _lib.GNF4_ERR_INVALID_ARG),
+    (dict(out=None), _lib.GNF4_ERR_INVALID_ARG),
+    (dict(E=0), _lib.GNF4_ERR_INVALID_ARG),
+    (dict(R=-1), _lib.GNF4_ERR_INVALID_ARG),
+    (dict(flags=0x40), _lib.GNF4_ERR_INVALID_ARG),
+    (dict(flags=_lib.GNF4_FORCE_DECODE | _lib.GNF4_FORCE_PREFILL), _lib.GNF4_ERR_INVALID_ARG),
+    (dict(K=96), _lib.GNF4_ERR_UNSUPPORTED_SHAPE),
+    (dict(N=120), _lib.GNF4_ERR_UNSUPPORTED_SHAPE),
+    (dict(E=4096), _lib.GNF4_ERR_UNSUPPORTED_SHAPE),
+    (dict(T_in=4), _lib.GNF4_ERR_INVALID_ARG),          # row_token NULL needs T_in >= R
+    (dict(T_out=4), _lib.GNF4_ERR_INVALID_ARG),         # row_dest NULL needs T_out >= R
+    (dict(x=FAKE + 8), _lib.GNF4_ERR_MISALIGNED),
+    (dict(out=FAKE + 2), _lib.GNF4_ERR_MISALIGNED),
+])
+def test_grouped_gemm_argument_errors(kw, status):
+    assert _gemm(**kw) == status
+    assert lib.gnf4_last_error()
+
+
+def test_mxfp4_shape_rule_is_k_multiple_of_32():
+    st = lib.gnf4_grouped_gemm_mxfp4(FAKE, FAKE, FAKE, FAKE, None, None, None, 4, 128, 48, 8, 8, 8,
+                                     FAKE, 0, None)
+    assert st == _lib.GNF4_ERR_UNSUPPORTED_SHAPE
+
+
+def test_quantize_argument_errors():
+    assert lib.gnf4_quantize_nf4(None, 4, 64, FAKE, FAKE, None) == _lib.GNF4_ERR_INVALID_ARG
+    assert lib.gnf4_quantize_nf4(FAKE, 4, 96, FAKE, FAKE, None) == _lib.GNF4_ERR_UNSUPPORTED_SHAPE
+    assert lib.gnf4_quantize_mxfp4(FAKE, 4, 48, FAKE, FAKE, None) == _lib.GNF4_ERR_UNSUPPORTED_SHAPE
+    assert lib.gnf4_quantize_mxfp4(FAKE, -1, 64, FAKE, FAKE, None) == _lib.GNF4_ERR_INVALID_ARG
+    assert lib.gnf4_quantize_nf4(FAKE + 4, 4, 64, FAKE, FAKE, None) == _lib.GNF4_ERR_MISALIGNED
