@@ -2,15 +2,23 @@
 
 The computation lives in ``libgnf4.so`` (hand-written CUDA for sm_100a, C ABI
 in ``include/gnf4.h``); this package holds the in-tree build script and a thin
-torch-facing binding. Importing it without the built library raises.
+torch-facing binding. The binding loads the library on first use and raises if
+it is missing -- there is no fallback implementation.
 """
-from .api import (  # noqa: F401
-    quantize_nf4,
-    quantize_mxfp4,
-    grouped_gemm,
-    grouped_gemm_nf4,
-    grouped_gemm_mxfp4,
-    launches_per_call,
-    version,
-)
-from ._lib import Gnf4Error, GNF4_CHECK, GNF4_FORCE_DECODE, GNF4_FORCE_PREFILL  # noqa: F401
+_API = ("quantize_nf4", "quantize_mxfp4", "grouped_gemm", "grouped_gemm_nf4", "grouped_gemm_mxfp4",
+        "launches_per_call", "device_status", "version")
+_LIB = ("Gnf4Error", "GNF4_CHECK", "GNF4_FORCE_DECODE", "GNF4_FORCE_PREFILL")
+
+__all__ = list(_API + _LIB)
+
+
+def __getattr__(name):
+    # load libgnf4.so only when the binding is used, so that the build script
+    # (a submodule of this package) can run before the library exists
+    if name in _API:
+        from . import api
+        return getattr(api, name)
+    if name in _LIB:
+        from . import _lib
+        return getattr(_lib, name)
+    raise AttributeError(name)

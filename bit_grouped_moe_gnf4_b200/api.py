@@ -114,6 +114,11 @@ def grouped_gemm_mxfp4(x, W, scales, expert_offsets, **kw):
     return grouped_gemm("mxfp4", x, W, scales, expert_offsets, **kw)
 
 
+def device_status(stream=None) -> None:
+    """Synchronise the stream; raise if a kernel gave up waiting on a barrier."""
+    check(lib.gnf4_device_status(_stream(stream)), "gnf4_device_status")
+
+
 def launches_per_call(R: int, flags: int = 0) -> int:
     return lib.gnf4_grouped_gemm_launches(R, flags)
 

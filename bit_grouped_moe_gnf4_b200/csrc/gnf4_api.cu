@@ -149,6 +149,7 @@ static gnf4_status grouped(int fmt, const void* x, const uint8_t* W, const void*
         return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K, N, T_in and T_out must fit in int32");
     if (!row_token && T_in < R) return fail(GNF4_ERR_INVALID_ARG, "row_token is NULL but T_in < R");
     if (!row_dest && T_out < R) return fail(GNF4_ERR_INVALID_ARG, "row_dest is NULL but T_out < R");
+    if (R > 0 && (T_in == 0 || T_out == 0)) return fail(GNF4_ERR_INVALID_ARG, "R > 0 needs T_in, T_out >= 1");
     if (!aligned16(x) || !aligned16(W) || !aligned16(out))
         return fail(GNF4_ERR_MISALIGNED, "x, W and out must be 16-byte aligned");
     if (!is_device_ptr(x) || !is_device_ptr(W) || !is_device_ptr(scales) || !is_device_ptr(offsets) ||
@@ -202,7 +203,7 @@ static gnf4_status grouped(int fmt, const void* x, const uint8_t* W, const void*
     if (split < INT_MAX && R > split) {
         a.m_lo = split + 1;
         a.m_hi = INT_MAX;
-        cudaError_t e = launch_prefill_band(fmt, a, s);
+        cudaError_t e = launch_prefill_band(fmt, a, T_in, s);
         if (e != cudaSuccess) return cuda_fail(e, "prefill band launch");
     }
 #endif
@@ -251,6 +252,20 @@ gnf4_status gnf4_grouped_gemm_mxfp4(const void* x, const uint8_t* W, const uint8
                                     void* out, int flags, void* stream) {
     return grouped(FMT_MXFP4, x, W, scales, expert_offsets, row_token, row_weight, row_dest, E,
                    N, K, R, T_in, T_out, out, flags, stream);
+}
+
+gnf4_status gnf4_device_status(void* stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    cudaError_t e1 = cudaSuccess, e2 = cudaSuccess;
+    const unsigned d = take_decode_error(&e1), pr = take_prefill_error(&e2);
+    if (e1 != cudaSuccess) return cuda_fail(e1, "read device status");
+    if (e2 != cudaSuccess) return cuda_fail(e2, "read device status");
+    if (d | pr)
+        return fail(GNF4_ERR_DEVICE_STATUS, "a kernel gave up waiting on a barrier (decode 0x%x, prefill 0x%x)",
+                    d, pr);
+    return GNF4_OK;
 }
 
 int gnf4_grouped_gemm_launches(int64_t R, int flags) {

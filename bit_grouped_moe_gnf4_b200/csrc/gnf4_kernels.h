@@ -19,12 +19,17 @@ cudaError_t launch_decode_band(int fmt, const GroupedArgs& a, cudaStream_t s);
 
 // Prefill band: tcgen05 MMAs into tensor memory with the per-block fp32
 // rescale outside the MMA. Takes the groups with a.m_lo <= m <= a.m_hi.
-cudaError_t launch_prefill_band(int fmt, const GroupedArgs& a, cudaStream_t s);
+cudaError_t launch_prefill_band(int fmt, const GroupedArgs& a, int64_t T_in, cudaStream_t s);
 
 // Device-side validation of the routing metadata; writes a status word.
 cudaError_t launch_check_routing(const GroupedArgs& a, int64_t T_in, int64_t T_out,
                                  unsigned* status_out, cudaStream_t s);
 
 int device_sm_count();
+
+// Read and clear the error word a band's kernels set when they give up waiting
+// on a barrier (synchronous; 0 = no event). Returns a CUDA error through *err.
+unsigned take_decode_error(cudaError_t* err);
+unsigned take_prefill_error(cudaError_t* err);
 
 }  // namespace gnf4

@@ -1,0 +1,583 @@
+// Prefill band of the grouped 4-bit GEMM: groups with many routed rows, where
+// the work is a dense contraction and runs on the 5th-generation tensor cores
+// (tcgen05, accumulators in tensor memory). The M-tile path of the solution
+// page "How do I run a grouped GEMM directly on NF4 packed MoE expert
+// weights, without dequantizing to bf16 first?" ("Supported scope": larger
+// groups take the M-tile path), redesigned for sm_100a.
+//
+// Tile = 128 weight rows (the MMA's M side, one tensor-memory lane each) x up
+// to 128 routed rows of one expert (the N side), all of K. Persistent CTAs walk
+// the tiles of every expert in the band, computed on the device from the
+// expert offsets. Roles (16 warps):
+//   warp 0      tensor-memory owner and MMA issuer (one thread)
+//   warps 1-3   activation loaders: TMA tile loads of contiguous rows, or
+//               16-byte cp.async of the rows named by row_token, both into the
+//               128B-swizzled K-major layout
+//   warps 4-7   decoders: one weight row per thread; packed bytes straight
+//               from HBM to registers, nibbles -> bf16 by byte permutes,
+//               written to shared memory in the 128B-swizzled K-major layout
+//   warps 8-15  rescale epilogue: per scale block, read the block's fp32 sums
+//               from tensor memory, multiply by the block scale and add into
+//               fp32 running sums held in registers; at the end of a tile,
+//               weight, round to bf16 and store (scatter) the outputs
+// The MMA chain of each scale block (64 K for NF4, 32 K for MXFP4) goes to
+// one of four tensor-memory buffers, so the scale is applied in fp32 outside
+// the MMA while the tensor core fills the next buffers.
+//
+// Every wait on a barrier is bounded: after ~2^32 cycles without progress the
+// CTA records an error in g_prefill_error, stops its roles and returns.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cstdint>
+
+#include "gnf4_common.cuh"
+#include "gnf4_kernels.h"
+
+namespace gnf4 {
+
+__device__ unsigned g_prefill_error;
+
+namespace pf {
+
+constexpr int kThreads = 512;
+constexpr int kBM = 128;             // weight rows per tile
+constexpr int kBNMax = 128;          // routed rows per tile (MMA N)
+constexpr int kStages = 5;
+constexpr int kAccBufs = 4;          // tensor-memory block accumulators of kBNMax columns
+constexpr int kKStage = 64;          // K per pipeline stage (one 128-byte swizzle row of bf16)
+constexpr int kAStageBytes = kBM * 128;
+constexpr int kBStageBytes = kBNMax * 128;
+constexpr int kMaxExperts = 2048;
+constexpr int kPrefetch = 4;         // packed-weight stages held ahead in decoder registers
+constexpr long long kTimeoutCycles = 1LL << 32;
+
+// shared memory map (offsets from a 1024-aligned base)
+constexpr int kOffA = 0;
+constexpr int kOffB = kOffA + kStages * kAStageBytes;
+constexpr int kOffBar = kOffB + kStages * kBStageBytes;
+constexpr int kNumBars = 3 * kStages + 2 * kAccBufs;
+constexpr int kOffTmem = kOffBar + kNumBars * 8;
+constexpr int kOffAbort = kOffTmem + 4;
+constexpr int kOffList = kOffTmem + 16;                       // int[kMaxExperts] experts of the band
+constexpr int kOffCum = kOffList + kMaxExperts * 4;           // int[kMaxExperts+1] tile prefix
+constexpr int kOffCount = kOffCum + (kMaxExperts + 1) * 4;
+constexpr int kSmemBytes = kOffCount + 16 + 1024;             // + alignment slack
+
+struct Tile {
+    int e;          // expert
+    int64_t r0;     // first routed row of the tile
+    int cnt;        // routed rows in the tile (<= kBNMax)
+    int bn;         // MMA N: cnt rounded up to 16
+    int n0;         // first weight row
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Bounded wait; on timeout (or when another role already gave up) sets the
+// CTA's abort flag and returns false.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > kTimeoutCycles) {
+            *abort_flag = 1;
+            atomicOr(&g_prefill_error, 1u);
+            return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// UMMA shared-memory descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+    uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;                 // leading byte offset (unused for swizzled K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;       // stride byte offset
+    d |= (uint64_t)1 << 46;                 // descriptor version
+    d |= (uint64_t)2 << 61;                 // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 D, both K-major, M = 128.
+__device__ __forceinline__ uint32_t idesc_bf16(int n) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tma_tile_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// acc[0..1] += v[0..1] * s, as one packed fp32x2 FMA
+__device__ __forceinline__ void ffma2(float& a0, float& a1, uint32_t v0, uint32_t v1, float s) {
+    uint64_t acc = ((uint64_t)__float_as_uint(a1) << 32) | __float_as_uint(a0);
+    const uint64_t vv = ((uint64_t)v1 << 32) | v0;
+    const uint64_t ss = ((uint64_t)__float_as_uint(s) << 32) | __float_as_uint(s);
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(vv), "l"(ss));
+    a0 = __uint_as_float((uint32_t)acc);
+    a1 = __uint_as_float((uint32_t)(acc >> 32));
+}
+
+struct Sched {
+    const int* list;
+    const int* cum;
+    int count;
+    int total;
+};
+
+__device__ __forceinline__ Tile tile_at(const GroupedArgs& p, const Sched& s, int t, int nnt) {
+    // expert i of the band with cum[i] <= t < cum[i+1]
+    int lo = 0, hi = s.count - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s.cum[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    Tile tl;
+    tl.e = s.list[lo];
+    const int local = t - s.cum[lo];
+    const int64_t base = p.offsets[tl.e];
+    const int m = (int)(p.offsets[tl.e + 1] - base);
+    const int ntt = (m + kBNMax - 1) / kBNMax;
+    const int tpt = (m + ntt - 1) / ntt;
+    const int tt = local / nnt;
+    tl.n0 = (local % nnt) * kBM;
+    tl.r0 = base + (int64_t)tt * tpt;
+    tl.cnt = min(tpt, m - tt * tpt);
+    tl.bn = (tl.cnt + 15) & ~15;
+    return tl;
+}
+
+}  // namespace pf
+
+template <int FMT>
+__global__ void __launch_bounds__(pf::kThreads, 1)
+prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xmap, const int gather) {
+    using namespace pf;
+    constexpr int SB = (FMT == FMT_NF4) ? 64 : 32;      // scale block
+    constexpr int SBPS = kKStage / SB;                  // scale blocks per stage (1 or 2)
+    constexpr int K16PSB = SB / 16;                     // k16 MMAs per scale block
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar_afull = sbase + kOffBar;                  // [kStages] decoders -> MMA
+    const uint32_t bar_bfull = bar_afull + 8 * kStages;          // [kStages] TMA -> MMA
+    const uint32_t bar_empty = bar_bfull + 8 * kStages;          // [kStages] MMA -> producers
+    const uint32_t bar_accfull = bar_empty + 8 * kStages;        // [kAccBufs] MMA -> epilogue
+    const uint32_t bar_accempty = bar_accfull + 8 * kAccBufs;    // [kAccBufs] epilogue -> MMA
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffTmem);
+    int* s_list = reinterpret_cast<int*>(smem + kOffList);
+    int* s_cum = reinterpret_cast<int*>(smem + kOffCum);
+    int* s_count = reinterpret_cast<int*>(smem + kOffCount);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nnt = (p.N + kBM - 1) / kBM;
+    const int nst = p.K / kKStage + ((p.K % kKStage) ? 1 : 0);   // stages per tile (last may be half, MXFP4)
+
+    // ---- set-up: band experts and tile prefix (warp 2), barriers (warp 3), tensor memory (warp 0)
+    if (warp == 2) {
+        int count = 0, tiles = 0;
+        for (int e0 = 0; e0 < p.E; e0 += 32) {
+            const int e = e0 + lane;
+            int m = 0;
+            bool act = false;
+            if (e < p.E) {
+                m = (int)(p.offsets[e + 1] - p.offsets[e]);
+                act = (m >= p.m_lo) && (m <= p.m_hi);
+            }
+            const int nt = act ? ((m + kBNMax - 1) / kBNMax) * nnt : 0;
+            // inclusive scan of tile counts across the warp
+            int inc = nt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += v;
+            }
+            const unsigned bal = __ballot_sync(0xffffffffu, act);
+            if (act) {
+                const int idx = count + __popc(bal & ((1u << lane) - 1u));
+                s_list[idx] = e;
+                s_cum[idx] = tiles + inc - nt;
+            }
+            count += __popc(bal);
+            tiles += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        if (lane == 0) {
+            s_cum[count] = tiles;
+            s_count[0] = count;
+            s_count[1] = tiles;
+        }
+    } else if (warp == 3 && lane == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(bar_afull + 8 * i, 128);
+            mbar_init(bar_bfull + 8 * i, gather ? 96 : 1);
+            mbar_init(bar_empty + 8 * i, 1);
+        }
+        for (int i = 0; i < kAccBufs; ++i) {
+            mbar_init(bar_accfull + 8 * i, 1);
+            mbar_init(bar_accempty + 8 * i, 8);
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    } else if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;"
+                     ::"r"(smem_u32(tmem_slot)) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    Sched sch{s_list, s_cum, s_count[0], s_count[1]};
+
+    if (warp == 0) {
+        // ================= MMA issuer =================
+        if (lane == 0) {
+            uint32_t stage_ctr = 0, acc_ctr = 0;
+            for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
+                const Tile tl = tile_at(p, sch, t, nnt);
+                const uint32_t idesc = idesc_bf16(tl.bn);
+                for (int s = 0; s < nst; ++s, ++stage_ctr) {
+                    const uint32_t slot = stage_ctr % kStages, ph = (stage_ctr / kStages) & 1u;
+                    if (!mbar_wait(bar_afull + 8 * slot, ph, abort_flag)) goto mma_done;
+                    if (!mbar_wait(bar_bfull + 8 * slot, ph, abort_flag)) goto mma_done;
+                    tc_fence_after();
+                    const uint32_t a_addr = sbase + kOffA + slot * kAStageBytes;
+                    const uint32_t b_addr = sbase + kOffB + slot * kBStageBytes;
+                    const int nsb = min(SBPS, (p.K - s * kKStage) / SB);
+                    for (int sb = 0; sb < nsb; ++sb, ++acc_ctr) {
+                        const uint32_t buf = acc_ctr % kAccBufs, aph = ((acc_ctr / kAccBufs) & 1u) ^ 1u;
+                        if (!mbar_wait(bar_accempty + 8 * buf, aph, abort_flag)) goto mma_done;
+                        tc_fence_after();
+#pragma unroll
+                        for (int q = 0; q < K16PSB; ++q) {
+                            const uint32_t koff = (uint32_t)(sb * K16PSB + q) * 32u;
+                            mma_bf16(tmem + buf * kBNMax, desc_sw128(a_addr + koff), desc_sw128(b_addr + koff),
+                                     idesc, q > 0 ? 1u : 0u);
+                        }
+                        mma_commit(bar_accfull + 8 * buf);
+                    }
+                    mma_commit(bar_empty + 8 * slot);
+                }
+            }
+        }
+    mma_done:
+        __syncwarp();
+    } else if (warp >= 1 && warp <= 3) {
+        // ================= activation loaders =================
+        if (!gather) {
+            // contiguous routed rows: TMA tile loads, 16 rows x 64 K per box, 128B-swizzled
+            if (warp == 1 && lane == 0) {
+                uint32_t stage_ctr = 0;
+                for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
+                    const Tile tl = tile_at(p, sch, t, nnt);
+                    for (int s = 0; s < nst; ++s, ++stage_ctr) {
+                        const uint32_t slot = stage_ctr % kStages, ph = ((stage_ctr / kStages) & 1u) ^ 1u;
+                        if (!mbar_wait(bar_empty + 8 * slot, ph, abort_flag)) goto load_done;
+                        const uint32_t full = bar_bfull + 8 * slot;
+                        const uint32_t dst = sbase + kOffB + slot * kBStageBytes;
+                        mbar_arrive_tx(full, (uint32_t)tl.bn * 128u);
+                        for (int j = 0; j < tl.bn; j += 16)
+                            tma_tile_2d(dst + j * 128, &xmap, s * kKStage, (int)(tl.r0 + j), full);
+                    }
+                }
+            }
+        } else {
+            // gathered rows (row_token): 16-byte cp.async per (row, chunk), written in the
+            // 128B-swizzled layout; each thread completes its copies of a stage, makes them
+            // visible to the tensor core (proxy fence) and arrives, two stages behind issue
+            const int l = threadIdx.x - 32;              // 0..95
+            const int c = l & 7;                         // 16-byte chunk of the 128-byte row
+            const int rb = l >> 3;                       // first row: rb, rb + 12, ...
+            constexpr int kRowsPer = (kBNMax + 11) / 12;   // rows per thread
+            uint32_t stage_ctr = 0;
+            int npend = 0;
+            uint32_t pend0 = 0, pend1 = 0;
+            for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
+                const Tile tl = tile_at(p, sch, t, nnt);
+                int tok[kRowsPer];
+#pragma unroll
+                for (int j = 0; j < kRowsPer; ++j) {
+                    const int row = rb + 12 * j;
+                    tok[j] = (row < tl.cnt) ? __ldg(p.row_token + tl.r0 + row) : -1;
+                }
+                for (int s = 0; s < nst; ++s, ++stage_ctr) {
+                    const uint32_t slot = stage_ctr % kStages, ph = ((stage_ctr / kStages) & 1u) ^ 1u;
+                    if (!mbar_wait(bar_empty + 8 * slot, ph, abort_flag)) goto load_done;
+                    const uint32_t dst = sbase + kOffB + slot * kBStageBytes;
+                    const int kx = s * kKStage + c * 8;
+                    if (kx < p.K) {
+#pragma unroll
+                        for (int j = 0; j < kRowsPer; ++j) {
+                            const int row = rb + 12 * j;
+                            if (tok[j] >= 0)
+                                cp_async16(dst + row * 128 + ((c ^ (row & 7)) << 4),
+                                           p.x + (int64_t)tok[j] * p.K + kx);
+                        }
+                    }
+                    cp_async_commit();
+                    if (npend == 0) { pend0 = slot; npend = 1; }
+                    else if (npend == 1) { pend1 = slot; npend = 2; }
+                    if (npend == 2) {
+                        cp_async_wait<1>();
+                        fence_proxy_async();
+                        mbar_arrive(bar_bfull + 8 * pend0);
+                        pend0 = pend1;
+                        npend = 1;
+                    }
+                }
+            }
+            cp_async_wait<0>();
+            fence_proxy_async();
+            if (npend == 1) mbar_arrive(bar_bfull + 8 * pend0);
+        }
+    load_done:
+        cp_async_wait<0>();
+        __syncwarp();
+    } else if (warp >= 4 && warp < 8) {
+        // ================= decoders: one weight row per thread =================
+        const int i = threadIdx.x - 128;                   // tile row
+        uint32_t stage_ctr = 0;
+        const int64_t rowbytes = p.K >> 1;
+        for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
+            const Tile tl = tile_at(p, sch, t, nnt);
+            const int n = tl.n0 + i;
+            const bool valid = n < p.N;
+            const uint8_t* wrow = p.W + ((int64_t)tl.e * p.N + (valid ? n : 0)) * rowbytes;
+            uint4 pre[kPrefetch][2];
+#pragma unroll
+            for (int q = 0; q < kPrefetch; ++q) {
+                pre[q][0] = pre[q][1] = make_uint4(0u, 0u, 0u, 0u);
+                if (valid && q < nst) {
+                    const uint4* src = reinterpret_cast<const uint4*>(wrow + q * 32);
+                    pre[q][0] = __ldg(src);
+                    if (q * kKStage + 32 < p.K) pre[q][1] = __ldg(src + 1);
+                }
+            }
+            for (int s0 = 0; s0 < nst; s0 += kPrefetch) {
+#pragma unroll
+                for (int q = 0; q < kPrefetch; ++q) {
+                    const int s = s0 + q;
+                    if (s < nst) {
+                        const uint32_t slot = stage_ctr % kStages, ph = ((stage_ctr / kStages) & 1u) ^ 1u;
+                        ++stage_ctr;
+                        const uint4 c0 = pre[q][0], c1 = pre[q][1];
+                        // refill this slot with stage s + kPrefetch
+                        const int sn = s + kPrefetch;
+                        if (valid && sn < nst) {
+                            const uint4* src = reinterpret_cast<const uint4*>(wrow + sn * 32);
+                            pre[q][0] = __ldg(src);
+                            if (sn * kKStage + 32 < p.K) pre[q][1] = __ldg(src + 1);
+                        }
+                        if (!mbar_wait(bar_empty + 8 * slot, ph, abort_flag)) goto dec_done;
+                        uint8_t* arow = smem + kOffA + slot * kAStageBytes + i * 128;
+                        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {          // 16-byte chunk c: K elements 8c .. 8c+7
+                            uint32_t o[4];
+                            decode_word<FMT>(words[c], p.lut, o);
+                            *reinterpret_cast<uint4*>(arow + ((c ^ (i & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                        }
+                        fence_proxy_async();
+                        mbar_arrive(bar_afull + 8 * slot);
+                    }
+                }
+            }
+        }
+    dec_done:;
+    } else if (warp >= 8) {
+        // ================= rescale epilogue =================
+        const int q4 = warp & 3;                      // tensor-memory lane quadrant
+        const int half = (warp - 8) >> 2;             // which 16-column chunks: half, half+2, ...
+        const int i = q4 * 32 + lane;                 // tile row = tensor-memory lane
+        const int nsbk = p.K / SB;                    // scale blocks per row
+        uint32_t acc_ctr = 0;
+        float acc[kBNMax / 32][16];
+        for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
+            const Tile tl = tile_at(p, sch, t, nnt);
+            const int n = tl.n0 + i;
+            const bool valid = n < p.N;
+            const int64_t srow = ((int64_t)tl.e * p.N + (valid ? n : 0)) * nsbk;
+            const int nck = tl.bn >> 4;
+#pragma unroll
+            for (int j = 0; j < kBNMax / 32; ++j)
+#pragma unroll
+                for (int c = 0; c < 16; ++c) acc[j][c] = 0.f;
+            float scale_next = load_scale<FMT>(p.scales, srow);
+            for (int b = 0; b < nsbk; ++b, ++acc_ctr) {
+                const float sc = scale_next;
+                if (b + 1 < nsbk) scale_next = load_scale<FMT>(p.scales, srow + b + 1);
+                const uint32_t buf = acc_ctr % kAccBufs, ph = (acc_ctr / kAccBufs) & 1u;
+                if (!mbar_wait(bar_accfull + 8 * buf, ph, abort_flag)) goto epi_done;
+                tc_fence_after();
+                const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16) + buf * kBNMax;
+#pragma unroll
+                for (int j = 0; j < kBNMax / 32; j += 2) {
+                    const int c0 = half + 2 * j, c1 = half + 2 * (j + 1);
+                    uint32_t v0[16], v1[16];
+                    if (c0 < nck) tmem_ld16(taddr + c0 * 16, v0);
+                    if (c1 < nck) tmem_ld16(taddr + c1 * 16, v1);
+                    tmem_wait_ld();
+                    if (c0 < nck) {
+#pragma unroll
+                        for (int c = 0; c < 16; c += 2) ffma2(acc[j][c], acc[j][c + 1], v0[c], v0[c + 1], sc);
+                    }
+                    if (c1 < nck) {
+#pragma unroll
+                        for (int c = 0; c < 16; c += 2) ffma2(acc[j + 1][c], acc[j + 1][c + 1], v1[c], v1[c + 1], sc);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_accempty + 8 * buf);
+            }
+            // outputs of this tile: row n, routed rows r0 .. r0+cnt-1
+            if (valid) {
+#pragma unroll
+                for (int j = 0; j < kBNMax / 32; ++j) {
+                    const int c0 = half + 2 * j;
+                    if (c0 < nck) {
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) {
+                            const int slot = c0 * 16 + c;
+                            if (slot < tl.cnt) {
+                                const int64_t r = tl.r0 + slot;
+                                float v = acc[j][c];
+                                if (p.row_weight) v *= __ldg(p.row_weight + r);
+                                const int64_t dst = p.row_dest ? (int64_t)__ldg(p.row_dest + r) : r;
+                                p.out[dst * p.N + n] = f32_to_bf16_rne(v);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+    epi_done:;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+template <int FMT>
+static cudaError_t launch_pf(const GroupedArgs& a, int64_t T_in, cudaStream_t s) {
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e = cudaFuncSetAttribute(prefill_band_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             pf::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    auto enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    const int gather = a.row_token != nullptr;
+    CUtensorMap map;
+    cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)T_in};
+    cuuint64_t strides[1] = {(cuuint64_t)a.K * 2};
+    cuuint32_t box[2] = {64, 16};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.x), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    const int grid = device_sm_count();
+    prefill_band_kernel<FMT><<<grid, pf::kThreads, pf::kSmemBytes, s>>>(a, map, gather);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_band(int fmt, const GroupedArgs& a, int64_t T_in, cudaStream_t s) {
+    return fmt == FMT_NF4 ? launch_pf<FMT_NF4>(a, T_in, s) : launch_pf<FMT_MXFP4>(a, T_in, s);
+}
+
+unsigned take_prefill_error(cudaError_t* err) {
+    unsigned v = 0;
+    const unsigned zero = 0;
+    *err = cudaMemcpyFromSymbol(&v, g_prefill_error, sizeof(unsigned));
+    if (*err == cudaSuccess && v) *err = cudaMemcpyToSymbol(g_prefill_error, &zero, sizeof(unsigned));
+    return v;
+}
+
+}  // namespace gnf4

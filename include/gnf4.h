@@ -135,6 +135,15 @@ gnf4_status gnf4_grouped_gemm_mxfp4(const void* x, const uint8_t* W, const uint8
                                     int flags, void* stream);
 
 /*
+ * Synchronise `stream` and report whether any grouped GEMM kernel since the last
+ * call gave up waiting on one of its internal barriers (every such wait is
+ * bounded, so a kernel never hangs; it stops, records the event and returns).
+ * Returns GNF4_ERR_DEVICE_STATUS (and clears the record) if one did, GNF4_ERR_CUDA
+ * if the stream reports an error, GNF4_OK otherwise.
+ */
+gnf4_status gnf4_device_status(void* stream);
+
+/*
  * How many kernels one grouped GEMM call with R routed rows and these flags
  * launches (0 when R == 0; GNF4_CHECK adds one). Host-only, no CUDA call.
  */

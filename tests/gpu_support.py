@@ -94,7 +94,7 @@ def run_gemm(fmt, x_bits, Wd, Sd, offsets, row_token=None, row_weight=None, row_
         out = torch.empty((R if T_out is None else T_out, Wd.shape[1]), dtype=torch.bfloat16, device="cuda")
     g.grouped_gemm(fmt, x, Wd, Sd, to_dev(np.asarray(offsets, np.int64)), row_token=to_dev(row_token),
                    row_weight=to_dev(row_weight), row_dest=to_dev(row_dest), out=out, flags=flags, R=R)
-    torch.cuda.synchronize()
+    g.device_status()          # synchronises; raises if a kernel gave up waiting on a barrier
     return bf16_host_bits(out)
 
 
