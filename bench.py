@@ -309,24 +309,29 @@ def run_ours(args, wl):
 
     fn = g.grouped_gemm
 
-    def one_call(c, copy, ev=None):
+    def one_call(c, copy):
         W, S = stacks[c["proj"].name][copy]
         d = c["d"]
-        if ev is not None:
-            ev[0].record(stream)
         fn(wl.fmt, d["x"], W, S, d["off"], row_token=d["tok"], row_weight=d["wt"], row_dest=d["dst"],
-           out=c["out"], R=c["b"].R, stream=stream)
-        if ev is not None:
-            ev[1].record(stream)
+           out=c["out"], R=c["b"].R, stream=torch.cuda.current_stream())
 
-    def step(i, evs=None):
-        copy = i % ncopies
-        for j, c in enumerate(prepared):
-            one_call(c, copy, None if evs is None else evs[j])
-
-    # warm-up
+    # warm-up through the public call
     for i in range(args.warmup):
-        step(i)
+        for c in prepared:
+            one_call(c, i % ncopies)
+    torch.cuda.synchronize()
+    g.device_status()
+
+    # each (call, weight copy) captured once as a CUDA graph, so the timed region
+    # measures device time, not the host's per-call argument checks
+    graphs = {}
+    cap = torch.cuda.Stream()
+    for j, c in enumerate(prepared):
+        for copy in range(ncopies):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=cap, capture_error_mode="thread_local"):
+                one_call(c, copy)
+            graphs[(j, copy)] = gr
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -341,16 +346,23 @@ def run_ours(args, wl):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    torch.cuda._sleep(int(2e6))          # let the host queue the whole timed region ahead of the GPU
     t_start.record(stream)
     for i in range(args.steps):
-        step(args.warmup + i, ev_calls[i])
+        copy = (args.warmup + i) % ncopies
+        for j in range(len(prepared)):
+            ev_calls[i][j][0].record(stream)
+            graphs[(j, copy)].replay()
+            ev_calls[i][j][1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
+    g.device_status()
     total_ms = t_start.elapsed_time(t_end)
     call_ms = np.array([[s.elapsed_time(e) for (s, e) in row] for row in ev_calls])  # [steps, calls]
+    del graphs
 
     # end-to-end: host buffers in, result back, through the same public call
     e2e_steps = max(3, min(args.steps, 10))

@@ -359,9 +359,13 @@ static cudaError_t launch_db(const GroupedArgs& a, cudaStream_t s) {
     if (nst < 2) return cudaErrorInvalidValue;
     plan.nstages = nst;
     const int smem = nst * plan.stage_bytes + fixed;
-    cudaError_t e = cudaFuncSetAttribute(decode_band_kernel<FMT, GMAX>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
+    static int smem_set = 0;                 // largest dynamic shared memory opted in so far
+    if (smem > smem_set) {
+        cudaError_t e = cudaFuncSetAttribute(decode_band_kernel<FMT, GMAX>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        smem_set = smem;
+    }
     const int64_t groups_max = a.R < (int64_t)a.E ? a.R : (int64_t)a.E;
     const int64_t items_max = groups_max * (a.N / 16);
     int64_t grid = (int64_t)device_sm_count() * per_sm;
