@@ -145,8 +145,8 @@ static gnf4_status grouped(int fmt, const void* x, const uint8_t* W, const void*
     if (K % kmul) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K must be a multiple of %lld", (long long)kmul);
     if (N % 16) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "N must be a multiple of 16");
     if (E > 2048) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "at most 2048 experts");
-    if (K > (int64_t)INT_MAX / 2 || N > (int64_t)INT_MAX || T_in > INT_MAX || T_out > INT_MAX)
-        return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K, N, T_in and T_out must fit in int32");
+    if (K > (int64_t)INT_MAX / 2 || E * N > (int64_t)INT_MAX || T_in > INT_MAX || T_out > INT_MAX)
+        return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K, E*N, T_in and T_out must fit in int32");
     if (!row_token && T_in < R) return fail(GNF4_ERR_INVALID_ARG, "row_token is NULL but T_in < R");
     if (!row_dest && T_out < R) return fail(GNF4_ERR_INVALID_ARG, "row_dest is NULL but T_out < R");
     if (R > 0 && (T_in == 0 || T_out == 0)) return fail(GNF4_ERR_INVALID_ARG, "R > 0 needs T_in, T_out >= 1");

@@ -117,4 +117,77 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+
+// ---------------------------------------------------------------------------
+// mbarrier helpers shared by the kernels that pipeline through shared memory
+// ---------------------------------------------------------------------------
+constexpr long long kWaitTimeoutCycles = 1LL << 32;   // ~2 s at B200 clocks
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// One bounded attempt: the thread may sleep up to ~hint_ns inside the instruction.
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(bar), "r"(parity), "r"(hint_ns) : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase with parity `parity` to complete. Bounded: after
+// kWaitTimeoutCycles without completion (or as soon as another warp of the CTA
+// has given up) it records `code` in *err, raises the CTA's abort flag and
+// returns false. The clock and the flag are polled only every 8th attempt.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                  unsigned* err, unsigned code) {
+    if (mbar_try_wait(bar, parity, 0u)) return true;
+    const long long t0 = clock64();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity, 2000u)) return true;
+        if ((it & 7u) == 0u) {
+            if (*abort_flag) return false;
+            if (clock64() - t0 > kWaitTimeoutCycles) {
+                *abort_flag = 1;
+                atomicOr(err, code);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// bf16 bit pattern of one 4-bit code (NF4: 16-entry table; MXFP4: magnitude
+// table of codes 0..7 plus the sign bit 3)
+template <int FMT>
+__device__ __forceinline__ uint32_t code_bf16(uint32_t c, const LutPlanes& L) {
+    if constexpr (FMT == FMT_NF4) {
+        const uint32_t sh = 8u * (c & 3u);
+        return (((L.hi[c >> 2] >> sh) & 0xFFu) << 8) | ((L.lo[c >> 2] >> sh) & 0xFFu);
+    } else {
+        const uint32_t m = c & 7u, sh = 8u * (m & 3u);
+        return (((L.hi[m >> 2] >> sh) & 0xFFu) << 8) | ((L.lo[m >> 2] >> sh) & 0xFFu) | ((c & 8u) << 12);
+    }
+}
+
+// bf16x2 word for one packed byte: the lower-k element in the low 16 bits
+// (NF4: the high nibble comes first; MXFP4: the low nibble comes first)
+template <int FMT>
+__device__ __forceinline__ uint32_t byte_bf16x2(uint32_t b, const LutPlanes& L) {
+    const uint32_t first = (FMT == FMT_NF4) ? (b >> 4) : (b & 15u);
+    const uint32_t second = (FMT == FMT_NF4) ? (b & 15u) : (b >> 4);
+    return code_bf16<FMT>(first, L) | (code_bf16<FMT>(second, L) << 16);
+}
+
 }  // namespace gnf4

@@ -4,20 +4,24 @@
 // without dequantizing to bf16 first?", "Supported scope": one-token groups
 // take the GEMV path).
 //
-// Work item = (active expert, 16 weight rows); each CTA takes a contiguous run
-// of items (consecutive items share an expert, so its activation rows stay in
-// L1). One producer warp streams every item's packed rows into a ring of
-// shared-memory stages with 1-D bulk copies (cp.async.bulk, completion counted
-// on an mbarrier), several items ahead of the consumers, so HBM sees many
-// bytes in flight per SM regardless of what the consumers are doing. Eight
-// consumer warps split each stage's K range; each decodes the nibbles with byte
-// permutes (tables in registers) and multiplies through warp-level bf16 MMAs
-// with the 16 weight rows as the M side and up to 8 routed rows per MMA as the
-// N side. Every MMA chain covers exactly one scale block (64 K for NF4, 32 K for
-// MXFP4), so the block sum leaves the tensor core in fp32 and is scaled and
-// accumulated in fp32 outside it. The 8 warp partials are summed in a fixed
-// order through shared memory (deterministic), weighted, rounded to bf16 and
-// stored at the destination rows.
+// One persistent CTA per SM takes a contiguous run of work items; an item is
+// (active expert, 16 weight rows). The CTA's 16 consumer warps form 4 groups of
+// 4 warps; group q takes items q, q+4, ... of the run. A producer warp (one
+// lane per group) streams each item's packed rows, one K chunk of 512 at a
+// time, into the group's ring of shared-memory stages with 1-D bulk copies
+// (cp.async.bulk, completion counted on an mbarrier), several chunks ahead, so
+// HBM always has many bytes in flight per SM.
+//
+// The 4 warps of a group split each chunk's scale blocks. Nibble pairs are
+// decoded by a table in shared memory that maps each packed byte to its two
+// bf16 values (one bf16x2 word), replicated per lane so that 32 lookups never
+// conflict; a byte permute forms the lookup address. The products run on
+// warp-level bf16 MMAs with the 16 weight rows as the M side and up to 8 routed
+// rows per MMA as the N side. Every MMA chain covers exactly one scale block
+// (64 K for NF4, 32 K for MXFP4), so the block sum leaves the tensor core in
+// fp32 and is scaled and accumulated in fp32 outside it. After the last chunk
+// the group's 4 partial sums are added in a fixed order through shared memory
+// (deterministic), weighted, rounded to bf16 and stored at the destination rows.
 //
 // MMA k-slot mapping: in m16n8k16, lane (g, t) supplies k-slots 2t, 2t+1,
 // 2t+8, 2t+9 of both operands. They are mapped to the four consecutive K
@@ -36,45 +40,21 @@ __device__ unsigned g_decode_error;
 
 namespace db {
 
-constexpr int kConsumers = 8;                    // consumer warps
-constexpr int kThreads = (kConsumers + 1) * 32;  // + one producer warp
+constexpr int kGroups = 4;                         // item groups per CTA
+constexpr int kGroupWarps = 4;                     // consumer warps per group (split of each chunk)
+constexpr int kConsumers = kGroups * kGroupWarps;  // 16
+constexpr int kThreads = (kConsumers + 1) * 32;    // + one producer warp
 constexpr int kMaxExperts = 2048;
-constexpr int kBlocksPerStage = 32;              // scale blocks per stage (4 per consumer warp)
-constexpr long long kTimeoutCycles = 1LL << 32;
+constexpr int kChunkK = 512;                       // K per stage
+constexpr int kLutBytes = 256 * 256;               // byte value b, lane l -> offset b*256 + l*4
 
 struct Plan {
-    int kch;          // K elements per stage (a multiple of the scale block)
+    int kch;          // K elements per stage
     int nch;          // stages per item pass
     int row_stride;   // bytes per weight row in a stage (chunk bytes + 16 of padding)
     int stage_bytes;  // 16 rows
-    int nstages;
+    int nstages;      // stages per group ring
 };
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-    return ok != 0;
-}
-// bounded wait: false after ~2^32 cycles (error recorded) or once another warp gave up
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    if (mbar_try(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (true) {
-        if (mbar_try(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (clock64() - t0 > kTimeoutCycles) {
-            *abort_flag = 1;
-            atomicOr(&g_decode_error, 1u);
-            return false;
-        }
-    }
-}
 
 struct Pos {
     int item, pass, kc;
@@ -83,26 +63,32 @@ struct Pos {
 }  // namespace db
 
 template <int FMT, int GMAX>
-__global__ void __maxnreg__(112) decode_band_kernel(const GroupedArgs p, const db::Plan plan) {
+__global__ void __launch_bounds__(db::kThreads, 1) decode_band_kernel(const GroupedArgs p, const db::Plan plan) {
     using namespace db;
     constexpr int SB = (FMT == FMT_NF4) ? 64 : 32;   // K elements per scale block
     constexpr int STEPS = SB / 16;                   // k16 MMA steps per block
     constexpr int BPL = SB / 8;                      // packed bytes per lane per row per block (8 or 4)
     constexpr int XW = SB / 8;                       // bf16x2 words of x per lane per block
-    constexpr int BPW = kBlocksPerStage / kConsumers;  // blocks per consumer warp per stage (4)
+    constexpr int BPW = (kChunkK / SB) / kGroupWarps;  // blocks per warp per full chunk (2 or 4)
 
-    extern __shared__ __align__(128) uint8_t smem[];
-    // layout: [stages][16 rows][row_stride] | red[8][GMAX][32] float4 | barriers | lists
-    float4* red = reinterpret_cast<float4*>(smem + plan.nstages * plan.stage_bytes);
-    uint8_t* tail = smem + plan.nstages * plan.stage_bytes + kConsumers * GMAX * 32 * sizeof(float4);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(tail);                 // full[ns], empty[ns]
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tail + 16 * 8 * 2);
-    int* s_nact = reinterpret_cast<int*>(tail + 16 * 8 * 2 + 16);
-    int* s_active = s_nact + 4;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t* lut = smem;                                            // [256][64] words
+    uint8_t* rings = smem + kLutBytes;                              // [groups][stages][16 rows][row_stride]
+    float4* red = reinterpret_cast<float4*>(rings + kGroups * plan.nstages * plan.stage_bytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(red + kConsumers * GMAX * 32);   // full[g][s], empty[g][s]
+    int* tailw = reinterpret_cast<int*>(bars + 2 * kGroups * plan.nstages);
+    volatile int* abort_flag = tailw;
+    int* s_nact = tailw + 4;
+    int* s_active = tailw + 8;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ns = plan.nstages;
 
+    // byte -> bf16x2 table, one copy per lane
+    for (int i = threadIdx.x; i < 256 * 32; i += kThreads) {
+        const int b = i >> 5, l = i & 31;
+        *reinterpret_cast<uint32_t*>(lut + b * 256 + l * 4) = byte_bf16x2<FMT>((uint32_t)b, p.lut);
+    }
     if (warp == 0) {
         // experts of this band, in id order (every CTA derives the same list)
         int count = 0;
@@ -119,10 +105,9 @@ __global__ void __maxnreg__(112) decode_band_kernel(const GroupedArgs p, const d
         }
         if (lane == 0) s_nact[0] = count;
     } else if (warp == kConsumers && lane == 0) {
-        for (int i = 0; i < ns; ++i) {
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bars + i)) : "memory");
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bars + 16 + i)),
-                         "r"(kConsumers) : "memory");
+        for (int i = 0; i < kGroups * ns; ++i) {
+            mbar_init(smem_addr(bars + i), 1);                                 // full: producer + tx bytes
+            mbar_init(smem_addr(bars + kGroups * ns + i), kGroupWarps);        // empty: the group's warps
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -136,58 +121,64 @@ __global__ void __maxnreg__(112) decode_band_kernel(const GroupedArgs p, const d
     const int64_t rowbytes = p.K >> 1;
     const int nbk = p.K / SB;                        // scale blocks per weight row
 
-    auto item_m = [&](int item) -> int {
-        const int e = s_active[item / nt];
-        return (int)(p.offsets[e + 1] - p.offsets[e]);
-    };
     auto advance = [&](Pos q) -> Pos {
         if (++q.kc == plan.nch) {
             q.kc = 0;
-            const int npass = (item_m(q.item) + 8 * GMAX - 1) / (8 * GMAX);
-            if (++q.pass == npass) {
+            const int e = s_active[q.item / nt];
+            const int m = (int)(p.offsets[e + 1] - p.offsets[e]);
+            if (++q.pass == (m + 8 * GMAX - 1) / (8 * GMAX)) {
                 q.pass = 0;
-                ++q.item;
+                q.item += kGroups;
             }
         }
         return q;
     };
 
     if (warp == kConsumers) {
-        // ================= producer: packed rows -> shared-memory stages =================
-        if (lane == 0) {
+        // ================= producer: lane q feeds group q's ring =================
+        if (lane < kGroups) {
+            const int q = lane;
+            uint64_t* full = bars + q * ns;
+            uint64_t* empty = bars + kGroups * ns + q * ns;
+            uint8_t* ring = rings + q * ns * plan.stage_bytes;
             uint32_t ctr = 0;
-            for (Pos q{i0, 0, 0}; q.item < i1; q = advance(q), ++ctr) {
+            for (Pos ps{i0 + q, 0, 0}; ps.item < i1; ps = advance(ps), ++ctr) {
                 const uint32_t slot = ctr % ns, ph = ((ctr / ns) & 1u) ^ 1u;
-                if (!mbar_wait(smem_u32(bars + 16 + slot), ph, abort_flag)) break;
-                const int e = s_active[q.item / nt];
-                const int n0 = (q.item % nt) << 4;
-                const int kb = q.kc * plan.kch;
+                if (!mbar_wait_bounded(smem_addr(empty + slot), ph, abort_flag, &g_decode_error, 1u)) break;
+                const int e = s_active[ps.item / nt];
+                const int n0 = (ps.item % nt) << 4;
+                const int kb = ps.kc * plan.kch;
                 const uint32_t bytes = (uint32_t)(min(plan.kch, p.K - kb) >> 1);
-                const uint32_t full = smem_u32(bars + slot);
-                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full), "r"(16u * bytes)
-                             : "memory");
+                const uint32_t fb = smem_addr(full + slot);
+                mbar_arrive_tx(fb, 16u * bytes);
                 const uint8_t* src = p.W + ((int64_t)e * p.N + n0) * rowbytes + (kb >> 1);
-                const uint32_t dst = smem_u32(smem + slot * plan.stage_bytes);
+                const uint32_t dst = smem_addr(ring + slot * plan.stage_bytes);
                 for (int r = 0; r < 16; ++r)
                     asm volatile(
                         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                        ::"r"(dst + r * plan.row_stride), "l"(src + r * rowbytes), "r"(bytes), "r"(full)
+                        ::"r"(dst + r * plan.row_stride), "l"(src + r * rowbytes), "r"(bytes), "r"(fb)
                         : "memory");
             }
         }
         __syncwarp();
     } else {
         // ================= consumers =================
+        const int q = warp / kGroupWarps, gw = warp % kGroupWarps;
         const int g = lane >> 2, t = lane & 3;
+        uint64_t* full = bars + q * ns;
+        uint64_t* empty = bars + kGroups * ns + q * ns;
+        const uint8_t* ring = rings + q * ns * plan.stage_bytes;
+        float4* gred = red + q * kGroupWarps * GMAX * 32;
+        const uint32_t lane_sel = (uint32_t)lane * 4u;   // lut offset of this lane's copy
         uint32_t ctr = 0;
         float acc[GMAX][4];
         float sc0[BPW], sc1[BPW], nsc0[BPW], nsc1[BPW];
-        auto load_scales = [&](const Pos& q, float (&s0)[BPW], float (&s1)[BPW]) {
-            const int e = s_active[q.item / nt];
-            const int n0 = (q.item % nt) << 4;
-            const int nbc = min(plan.kch, p.K - q.kc * plan.kch) / SB;
-            const int b0 = warp * nbc / kConsumers, b1 = (warp + 1) * nbc / kConsumers;
-            const int64_t base0 = ((int64_t)e * p.N + n0 + g) * nbk + q.kc * (plan.kch / SB);
+        auto load_scales = [&](const Pos& ps, float (&s0)[BPW], float (&s1)[BPW]) {
+            const int e = s_active[ps.item / nt];
+            const int n0 = (ps.item % nt) << 4;
+            const int nbc = min(plan.kch, p.K - ps.kc * plan.kch) / SB;
+            const int b0 = gw * nbc / kGroupWarps, b1 = (gw + 1) * nbc / kGroupWarps;
+            const int64_t base0 = ((int64_t)e * p.N + n0 + g) * nbk + ps.kc * (plan.kch / SB);
 #pragma unroll
             for (int c = 0; c < BPW; ++c) {
                 s0[c] = s1[c] = 0.f;
@@ -197,7 +188,7 @@ __global__ void __maxnreg__(112) decode_band_kernel(const GroupedArgs p, const d
                 }
             }
         };
-        Pos cur{i0, 0, 0};
+        Pos cur{i0 + q, 0, 0};
         if (cur.item < i1) load_scales(cur, nsc0, nsc1);
         while (cur.item < i1) {
             const int e = s_active[cur.item / nt];
@@ -216,7 +207,7 @@ __global__ void __maxnreg__(112) decode_band_kernel(const GroupedArgs p, const d
             }
             const int kb = cur.kc * plan.kch;
             const int nbc = min(plan.kch, p.K - kb) / SB;
-            const int b0 = warp * nbc / kConsumers, b1 = (warp + 1) * nbc / kConsumers;
+            const int b0 = gw * nbc / kGroupWarps, b1 = (gw + 1) * nbc / kGroupWarps;
             // activation row of this lane's token column g, per 8-row group (-1: none)
             int xtk[GMAX];
 #pragma unroll
@@ -234,24 +225,25 @@ __global__ void __maxnreg__(112) decode_band_kernel(const GroupedArgs p, const d
 #pragma unroll
             for (int c = 0; c < BPW; ++c) {
 #pragma unroll
-                for (int q = 0; q < XW; ++q) xw0[c][q] = 0u;
+                for (int w = 0; w < XW; ++w) xw0[c][w] = 0u;
                 if (b0 + c < b1 && xtk[0] >= 0) {
 #pragma unroll
-                    for (int q = 0; q < XW / 4; ++q) {
+                    for (int w = 0; w < XW / 4; ++w) {
                         const uint4 v = __ldg(reinterpret_cast<const uint4*>(
-                            xbase + (int64_t)xtk[0] * p.K + (b0 + c) * SB) + q);
-                        xw0[c][4 * q] = v.x; xw0[c][4 * q + 1] = v.y; xw0[c][4 * q + 2] = v.z; xw0[c][4 * q + 3] = v.w;
+                            xbase + (int64_t)xtk[0] * p.K + (b0 + c) * SB) + w);
+                        xw0[c][4 * w] = v.x; xw0[c][4 * w + 1] = v.y; xw0[c][4 * w + 2] = v.z; xw0[c][4 * w + 3] = v.w;
                     }
                 }
             }
             const uint32_t slot = ctr % ns, ph = (ctr / ns) & 1u;
             ++ctr;
-            if (!mbar_wait(smem_u32(bars + slot), ph, abort_flag)) break;
-            const uint8_t* st = smem + slot * plan.stage_bytes;
+            if (!mbar_wait_bounded(smem_addr(full + slot), ph, abort_flag, &g_decode_error, 2u)) break;
+            const uint8_t* st = ring + slot * plan.stage_bytes;
 #pragma unroll
             for (int c = 0; c < BPW; ++c) {
                 if (b0 + c < b1) {
                     const int b = b0 + c;
+                    // this lane's packed bytes of rows g and g+8
                     uint32_t w0[BPL / 4], w1[BPL / 4];
                     const uint8_t* rp0 = st + g * plan.row_stride + b * (SB / 2) + t * BPL;
                     const uint8_t* rp1 = rp0 + 8 * plan.row_stride;
@@ -264,14 +256,13 @@ __global__ void __maxnreg__(112) decode_band_kernel(const GroupedArgs p, const d
                         w0[0] = *reinterpret_cast<const uint32_t*>(rp0);
                         w1[0] = *reinterpret_cast<const uint32_t*>(rp1);
                     }
-                    uint32_t d0[2 * BPL / 2], d1[2 * BPL / 2];
+                    // byte j -> bf16x2 word j (table lookup; address = byte*256 + lane*4)
+                    uint32_t d0[BPL], d1[BPL];
 #pragma unroll
-                    for (int q = 0; q < BPL / 4; ++q) {
-                        uint32_t o[4];
-                        decode_word<FMT>(w0[q], p.lut, o);
-                        d0[4 * q] = o[0]; d0[4 * q + 1] = o[1]; d0[4 * q + 2] = o[2]; d0[4 * q + 3] = o[3];
-                        decode_word<FMT>(w1[q], p.lut, o);
-                        d1[4 * q] = o[0]; d1[4 * q + 1] = o[1]; d1[4 * q + 2] = o[2]; d1[4 * q + 3] = o[3];
+                    for (int j = 0; j < BPL; ++j) {
+                        const uint32_t sel = 0x5504u | ((uint32_t)(j & 3) << 4);
+                        d0[j] = *reinterpret_cast<const uint32_t*>(lut + prmt(w0[j >> 2], lane_sel, sel));
+                        d1[j] = *reinterpret_cast<const uint32_t*>(lut + prmt(w1[j >> 2], lane_sel, sel));
                     }
 #pragma unroll
                     for (int j = 0; j < GMAX; ++j) {
@@ -279,17 +270,17 @@ __global__ void __maxnreg__(112) decode_band_kernel(const GroupedArgs p, const d
                             uint32_t xw[XW];
                             if (j == 0) {
 #pragma unroll
-                                for (int q = 0; q < XW; ++q) xw[q] = xw0[c][q];
+                                for (int w = 0; w < XW; ++w) xw[w] = xw0[c][w];
                             } else if (xtk[j] >= 0) {
 #pragma unroll
-                                for (int q = 0; q < XW / 4; ++q) {
+                                for (int w = 0; w < XW / 4; ++w) {
                                     const uint4 v = __ldg(reinterpret_cast<const uint4*>(
-                                        xbase + (int64_t)xtk[j] * p.K + b * SB) + q);
-                                    xw[4 * q] = v.x; xw[4 * q + 1] = v.y; xw[4 * q + 2] = v.z; xw[4 * q + 3] = v.w;
+                                        xbase + (int64_t)xtk[j] * p.K + b * SB) + w);
+                                    xw[4 * w] = v.x; xw[4 * w + 1] = v.y; xw[4 * w + 2] = v.z; xw[4 * w + 3] = v.w;
                                 }
                             } else {
 #pragma unroll
-                                for (int q = 0; q < XW; ++q) xw[q] = 0u;
+                                for (int w = 0; w < XW; ++w) xw[w] = 0u;
                             }
                             float cb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -305,30 +296,30 @@ __global__ void __maxnreg__(112) decode_band_kernel(const GroupedArgs p, const d
                 }
             }
             __syncwarp();
-            if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bars + 16 + slot))
-                                        : "memory");
+            if (lane == 0) mbar_arrive(smem_addr(empty + slot));
             if (cur.kc == plan.nch - 1) {
-                // sum the 8 warp partials in a fixed order, then the epilogue
+                // the group's 4 partial sums, added in a fixed order, then the epilogue
 #pragma unroll
                 for (int j = 0; j < GMAX; ++j)
-                    if (j < G) red[(warp * GMAX + j) * 32 + lane] = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
-                asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");
-                for (int q = threadIdx.x; q < G * 128; q += kConsumers * 32) {
-                    const int j = q >> 7, ln = (q >> 2) & 31, i = q & 3;
+                    if (j < G) gred[(gw * GMAX + j) * 32 + lane] = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+                asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "n"(kGroupWarps * 32) : "memory");
+                const int tid = gw * 32 + lane;
+                for (int qq = tid; qq < G * 128; qq += kGroupWarps * 32) {
+                    const int j = qq >> 7, ln = (qq >> 2) & 31, i = qq & 3;
                     float v = 0.f;
 #pragma unroll
-                    for (int w = 0; w < kConsumers; ++w)
-                        v += reinterpret_cast<const float*>(&red[(w * GMAX + j) * 32 + ln])[i];
-                    const int slot_row = mc + 8 * j + 2 * (ln & 3) + (i & 1);   // C column 2t (+1)
-                    if (slot_row < m) {
-                        const int64_t r = r0 + slot_row;
+                    for (int w = 0; w < kGroupWarps; ++w)
+                        v += reinterpret_cast<const float*>(&gred[(w * GMAX + j) * 32 + ln])[i];
+                    const int row = mc + 8 * j + 2 * (ln & 3) + (i & 1);   // C column 2t (+1)
+                    if (row < m) {
+                        const int64_t r = r0 + row;
                         if (p.row_weight) v *= __ldg(p.row_weight + r);
                         const int64_t dst = p.row_dest ? (int64_t)__ldg(p.row_dest + r) : r;
-                        const int n = n0 + (ln >> 2) + ((i & 2) ? 8 : 0);        // C row g (+8)
+                        const int n = n0 + (ln >> 2) + ((i & 2) ? 8 : 0);   // C row g (+8)
                         p.out[dst * p.N + n] = f32_to_bf16_rne(v);
                     }
                 }
-                asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");
+                asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "n"(kGroupWarps * 32) : "memory");
             }
             cur = nxt;
         }
@@ -338,27 +329,20 @@ __global__ void __maxnreg__(112) decode_band_kernel(const GroupedArgs p, const d
 template <int FMT, int GMAX>
 static cudaError_t launch_db(const GroupedArgs& a, cudaStream_t s) {
     using namespace db;
-    constexpr int SB = (FMT == FMT_NF4) ? 64 : 32;
     Plan plan;
-    plan.kch = kBlocksPerStage * SB;
-    if (plan.kch > a.K) plan.kch = a.K;
+    plan.kch = kChunkK < a.K ? kChunkK : a.K;
     plan.nch = (a.K + plan.kch - 1) / plan.kch;
     plan.row_stride = plan.kch / 2 + 16;
     plan.stage_bytes = ((16 * plan.row_stride + 127) / 128) * 128;
     const int red_bytes = kConsumers * GMAX * 32 * (int)sizeof(float4);
-    const int fixed = red_bytes + 16 * 8 * 2 + 16 + 16 + kMaxExperts * 4;
-    int per_sm = 2;
-    int budget = 113 * 1024;
-    int nst = (budget - fixed) / plan.stage_bytes;
-    if (nst < 2) {
-        per_sm = 1;
-        budget = 225 * 1024;
-        nst = (budget - fixed) / plan.stage_bytes;
-    }
+    const int tail = 2 * kGroups * 16 * 8 + 32 + kMaxExperts * 4;
+    const int budget = 226 * 1024 - kLutBytes - red_bytes - tail;
+    int nst = budget / (kGroups * plan.stage_bytes);
     if (nst > 8) nst = 8;
     if (nst < 2) return cudaErrorInvalidValue;
     plan.nstages = nst;
-    const int smem = nst * plan.stage_bytes + fixed;
+    const int smem = kLutBytes + kGroups * nst * plan.stage_bytes + red_bytes + 2 * kGroups * nst * 8 + 32 +
+                     kMaxExperts * 4;
     static int smem_set = 0;                 // largest dynamic shared memory opted in so far
     if (smem > smem_set) {
         cudaError_t e = cudaFuncSetAttribute(decode_band_kernel<FMT, GMAX>,
@@ -368,7 +352,7 @@ static cudaError_t launch_db(const GroupedArgs& a, cudaStream_t s) {
     }
     const int64_t groups_max = a.R < (int64_t)a.E ? a.R : (int64_t)a.E;
     const int64_t items_max = groups_max * (a.N / 16);
-    int64_t grid = (int64_t)device_sm_count() * per_sm;
+    int64_t grid = device_sm_count();
     if (items_max < grid) grid = items_max;
     if (grid < 1) return cudaSuccess;
     decode_band_kernel<FMT, GMAX><<<(unsigned)grid, kThreads, smem, s>>>(a, plan);

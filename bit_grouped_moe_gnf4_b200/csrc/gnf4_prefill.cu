@@ -10,12 +10,14 @@
 // the tiles of every expert in the band, computed on the device from the
 // expert offsets. Roles (16 warps):
 //   warp 0      tensor-memory owner and MMA issuer (one thread)
-//   warps 1-3   activation loaders: TMA tile loads of contiguous rows, or
-//               16-byte cp.async of the rows named by row_token, both into the
-//               128B-swizzled K-major layout
-//   warps 4-7   decoders: one weight row per thread; packed bytes straight
-//               from HBM to registers, nibbles -> bf16 by byte permutes,
-//               written to shared memory in the 128B-swizzled K-major layout
+//   warps 1-2   activation loaders: TMA tile loads of contiguous rows (one
+//               thread), or 16-byte cp.async of the rows named by row_token,
+//               both into the 128B-swizzled K-major layout
+//   warp 3      packed-weight loader: TMA loads of the tile's 128 rows x 32
+//               bytes per 64 K into a deep ring of its own
+//   warps 4-7   decoders: one weight row per thread; nibbles -> bf16 by byte
+//               permutes, written to shared memory in the 128B-swizzled
+//               K-major layout the MMA reads
 //   warps 8-15  rescale epilogue: per scale block, read the block's fp32 sums
 //               from tensor memory, multiply by the block scale and add into
 //               fp32 running sums held in registers; at the end of a tile,
@@ -45,20 +47,22 @@ namespace pf {
 constexpr int kThreads = 512;
 constexpr int kBM = 128;             // weight rows per tile
 constexpr int kBNMax = 128;          // routed rows per tile (MMA N)
-constexpr int kStages = 5;
+constexpr int kStages = 4;           // A (decoded weights) + B (activations) stages
+constexpr int kWStages = 12;         // packed-weight stages (128 rows x 32 bytes)
 constexpr int kAccBufs = 4;          // tensor-memory block accumulators of kBNMax columns
 constexpr int kKStage = 64;          // K per pipeline stage (one 128-byte swizzle row of bf16)
 constexpr int kAStageBytes = kBM * 128;
 constexpr int kBStageBytes = kBNMax * 128;
+constexpr int kWStageBytes = kBM * 32;
 constexpr int kMaxExperts = 2048;
-constexpr int kPrefetch = 4;         // packed-weight stages held ahead in decoder registers
-constexpr long long kTimeoutCycles = 1LL << 32;
+constexpr int kGatherThreads = 64;   // warps 1-2
 
 // shared memory map (offsets from a 1024-aligned base)
 constexpr int kOffA = 0;
 constexpr int kOffB = kOffA + kStages * kAStageBytes;
-constexpr int kOffBar = kOffB + kStages * kBStageBytes;
-constexpr int kNumBars = 3 * kStages + 2 * kAccBufs;
+constexpr int kOffW = kOffB + kStages * kBStageBytes;
+constexpr int kOffBar = kOffW + kWStages * kWStageBytes;
+constexpr int kNumBars = 3 * kStages + 2 * kWStages + 2 * kAccBufs;
 constexpr int kOffTmem = kOffBar + kNumBars * 8;
 constexpr int kOffAbort = kOffTmem + 4;
 constexpr int kOffList = kOffTmem + 16;                       // int[kMaxExperts] experts of the band
@@ -73,44 +77,6 @@ struct Tile {
     int bn;         // MMA N: cnt rounded up to 16
     int n0;         // first weight row
 };
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-    return ok != 0;
-}
-
-// Bounded wait; on timeout (or when another role already gave up) sets the
-// CTA's abort flag and returns false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    if (mbar_try(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (true) {
-        if (mbar_try(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (clock64() - t0 > kTimeoutCycles) {
-            *abort_flag = 1;
-            atomicOr(&g_prefill_error, 1u);
-            return false;
-        }
-    }
-}
 
 __device__ __forceinline__ void fence_proxy_async() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -214,7 +180,8 @@ __device__ __forceinline__ Tile tile_at(const GroupedArgs& p, const Sched& s, in
 
 template <int FMT>
 __global__ void __launch_bounds__(pf::kThreads, 1)
-prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xmap, const int gather) {
+prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xmap,
+                    const __grid_constant__ CUtensorMap wmap, const int gather) {
     using namespace pf;
     constexpr int SB = (FMT == FMT_NF4) ? 64 : 32;      // scale block
     constexpr int SBPS = kKStage / SB;                  // scale blocks per stage (1 or 2)
@@ -222,17 +189,20 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t sbase = smem_u32(smem);
+    const uint32_t sbase = smem_addr(smem);
     const uint32_t bar_afull = sbase + kOffBar;                  // [kStages] decoders -> MMA
-    const uint32_t bar_bfull = bar_afull + 8 * kStages;          // [kStages] TMA -> MMA
-    const uint32_t bar_empty = bar_bfull + 8 * kStages;          // [kStages] MMA -> producers
-    const uint32_t bar_accfull = bar_empty + 8 * kStages;        // [kAccBufs] MMA -> epilogue
+    const uint32_t bar_bfull = bar_afull + 8 * kStages;          // [kStages] activation loaders -> MMA
+    const uint32_t bar_empty = bar_bfull + 8 * kStages;          // [kStages] MMA -> decoders, loaders
+    const uint32_t bar_wfull = bar_empty + 8 * kStages;          // [kWStages] weight loader -> decoders
+    const uint32_t bar_wempty = bar_wfull + 8 * kWStages;        // [kWStages] decoders -> weight loader
+    const uint32_t bar_accfull = bar_wempty + 8 * kWStages;      // [kAccBufs] MMA -> epilogue
     const uint32_t bar_accempty = bar_accfull + 8 * kAccBufs;    // [kAccBufs] epilogue -> MMA
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffTmem);
     int* s_list = reinterpret_cast<int*>(smem + kOffList);
     int* s_cum = reinterpret_cast<int*>(smem + kOffCum);
     int* s_count = reinterpret_cast<int*>(smem + kOffCount);
+    unsigned* err = &g_prefill_error;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nnt = (p.N + kBM - 1) / kBM;
@@ -250,8 +220,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
                 act = (m >= p.m_lo) && (m <= p.m_hi);
             }
             const int nt = act ? ((m + kBNMax - 1) / kBNMax) * nnt : 0;
-            // inclusive scan of tile counts across the warp
-            int inc = nt;
+            int inc = nt;                        // inclusive scan of tile counts across the warp
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int v = __shfl_up_sync(0xffffffffu, inc, o);
@@ -274,8 +243,12 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
     } else if (warp == 3 && lane == 0) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(bar_afull + 8 * i, 128);
-            mbar_init(bar_bfull + 8 * i, gather ? 96 : 1);
+            mbar_init(bar_bfull + 8 * i, gather ? kGatherThreads : 1);
             mbar_init(bar_empty + 8 * i, 1);
+        }
+        for (int i = 0; i < kWStages; ++i) {
+            mbar_init(bar_wfull + 8 * i, 1);
+            mbar_init(bar_wempty + 8 * i, 4);
         }
         for (int i = 0; i < kAccBufs; ++i) {
             mbar_init(bar_accfull + 8 * i, 1);
@@ -285,7 +258,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     } else if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;"
-                     ::"r"(smem_u32(tmem_slot)) : "memory");
+                     ::"r"(smem_addr(tmem_slot)) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
@@ -303,15 +276,15 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
                 const uint32_t idesc = idesc_bf16(tl.bn);
                 for (int s = 0; s < nst; ++s, ++stage_ctr) {
                     const uint32_t slot = stage_ctr % kStages, ph = (stage_ctr / kStages) & 1u;
-                    if (!mbar_wait(bar_afull + 8 * slot, ph, abort_flag)) goto mma_done;
-                    if (!mbar_wait(bar_bfull + 8 * slot, ph, abort_flag)) goto mma_done;
+                    if (!mbar_wait_bounded(bar_afull + 8 * slot, ph, abort_flag, err, 1u)) goto mma_done;
+                    if (!mbar_wait_bounded(bar_bfull + 8 * slot, ph, abort_flag, err, 2u)) goto mma_done;
                     tc_fence_after();
                     const uint32_t a_addr = sbase + kOffA + slot * kAStageBytes;
                     const uint32_t b_addr = sbase + kOffB + slot * kBStageBytes;
                     const int nsb = min(SBPS, (p.K - s * kKStage) / SB);
                     for (int sb = 0; sb < nsb; ++sb, ++acc_ctr) {
                         const uint32_t buf = acc_ctr % kAccBufs, aph = ((acc_ctr / kAccBufs) & 1u) ^ 1u;
-                        if (!mbar_wait(bar_accempty + 8 * buf, aph, abort_flag)) goto mma_done;
+                        if (!mbar_wait_bounded(bar_accempty + 8 * buf, aph, abort_flag, err, 4u)) goto mma_done;
                         tc_fence_after();
 #pragma unroll
                         for (int q = 0; q < K16PSB; ++q) {
@@ -327,7 +300,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
         }
     mma_done:
         __syncwarp();
-    } else if (warp >= 1 && warp <= 3) {
+    } else if (warp == 1 || warp == 2) {
         // ================= activation loaders =================
         if (!gather) {
             // contiguous routed rows: TMA tile loads, 16 rows x 64 K per box, 128B-swizzled
@@ -337,7 +310,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
                     const Tile tl = tile_at(p, sch, t, nnt);
                     for (int s = 0; s < nst; ++s, ++stage_ctr) {
                         const uint32_t slot = stage_ctr % kStages, ph = ((stage_ctr / kStages) & 1u) ^ 1u;
-                        if (!mbar_wait(bar_empty + 8 * slot, ph, abort_flag)) goto load_done;
+                        if (!mbar_wait_bounded(bar_empty + 8 * slot, ph, abort_flag, err, 8u)) goto load_done;
                         const uint32_t full = bar_bfull + 8 * slot;
                         const uint32_t dst = sbase + kOffB + slot * kBStageBytes;
                         mbar_arrive_tx(full, (uint32_t)tl.bn * 128u);
@@ -350,102 +323,100 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
             // gathered rows (row_token): 16-byte cp.async per (row, chunk), written in the
             // 128B-swizzled layout; each thread completes its copies of a stage, makes them
             // visible to the tensor core (proxy fence) and arrives, two stages behind issue
-            const int l = threadIdx.x - 32;              // 0..95
+            const int l = threadIdx.x - 32;              // 0..63
             const int c = l & 7;                         // 16-byte chunk of the 128-byte row
-            const int rb = l >> 3;                       // first row: rb, rb + 12, ...
-            constexpr int kRowsPer = (kBNMax + 11) / 12;   // rows per thread
+            const int rb = l >> 3;                       // rows rb, rb + 8, ...: row & 7 == rb
+            const uint32_t swz = (uint32_t)((c ^ rb) << 4);
+            constexpr int kRowsPer = kBNMax / 8;
             uint32_t stage_ctr = 0;
             int npend = 0;
-            uint32_t pend0 = 0, pend1 = 0;
+            uint32_t pend0 = 0, pend1 = 0, pend2 = 0;
             for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
                 const Tile tl = tile_at(p, sch, t, nnt);
                 int tok[kRowsPer];
 #pragma unroll
                 for (int j = 0; j < kRowsPer; ++j) {
-                    const int row = rb + 12 * j;
+                    const int row = rb + 8 * j;
                     tok[j] = (row < tl.cnt) ? __ldg(p.row_token + tl.r0 + row) : -1;
                 }
                 for (int s = 0; s < nst; ++s, ++stage_ctr) {
                     const uint32_t slot = stage_ctr % kStages, ph = ((stage_ctr / kStages) & 1u) ^ 1u;
-                    if (!mbar_wait(bar_empty + 8 * slot, ph, abort_flag)) goto load_done;
-                    const uint32_t dst = sbase + kOffB + slot * kBStageBytes;
+                    if (!mbar_wait_bounded(bar_empty + 8 * slot, ph, abort_flag, err, 8u)) goto load_done;
+                    const uint32_t dst = sbase + kOffB + slot * kBStageBytes + swz;
                     const int kx = s * kKStage + c * 8;
                     if (kx < p.K) {
 #pragma unroll
                         for (int j = 0; j < kRowsPer; ++j) {
-                            const int row = rb + 12 * j;
                             if (tok[j] >= 0)
-                                cp_async16(dst + row * 128 + ((c ^ (row & 7)) << 4),
-                                           p.x + (int64_t)tok[j] * p.K + kx);
+                                cp_async16(dst + (rb + 8 * j) * 128, p.x + (int64_t)tok[j] * p.K + kx);
                         }
                     }
                     cp_async_commit();
-                    if (npend == 0) { pend0 = slot; npend = 1; }
-                    else if (npend == 1) { pend1 = slot; npend = 2; }
-                    if (npend == 2) {
-                        cp_async_wait<1>();
+                    if (npend == 0) pend0 = slot;
+                    else if (npend == 1) pend1 = slot;
+                    else pend2 = slot;
+                    ++npend;
+                    if (npend == 3) {
+                        cp_async_wait<2>();
                         fence_proxy_async();
                         mbar_arrive(bar_bfull + 8 * pend0);
                         pend0 = pend1;
-                        npend = 1;
+                        pend1 = pend2;
+                        npend = 2;
                     }
                 }
             }
             cp_async_wait<0>();
             fence_proxy_async();
-            if (npend == 1) mbar_arrive(bar_bfull + 8 * pend0);
+            if (npend >= 1) mbar_arrive(bar_bfull + 8 * pend0);
+            if (npend >= 2) mbar_arrive(bar_bfull + 8 * pend1);
         }
     load_done:
         cp_async_wait<0>();
+        __syncwarp();
+    } else if (warp == 3) {
+        // ================= packed-weight loader (TMA) =================
+        if (lane == 0) {
+            uint32_t ctr = 0;
+            for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
+                const Tile tl = tile_at(p, sch, t, nnt);
+                const int row0 = tl.e * p.N + tl.n0;
+                for (int s = 0; s < nst; ++s, ++ctr) {
+                    const uint32_t slot = ctr % kWStages, ph = ((ctr / kWStages) & 1u) ^ 1u;
+                    if (!mbar_wait_bounded(bar_wempty + 8 * slot, ph, abort_flag, err, 16u)) goto wload_done;
+                    const uint32_t full = bar_wfull + 8 * slot;
+                    mbar_arrive_tx(full, (uint32_t)kWStageBytes);
+                    tma_tile_2d(sbase + kOffW + slot * kWStageBytes, &wmap, s * 32, row0, full);
+                }
+            }
+        }
+    wload_done:
         __syncwarp();
     } else if (warp >= 4 && warp < 8) {
         // ================= decoders: one weight row per thread =================
         const int i = threadIdx.x - 128;                   // tile row
         uint32_t stage_ctr = 0;
-        const int64_t rowbytes = p.K >> 1;
         for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
-            const Tile tl = tile_at(p, sch, t, nnt);
-            const int n = tl.n0 + i;
-            const bool valid = n < p.N;
-            const uint8_t* wrow = p.W + ((int64_t)tl.e * p.N + (valid ? n : 0)) * rowbytes;
-            uint4 pre[kPrefetch][2];
+            for (int s = 0; s < nst; ++s, ++stage_ctr) {
+                // packed bytes of row i for this stage, from the weight ring
+                const uint32_t wslot = stage_ctr % kWStages, wph = (stage_ctr / kWStages) & 1u;
+                if (!mbar_wait_bounded(bar_wfull + 8 * wslot, wph, abort_flag, err, 32u)) goto dec_done;
+                const uint4* wsrc = reinterpret_cast<const uint4*>(smem + kOffW + wslot * kWStageBytes + i * 32);
+                const uint4 c0 = wsrc[0], c1 = wsrc[1];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_wempty + 8 * wslot);
+                const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                uint32_t o[8][4];
 #pragma unroll
-            for (int q = 0; q < kPrefetch; ++q) {
-                pre[q][0] = pre[q][1] = make_uint4(0u, 0u, 0u, 0u);
-                if (valid && q < nst) {
-                    const uint4* src = reinterpret_cast<const uint4*>(wrow + q * 32);
-                    pre[q][0] = __ldg(src);
-                    if (q * kKStage + 32 < p.K) pre[q][1] = __ldg(src + 1);
-                }
-            }
-            for (int s0 = 0; s0 < nst; s0 += kPrefetch) {
+                for (int c = 0; c < 8; ++c) decode_word<FMT>(words[c], p.lut, o[c]);
+                const uint32_t slot = stage_ctr % kStages, ph = ((stage_ctr / kStages) & 1u) ^ 1u;
+                if (!mbar_wait_bounded(bar_empty + 8 * slot, ph, abort_flag, err, 64u)) goto dec_done;
+                uint8_t* arow = smem + kOffA + slot * kAStageBytes + i * 128;
 #pragma unroll
-                for (int q = 0; q < kPrefetch; ++q) {
-                    const int s = s0 + q;
-                    if (s < nst) {
-                        const uint32_t slot = stage_ctr % kStages, ph = ((stage_ctr / kStages) & 1u) ^ 1u;
-                        ++stage_ctr;
-                        const uint4 c0 = pre[q][0], c1 = pre[q][1];
-                        // refill this slot with stage s + kPrefetch
-                        const int sn = s + kPrefetch;
-                        if (valid && sn < nst) {
-                            const uint4* src = reinterpret_cast<const uint4*>(wrow + sn * 32);
-                            pre[q][0] = __ldg(src);
-                            if (sn * kKStage + 32 < p.K) pre[q][1] = __ldg(src + 1);
-                        }
-                        if (!mbar_wait(bar_empty + 8 * slot, ph, abort_flag)) goto dec_done;
-                        uint8_t* arow = smem + kOffA + slot * kAStageBytes + i * 128;
-                        const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {          // 16-byte chunk c: K elements 8c .. 8c+7
-                            uint32_t o[4];
-                            decode_word<FMT>(words[c], p.lut, o);
-                            *reinterpret_cast<uint4*>(arow + ((c ^ (i & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-                        }
-                        fence_proxy_async();
-                        mbar_arrive(bar_afull + 8 * slot);
-                    }
-                }
+                for (int c = 0; c < 8; ++c)          // 16-byte chunk c: K elements 8c .. 8c+7
+                    *reinterpret_cast<uint4*>(arow + ((c ^ (i & 7)) << 4)) = make_uint4(o[c][0], o[c][1], o[c][2], o[c][3]);
+                fence_proxy_async();
+                mbar_arrive(bar_afull + 8 * slot);
             }
         }
     dec_done:;
@@ -472,7 +443,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
                 const float sc = scale_next;
                 if (b + 1 < nsbk) scale_next = load_scale<FMT>(p.scales, srow + b + 1);
                 const uint32_t buf = acc_ctr % kAccBufs, ph = (acc_ctr / kAccBufs) & 1u;
-                if (!mbar_wait(bar_accfull + 8 * buf, ph, abort_flag)) goto epi_done;
+                if (!mbar_wait_bounded(bar_accfull + 8 * buf, ph, abort_flag, err, 128u)) goto epi_done;
                 tc_fence_after();
                 const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16) + buf * kBNMax;
 #pragma unroll
@@ -554,17 +525,31 @@ static cudaError_t launch_pf(const GroupedArgs& a, int64_t T_in, cudaStream_t s)
     auto enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
     const int gather = a.row_token != nullptr;
-    CUtensorMap map;
-    cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)T_in};
-    cuuint64_t strides[1] = {(cuuint64_t)a.K * 2};
-    cuuint32_t box[2] = {64, 16};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.x), dims, strides, box,
-                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    CUtensorMap xmap, wmap;
+    {
+        // activations: bf16 [T_in, K], boxes of 64 K x 16 rows, 128B swizzle
+        cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)T_in};
+        cuuint64_t strides[1] = {(cuuint64_t)a.K * 2};
+        cuuint32_t box[2] = {64, 16};
+        cuuint32_t estr[2] = {1, 1};
+        CUresult r = enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.x), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    }
+    {
+        // packed weights: bytes [E*N, K/2], boxes of 32 bytes x 128 rows, no swizzle
+        cuuint64_t dims[2] = {(cuuint64_t)(a.K / 2), (cuuint64_t)a.E * (cuuint64_t)a.N};
+        cuuint64_t strides[1] = {(cuuint64_t)(a.K / 2)};
+        cuuint32_t box[2] = {32, pf::kBM};
+        cuuint32_t estr[2] = {1, 1};
+        CUresult r = enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.W), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    }
     const int grid = device_sm_count();
-    prefill_band_kernel<FMT><<<grid, pf::kThreads, pf::kSmemBytes, s>>>(a, map, gather);
+    prefill_band_kernel<FMT><<<grid, pf::kThreads, pf::kSmemBytes, s>>>(a, xmap, wmap, gather);
     return cudaGetLastError();
 }
 
