@@ -53,7 +53,8 @@ struct Plan {
     int nch;          // stages per item pass
     int row_stride;   // bytes per weight row in a stage (chunk bytes + 16 of padding)
     int stage_bytes;  // 16 rows
-    int nstages;      // stages per group ring
+    int scale_bytes;  // slot for one item's scales (16 rows x all blocks, contiguous in memory), rounded to 128
+    int nstages;      // stages (and item scale slots) per group ring
 };
 
 struct Pos {
@@ -72,14 +73,19 @@ __global__ void __launch_bounds__(db::kThreads, 1) decode_band_kernel(const Grou
     constexpr int BPW = (kChunkK / SB) / kGroupWarps;  // blocks per warp per full chunk (2 or 4)
 
     extern __shared__ __align__(1024) uint8_t smem[];
+    // [lut][rings: groups x stages x stage_bytes][scale slots: groups x stages x scale_bytes]
+    // [red][barriers][abort, counts][active experts: id, first row, rows]
     uint8_t* lut = smem;                                            // [256][64] words
-    uint8_t* rings = smem + kLutBytes;                              // [groups][stages][16 rows][row_stride]
-    float4* red = reinterpret_cast<float4*>(rings + kGroups * plan.nstages * plan.stage_bytes);
+    uint8_t* rings = smem + kLutBytes;
+    uint8_t* sslots = rings + kGroups * plan.nstages * plan.stage_bytes;
+    float4* red = reinterpret_cast<float4*>(sslots + kGroups * plan.nstages * plan.scale_bytes);
     uint64_t* bars = reinterpret_cast<uint64_t*>(red + kConsumers * GMAX * 32);   // full[g][s], empty[g][s]
     int* tailw = reinterpret_cast<int*>(bars + 2 * kGroups * plan.nstages);
     volatile int* abort_flag = tailw;
     int* s_nact = tailw + 4;
-    int* s_active = tailw + 8;
+    int64_t* s_r0 = reinterpret_cast<int64_t*>(tailw + 8);         // [E] first routed row
+    int* s_active = reinterpret_cast<int*>(s_r0 + p.E);            // [E] expert id
+    int* s_cnt = s_active + p.E;                                   // [E] routed rows
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ns = plan.nstages;
@@ -100,7 +106,12 @@ __global__ void __launch_bounds__(db::kThreads, 1) decode_band_kernel(const Grou
                 act = (m >= p.m_lo) && (m <= p.m_hi);
             }
             const unsigned bal = __ballot_sync(0xffffffffu, act);
-            if (act) s_active[count + __popc(bal & ((1u << lane) - 1u))] = e;
+            if (act) {
+                const int idx = count + __popc(bal & ((1u << lane) - 1u));
+                s_active[idx] = e;
+                s_r0[idx] = p.offsets[e];
+                s_cnt[idx] = (int)(p.offsets[e + 1] - p.offsets[e]);
+            }
             count += __popc(bal);
         }
         if (lane == 0) s_nact[0] = count;
@@ -124,8 +135,7 @@ __global__ void __launch_bounds__(db::kThreads, 1) decode_band_kernel(const Grou
     auto advance = [&](Pos q) -> Pos {
         if (++q.kc == plan.nch) {
             q.kc = 0;
-            const int e = s_active[q.item / nt];
-            const int m = (int)(p.offsets[e + 1] - p.offsets[e]);
+            const int m = s_cnt[q.item / nt];
             if (++q.pass == (m + 8 * GMAX - 1) / (8 * GMAX)) {
                 q.pass = 0;
                 q.item += kGroups;
@@ -141,7 +151,9 @@ __global__ void __launch_bounds__(db::kThreads, 1) decode_band_kernel(const Grou
             uint64_t* full = bars + q * ns;
             uint64_t* empty = bars + kGroups * ns + q * ns;
             uint8_t* ring = rings + q * ns * plan.stage_bytes;
-            uint32_t ctr = 0;
+            uint8_t* sring = sslots + q * ns * plan.scale_bytes;
+            const int ssz = FMT == FMT_NF4 ? 4 : 1;
+            uint32_t ctr = 0, jitem = 0;
             for (Pos ps{i0 + q, 0, 0}; ps.item < i1; ps = advance(ps), ++ctr) {
                 const uint32_t slot = ctr % ns, ph = ((ctr / ns) & 1u) ^ 1u;
                 if (!mbar_wait_bounded(smem_addr(empty + slot), ph, abort_flag, &g_decode_error, 1u)) break;
@@ -150,7 +162,19 @@ __global__ void __launch_bounds__(db::kThreads, 1) decode_band_kernel(const Grou
                 const int kb = ps.kc * plan.kch;
                 const uint32_t bytes = (uint32_t)(min(plan.kch, p.K - kb) >> 1);
                 const uint32_t fb = smem_addr(full + slot);
-                mbar_arrive_tx(fb, 16u * bytes);
+                const bool first = ps.kc == 0 && ps.pass == 0;
+                const uint32_t sbytes = (uint32_t)(16 * nbk * ssz);      // exact, a multiple of 16
+                mbar_arrive_tx(fb, 16u * bytes + (first ? sbytes : 0u));
+                if (first) {
+                    // the item's scales: 16 rows x all blocks, one contiguous range
+                    const uint8_t* ssrc = reinterpret_cast<const uint8_t*>(p.scales) +
+                                          ((int64_t)e * p.N + n0) * nbk * ssz;
+                    asm volatile(
+                        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                        ::"r"(smem_addr(sring + (jitem % ns) * plan.scale_bytes)), "l"(ssrc),
+                          "r"(sbytes), "r"(fb) : "memory");
+                    ++jitem;
+                }
                 const uint8_t* src = p.W + ((int64_t)e * p.N + n0) * rowbytes + (kb >> 1);
                 const uint32_t dst = smem_addr(ring + slot * plan.stage_bytes);
                 for (int r = 0; r < 16; ++r)
@@ -168,81 +192,81 @@ __global__ void __launch_bounds__(db::kThreads, 1) decode_band_kernel(const Grou
         uint64_t* full = bars + q * ns;
         uint64_t* empty = bars + kGroups * ns + q * ns;
         const uint8_t* ring = rings + q * ns * plan.stage_bytes;
+        const uint8_t* sring = sslots + q * ns * plan.scale_bytes;
         float4* gred = red + q * kGroupWarps * GMAX * 32;
         const uint32_t lane_sel = (uint32_t)lane * 4u;   // lut offset of this lane's copy
-        uint32_t ctr = 0;
+        uint32_t ctr = 0, jitem = 0;
         float acc[GMAX][4];
-        float sc0[BPW], sc1[BPW], nsc0[BPW], nsc1[BPW];
-        auto load_scales = [&](const Pos& ps, float (&s0)[BPW], float (&s1)[BPW]) {
-            const int e = s_active[ps.item / nt];
-            const int n0 = (ps.item % nt) << 4;
-            const int nbc = min(plan.kch, p.K - ps.kc * plan.kch) / SB;
-            const int b0 = gw * nbc / kGroupWarps, b1 = (gw + 1) * nbc / kGroupWarps;
-            const int64_t base0 = ((int64_t)e * p.N + n0 + g) * nbk + ps.kc * (plan.kch / SB);
+        // activation row of this lane's token column g, per 8-row group (-1: none), for the
+        // current and the next item; the next item's rows are prefetched into L1 early
+        int xtk[GMAX], ntk[GMAX];
+        auto tokens_of = [&](int item, int pass, int (&tk)[GMAX]) {
 #pragma unroll
-            for (int c = 0; c < BPW; ++c) {
-                s0[c] = s1[c] = 0.f;
-                if (b0 + c < b1) {
-                    s0[c] = load_scale<FMT>(p.scales, base0 + b0 + c);
-                    s1[c] = load_scale<FMT>(p.scales, base0 + 8 * (int64_t)nbk + b0 + c);
+            for (int j = 0; j < GMAX; ++j) tk[j] = -1;
+            if (item >= i1) return;
+            const int a = item / nt;
+            const int64_t r0 = s_r0[a];
+            const int m = s_cnt[a];
+            const int mc = pass * 8 * GMAX;
+#pragma unroll
+            for (int j = 0; j < GMAX; ++j) {
+                const int rr = mc + 8 * j + g;
+                if (rr < m) tk[j] = p.row_token ? __ldg(p.row_token + r0 + rr) : (int)(r0 + rr);
+            }
+        };
+        auto prefetch_x = [&](const int (&tk)[GMAX]) {
+            // this lane's 16-byte pieces of x for every block of this warp, all chunks
+#pragma unroll
+            for (int j = 0; j < GMAX; ++j) {
+                if (tk[j] < 0) continue;
+                const uint16_t* xr = p.x + (int64_t)tk[j] * p.K + t * (SB / 4);
+                for (int kc = 0; kc < plan.nch; ++kc) {
+                    const int kb = kc * plan.kch;
+                    const int nbc = min(plan.kch, p.K - kb) / SB;
+                    for (int b = gw * nbc / kGroupWarps; b < (gw + 1) * nbc / kGroupWarps; ++b)
+                        asm volatile("prefetch.global.L1 [%0];" ::"l"(xr + kb + b * SB));
                 }
             }
         };
         Pos cur{i0 + q, 0, 0};
-        if (cur.item < i1) load_scales(cur, nsc0, nsc1);
+        tokens_of(cur.item, 0, xtk);
+        prefetch_x(xtk);
+        tokens_of(cur.item + kGroups, 0, ntk);
         while (cur.item < i1) {
-            const int e = s_active[cur.item / nt];
+            const int a = cur.item / nt;
             const int n0 = (cur.item % nt) << 4;
-            const int64_t r0 = p.offsets[e];
-            const int m = (int)(p.offsets[e + 1] - r0);
+            const int64_t r0 = s_r0[a];
+            const int m = s_cnt[a];
             const int mc = cur.pass * 8 * GMAX;
             const int G = min(GMAX, (m - mc + 7) >> 3);
-#pragma unroll
-            for (int c = 0; c < BPW; ++c) { sc0[c] = nsc0[c]; sc1[c] = nsc1[c]; }
             const Pos nxt = advance(cur);
-            if (nxt.item < i1) load_scales(nxt, nsc0, nsc1);
             if (cur.kc == 0) {
 #pragma unroll
                 for (int j = 0; j < GMAX; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+                if (cur.pass == 0) prefetch_x(ntk);       // next item's rows, one item ahead
             }
             const int kb = cur.kc * plan.kch;
             const int nbc = min(plan.kch, p.K - kb) / SB;
             const int b0 = gw * nbc / kGroupWarps, b1 = (gw + 1) * nbc / kGroupWarps;
-            // activation row of this lane's token column g, per 8-row group (-1: none)
-            int xtk[GMAX];
-#pragma unroll
-            for (int j = 0; j < GMAX; ++j) {
-                const int rr = mc + 8 * j + g;
-                xtk[j] = -1;
-                if (j < G && rr < m) {
-                    const int64_t r = r0 + rr;
-                    xtk[j] = p.row_token ? __ldg(p.row_token + r) : (int)r;
-                }
-            }
             const uint16_t* xbase = p.x + kb + t * (SB / 4);
-            // group 0's activation words for this warp's blocks, loaded before the wait
-            uint32_t xw0[BPW][XW];
-#pragma unroll
-            for (int c = 0; c < BPW; ++c) {
-#pragma unroll
-                for (int w = 0; w < XW; ++w) xw0[c][w] = 0u;
-                if (b0 + c < b1 && xtk[0] >= 0) {
-#pragma unroll
-                    for (int w = 0; w < XW / 4; ++w) {
-                        const uint4 v = __ldg(reinterpret_cast<const uint4*>(
-                            xbase + (int64_t)xtk[0] * p.K + (b0 + c) * SB) + w);
-                        xw0[c][4 * w] = v.x; xw0[c][4 * w + 1] = v.y; xw0[c][4 * w + 2] = v.z; xw0[c][4 * w + 3] = v.w;
-                    }
-                }
-            }
             const uint32_t slot = ctr % ns, ph = (ctr / ns) & 1u;
             ++ctr;
             if (!mbar_wait_bounded(smem_addr(full + slot), ph, abort_flag, &g_decode_error, 2u)) break;
             const uint8_t* st = ring + slot * plan.stage_bytes;
+            const uint8_t* ss = sring + (jitem % ns) * plan.scale_bytes;
+            const int bg0 = cur.kc * (plan.kch / SB);     // first scale block of the chunk
 #pragma unroll
             for (int c = 0; c < BPW; ++c) {
                 if (b0 + c < b1) {
                     const int b = b0 + c;
+                    float s0, s1;
+                    if constexpr (FMT == FMT_NF4) {
+                        s0 = reinterpret_cast<const float*>(ss)[g * nbk + bg0 + b];
+                        s1 = reinterpret_cast<const float*>(ss)[(g + 8) * nbk + bg0 + b];
+                    } else {
+                        s0 = e8m0_to_f32(ss[g * nbk + bg0 + b]);
+                        s1 = e8m0_to_f32(ss[(g + 8) * nbk + bg0 + b]);
+                    }
                     // this lane's packed bytes of rows g and g+8
                     uint32_t w0[BPL / 4], w1[BPL / 4];
                     const uint8_t* rp0 = st + g * plan.row_stride + b * (SB / 2) + t * BPL;
@@ -268,10 +292,7 @@ __global__ void __launch_bounds__(db::kThreads, 1) decode_band_kernel(const Grou
                     for (int j = 0; j < GMAX; ++j) {
                         if (j < G) {
                             uint32_t xw[XW];
-                            if (j == 0) {
-#pragma unroll
-                                for (int w = 0; w < XW; ++w) xw[w] = xw0[c][w];
-                            } else if (xtk[j] >= 0) {
+                            if (xtk[j] >= 0) {
 #pragma unroll
                                 for (int w = 0; w < XW / 4; ++w) {
                                     const uint4 v = __ldg(reinterpret_cast<const uint4*>(
@@ -287,10 +308,10 @@ __global__ void __launch_bounds__(db::kThreads, 1) decode_band_kernel(const Grou
                             for (int s = 0; s < STEPS; ++s)
                                 mma_bf16_16816(cb, d0[2 * s], d1[2 * s], d0[2 * s + 1], d1[2 * s + 1], xw[2 * s],
                                                xw[2 * s + 1]);
-                            acc[j][0] = fmaf(cb[0], sc0[c], acc[j][0]);
-                            acc[j][1] = fmaf(cb[1], sc0[c], acc[j][1]);
-                            acc[j][2] = fmaf(cb[2], sc1[c], acc[j][2]);
-                            acc[j][3] = fmaf(cb[3], sc1[c], acc[j][3]);
+                            acc[j][0] = fmaf(cb[0], s0, acc[j][0]);
+                            acc[j][1] = fmaf(cb[1], s0, acc[j][1]);
+                            acc[j][2] = fmaf(cb[2], s1, acc[j][2]);
+                            acc[j][3] = fmaf(cb[3], s1, acc[j][3]);
                         }
                     }
                 }
@@ -320,6 +341,15 @@ __global__ void __launch_bounds__(db::kThreads, 1) decode_band_kernel(const Grou
                     }
                 }
                 asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "n"(kGroupWarps * 32) : "memory");
+                // next pass of this item, or the next item
+                if (nxt.item != cur.item) {
+                    ++jitem;
+#pragma unroll
+                    for (int j = 0; j < GMAX; ++j) xtk[j] = ntk[j];
+                    tokens_of(nxt.item + kGroups, 0, ntk);
+                } else {
+                    tokens_of(nxt.item, nxt.pass, xtk);
+                }
             }
             cur = nxt;
         }
@@ -334,15 +364,17 @@ static cudaError_t launch_db(const GroupedArgs& a, cudaStream_t s) {
     plan.nch = (a.K + plan.kch - 1) / plan.kch;
     plan.row_stride = plan.kch / 2 + 16;
     plan.stage_bytes = ((16 * plan.row_stride + 127) / 128) * 128;
+    const int SB = (FMT == FMT_NF4) ? 64 : 32;
+    plan.scale_bytes = ((16 * (a.K / SB) * (FMT == FMT_NF4 ? 4 : 1) + 127) / 128) * 128;
     const int red_bytes = kConsumers * GMAX * 32 * (int)sizeof(float4);
-    const int tail = 2 * kGroups * 16 * 8 + 32 + kMaxExperts * 4;
-    const int budget = 226 * 1024 - kLutBytes - red_bytes - tail;
-    int nst = budget / (kGroups * plan.stage_bytes);
+    const int tables = 32 + 16 * a.E;
+    const int fixed = kLutBytes + red_bytes + 2 * kGroups * 8 * 8 + tables;
+    int nst = (226 * 1024 - fixed) / (kGroups * (plan.stage_bytes + plan.scale_bytes));
     if (nst > 8) nst = 8;
     if (nst < 2) return cudaErrorInvalidValue;
     plan.nstages = nst;
-    const int smem = kLutBytes + kGroups * nst * plan.stage_bytes + red_bytes + 2 * kGroups * nst * 8 + 32 +
-                     kMaxExperts * 4;
+    const int smem = kLutBytes + kGroups * nst * (plan.stage_bytes + plan.scale_bytes) + red_bytes +
+                     2 * kGroups * nst * 8 + tables;
     static int smem_set = 0;                 // largest dynamic shared memory opted in so far
     if (smem > smem_set) {
         cudaError_t e = cudaFuncSetAttribute(decode_band_kernel<FMT, GMAX>,

@@ -8,17 +8,17 @@
 // Tile = 128 weight rows (the MMA's M side, one tensor-memory lane each) x up
 // to 128 routed rows of one expert (the N side), all of K. Persistent CTAs walk
 // the tiles of every expert in the band, computed on the device from the
-// expert offsets. Roles (16 warps):
+// expert offsets. Roles (19 warps):
 //   warp 0      tensor-memory owner and MMA issuer (one thread)
-//   warps 1-2   activation loaders: TMA tile loads of contiguous rows (one
+//   warp 1      activation loader: TMA tile loads of contiguous rows (one
 //               thread), or 16-byte cp.async of the rows named by row_token,
 //               both into the 128B-swizzled K-major layout
-//   warp 3      packed-weight loader: TMA loads of the tile's 128 rows x 32
+//   warp 2      packed-weight loader: TMA loads of the tile's 128 rows x 32
 //               bytes per 64 K into a deep ring of its own
-//   warps 4-7   decoders: one weight row per thread; nibbles -> bf16 by byte
-//               permutes, written to shared memory in the 128B-swizzled
+//   warps 3-10  decoders: half a weight row per thread; nibbles -> bf16 by
+//               byte permutes, written to shared memory in the 128B-swizzled
 //               K-major layout the MMA reads
-//   warps 8-15  rescale epilogue: per scale block, read the block's fp32 sums
+//   warps 11-18 rescale epilogue: per scale block, read the block's fp32 sums
 //               from tensor memory, multiply by the block scale and add into
 //               fp32 running sums held in registers; at the end of a tile,
 //               weight, round to bf16 and store (scatter) the outputs
@@ -44,7 +44,7 @@ __device__ unsigned g_prefill_error;
 
 namespace pf {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 19 * 32;  // see the role list above
 constexpr int kBM = 128;             // weight rows per tile
 constexpr int kBNMax = 128;          // routed rows per tile (MMA N)
 constexpr int kStages = 4;           // A (decoded weights) + B (activations) stages
@@ -55,7 +55,10 @@ constexpr int kAStageBytes = kBM * 128;
 constexpr int kBStageBytes = kBNMax * 128;
 constexpr int kWStageBytes = kBM * 32;
 constexpr int kMaxExperts = 2048;
-constexpr int kGatherThreads = 64;   // warps 1-2
+constexpr int kDecWarp0 = 3;         // decoders: warps 3-10
+constexpr int kDecWarps = 8;
+constexpr int kEpiWarp0 = 11;        // epilogue: warps 11-18
+constexpr int kScaleAhead = 4;       // block scales held ahead in epilogue registers
 
 // shared memory map (offsets from a 1024-aligned base)
 constexpr int kOffA = 0;
@@ -65,7 +68,8 @@ constexpr int kOffBar = kOffW + kWStages * kWStageBytes;
 constexpr int kNumBars = 3 * kStages + 2 * kWStages + 2 * kAccBufs;
 constexpr int kOffTmem = kOffBar + kNumBars * 8;
 constexpr int kOffAbort = kOffTmem + 4;
-constexpr int kOffList = kOffTmem + 16;                       // int[kMaxExperts] experts of the band
+constexpr int kOffRows = kOffTmem + 16;                       // int[kBNMax] gathered rows of the loader's tile
+constexpr int kOffList = kOffRows + kBNMax * 4;               // int[kMaxExperts] experts of the band
 constexpr int kOffCum = kOffList + kMaxExperts * 4;           // int[kMaxExperts+1] tile prefix
 constexpr int kOffCount = kOffCum + (kMaxExperts + 1) * 4;
 constexpr int kSmemBytes = kOffCount + 16 + 1024;             // + alignment slack
@@ -208,8 +212,8 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
     const int nnt = (p.N + kBM - 1) / kBM;
     const int nst = p.K / kKStage + ((p.K % kKStage) ? 1 : 0);   // stages per tile (last may be half, MXFP4)
 
-    // ---- set-up: band experts and tile prefix (warp 2), barriers (warp 3), tensor memory (warp 0)
-    if (warp == 2) {
+    // ---- set-up: band experts and tile prefix (warp 1), barriers (warp 2), tensor memory (warp 0)
+    if (warp == 1) {
         int count = 0, tiles = 0;
         for (int e0 = 0; e0 < p.E; e0 += 32) {
             const int e = e0 + lane;
@@ -240,15 +244,15 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
             s_count[0] = count;
             s_count[1] = tiles;
         }
-    } else if (warp == 3 && lane == 0) {
+    } else if (warp == 2 && lane == 0) {
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(bar_afull + 8 * i, 128);
-            mbar_init(bar_bfull + 8 * i, gather ? kGatherThreads : 1);
+            mbar_init(bar_afull + 8 * i, 32 * kDecWarps);
+            mbar_init(bar_bfull + 8 * i, gather ? 32 : 1);
             mbar_init(bar_empty + 8 * i, 1);
         }
         for (int i = 0; i < kWStages; ++i) {
             mbar_init(bar_wfull + 8 * i, 1);
-            mbar_init(bar_wempty + 8 * i, 4);
+            mbar_init(bar_wempty + 8 * i, kDecWarps);
         }
         for (int i = 0; i < kAccBufs; ++i) {
             mbar_init(bar_accfull + 8 * i, 1);
@@ -300,11 +304,11 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
         }
     mma_done:
         __syncwarp();
-    } else if (warp == 1 || warp == 2) {
-        // ================= activation loaders =================
+    } else if (warp == 1) {
+        // ================= activation loader =================
         if (!gather) {
             // contiguous routed rows: TMA tile loads, 16 rows x 64 K per box, 128B-swizzled
-            if (warp == 1 && lane == 0) {
+            if (lane == 0) {
                 uint32_t stage_ctr = 0;
                 for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
                     const Tile tl = tile_at(p, sch, t, nnt);
@@ -321,34 +325,33 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
             }
         } else {
             // gathered rows (row_token): 16-byte cp.async per (row, chunk), written in the
-            // 128B-swizzled layout; each thread completes its copies of a stage, makes them
+            // 128B-swizzled layout; each lane completes its copies of a stage, makes them
             // visible to the tensor core (proxy fence) and arrives, two stages behind issue
-            const int l = threadIdx.x - 32;              // 0..63
-            const int c = l & 7;                         // 16-byte chunk of the 128-byte row
-            const int rb = l >> 3;                       // rows rb, rb + 8, ...: row & 7 == rb
-            const uint32_t swz = (uint32_t)((c ^ rb) << 4);
-            constexpr int kRowsPer = kBNMax / 8;
+            const int c = lane & 7;                      // 16-byte chunk of the 128-byte row
+            const int rb = lane >> 3;                    // rows rb, rb + 4, ...
+            constexpr int kRowsPer = kBNMax / 4;
+            int* s_rows = reinterpret_cast<int*>(smem + kOffRows);
             uint32_t stage_ctr = 0;
             int npend = 0;
             uint32_t pend0 = 0, pend1 = 0, pend2 = 0;
             for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
                 const Tile tl = tile_at(p, sch, t, nnt);
-                int tok[kRowsPer];
-#pragma unroll
-                for (int j = 0; j < kRowsPer; ++j) {
-                    const int row = rb + 8 * j;
-                    tok[j] = (row < tl.cnt) ? __ldg(p.row_token + tl.r0 + row) : -1;
-                }
+                __syncwarp();
+                for (int row = lane; row < kBNMax; row += 32)
+                    s_rows[row] = (row < tl.cnt) ? __ldg(p.row_token + tl.r0 + row) : -1;
+                __syncwarp();
                 for (int s = 0; s < nst; ++s, ++stage_ctr) {
                     const uint32_t slot = stage_ctr % kStages, ph = ((stage_ctr / kStages) & 1u) ^ 1u;
                     if (!mbar_wait_bounded(bar_empty + 8 * slot, ph, abort_flag, err, 8u)) goto load_done;
-                    const uint32_t dst = sbase + kOffB + slot * kBStageBytes + swz;
+                    const uint32_t dst = sbase + kOffB + slot * kBStageBytes;
                     const int kx = s * kKStage + c * 8;
                     if (kx < p.K) {
-#pragma unroll
+#pragma unroll 4
                         for (int j = 0; j < kRowsPer; ++j) {
-                            if (tok[j] >= 0)
-                                cp_async16(dst + (rb + 8 * j) * 128, p.x + (int64_t)tok[j] * p.K + kx);
+                            const int row = rb + 4 * j;
+                            const int tk = s_rows[row];
+                            if (tk >= 0)
+                                cp_async16(dst + row * 128 + ((c ^ (row & 7)) << 4), p.x + (int64_t)tk * p.K + kx);
                         }
                     }
                     cp_async_commit();
@@ -374,7 +377,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
     load_done:
         cp_async_wait<0>();
         __syncwarp();
-    } else if (warp == 3) {
+    } else if (warp == 2) {
         // ================= packed-weight loader (TMA) =================
         if (lane == 0) {
             uint32_t ctr = 0;
@@ -392,38 +395,41 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
         }
     wload_done:
         __syncwarp();
-    } else if (warp >= 4 && warp < 8) {
-        // ================= decoders: one weight row per thread =================
-        const int i = threadIdx.x - 128;                   // tile row
+    } else if (warp >= kDecWarp0 && warp < kDecWarp0 + kDecWarps) {
+        // ================= decoders: half a weight row per thread =================
+        const int d = warp - kDecWarp0;
+        const int i = (d & 3) * 32 + lane;                 // tile row
+        const int hf = d >> 2;                             // 16-byte chunks 4hf .. 4hf+3 of the row
         uint32_t stage_ctr = 0;
         for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
             for (int s = 0; s < nst; ++s, ++stage_ctr) {
-                // packed bytes of row i for this stage, from the weight ring
+                // packed bytes of this half row for this stage, from the weight ring
                 const uint32_t wslot = stage_ctr % kWStages, wph = (stage_ctr / kWStages) & 1u;
                 if (!mbar_wait_bounded(bar_wfull + 8 * wslot, wph, abort_flag, err, 32u)) goto dec_done;
-                const uint4* wsrc = reinterpret_cast<const uint4*>(smem + kOffW + wslot * kWStageBytes + i * 32);
-                const uint4 c0 = wsrc[0], c1 = wsrc[1];
+                const uint4 cw = *reinterpret_cast<const uint4*>(smem + kOffW + wslot * kWStageBytes + i * 32 + hf * 16);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_wempty + 8 * wslot);
-                const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                uint32_t o[8][4];
+                const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+                uint32_t o[4][4];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) decode_word<FMT>(words[c], p.lut, o[c]);
+                for (int c = 0; c < 4; ++c) decode_word<FMT>(words[c], p.lut, o[c]);
                 const uint32_t slot = stage_ctr % kStages, ph = ((stage_ctr / kStages) & 1u) ^ 1u;
                 if (!mbar_wait_bounded(bar_empty + 8 * slot, ph, abort_flag, err, 64u)) goto dec_done;
                 uint8_t* arow = smem + kOffA + slot * kAStageBytes + i * 128;
 #pragma unroll
-                for (int c = 0; c < 8; ++c)          // 16-byte chunk c: K elements 8c .. 8c+7
-                    *reinterpret_cast<uint4*>(arow + ((c ^ (i & 7)) << 4)) = make_uint4(o[c][0], o[c][1], o[c][2], o[c][3]);
+                for (int c = 0; c < 4; ++c) {         // 16-byte chunk cc: K elements 8cc .. 8cc+7
+                    const int cc = 4 * hf + c;
+                    *reinterpret_cast<uint4*>(arow + ((cc ^ (i & 7)) << 4)) = make_uint4(o[c][0], o[c][1], o[c][2], o[c][3]);
+                }
                 fence_proxy_async();
                 mbar_arrive(bar_afull + 8 * slot);
             }
         }
     dec_done:;
-    } else if (warp >= 8) {
+    } else if (warp >= kEpiWarp0) {
         // ================= rescale epilogue =================
         const int q4 = warp & 3;                      // tensor-memory lane quadrant
-        const int half = (warp - 8) >> 2;             // which 16-column chunks: half, half+2, ...
+        const int half = (warp - kEpiWarp0) >> 2;     // which 16-column chunks: half, half+2, ...
         const int i = q4 * 32 + lane;                 // tile row = tensor-memory lane
         const int nsbk = p.K / SB;                    // scale blocks per row
         uint32_t acc_ctr = 0;
@@ -438,33 +444,37 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
             for (int j = 0; j < kBNMax / 32; ++j)
 #pragma unroll
                 for (int c = 0; c < 16; ++c) acc[j][c] = 0.f;
-            float scale_next = load_scale<FMT>(p.scales, srow);
-            for (int b = 0; b < nsbk; ++b, ++acc_ctr) {
-                const float sc = scale_next;
-                if (b + 1 < nsbk) scale_next = load_scale<FMT>(p.scales, srow + b + 1);
-                const uint32_t buf = acc_ctr % kAccBufs, ph = (acc_ctr / kAccBufs) & 1u;
-                if (!mbar_wait_bounded(bar_accfull + 8 * buf, ph, abort_flag, err, 128u)) goto epi_done;
-                tc_fence_after();
-                const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16) + buf * kBNMax;
+            float sring[kScaleAhead];                 // scales of blocks b .. b+kScaleAhead-1
 #pragma unroll
-                for (int j = 0; j < kBNMax / 32; j += 2) {
-                    const int c0 = half + 2 * j, c1 = half + 2 * (j + 1);
-                    uint32_t v0[16], v1[16];
-                    if (c0 < nck) tmem_ld16(taddr + c0 * 16, v0);
-                    if (c1 < nck) tmem_ld16(taddr + c1 * 16, v1);
-                    tmem_wait_ld();
-                    if (c0 < nck) {
+            for (int u = 0; u < kScaleAhead; ++u) sring[u] = (u < nsbk) ? load_scale<FMT>(p.scales, srow + u) : 0.f;
+            for (int b0 = 0; b0 < nsbk; b0 += kScaleAhead) {
 #pragma unroll
-                        for (int c = 0; c < 16; c += 2) ffma2(acc[j][c], acc[j][c + 1], v0[c], v0[c + 1], sc);
-                    }
-                    if (c1 < nck) {
+                for (int u = 0; u < kScaleAhead; ++u) {
+                    const int b = b0 + u;
+                    if (b < nsbk) {
+                        const float sc = sring[u];
+                        if (b + kScaleAhead < nsbk) sring[u] = load_scale<FMT>(p.scales, srow + b + kScaleAhead);
+                        const uint32_t buf = acc_ctr % kAccBufs, ph = (acc_ctr / kAccBufs) & 1u;
+                        ++acc_ctr;
+                        if (!mbar_wait_bounded(bar_accfull + 8 * buf, ph, abort_flag, err, 128u)) goto epi_done;
+                        tc_fence_after();
+                        const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16) + buf * kBNMax;
 #pragma unroll
-                        for (int c = 0; c < 16; c += 2) ffma2(acc[j + 1][c], acc[j + 1][c + 1], v1[c], v1[c + 1], sc);
+                        for (int j = 0; j < kBNMax / 32; ++j) {
+                            const int c0 = half + 2 * j;
+                            if (c0 < nck) {
+                                uint32_t v[16];
+                                tmem_ld16(taddr + c0 * 16, v);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int c = 0; c < 16; c += 2) ffma2(acc[j][c], acc[j][c + 1], v[c], v[c + 1], sc);
+                            }
+                        }
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar_accempty + 8 * buf);
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_accempty + 8 * buf);
             }
             // outputs of this tile: row n, routed rows r0 .. r0+cnt-1
             if (valid) {
