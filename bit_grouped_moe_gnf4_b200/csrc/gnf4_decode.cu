@@ -40,10 +40,9 @@ __device__ unsigned g_decode_error;
 
 namespace db {
 
-constexpr int kGroups = 4;                         // item groups per CTA
+constexpr int kMaxGroups = 4;                      // item groups per CTA (fewer when shared memory is short)
 constexpr int kGroupWarps = 4;                     // consumer warps per group (split of each chunk)
-constexpr int kConsumers = kGroups * kGroupWarps;  // 16
-constexpr int kThreads = (kConsumers + 1) * 32;    // + one producer warp
+constexpr int kMaxThreads = (kMaxGroups * kGroupWarps + 1) * 32;   // + one producer warp
 constexpr int kMaxExperts = 2048;
 constexpr int kChunkK = 512;                       // K per stage
 constexpr int kLutBytes = 256 * 256;               // byte value b, lane l -> offset b*256 + l*4
@@ -54,7 +53,9 @@ struct Plan {
     int row_stride;   // bytes per weight row in a stage (chunk bytes + 16 of padding)
     int stage_bytes;  // 16 rows
     int scale_bytes;  // slot for one item's scales (16 rows x all blocks, contiguous in memory), rounded to 128
-    int nstages;      // stages (and item scale slots) per group ring
+    int nstages;      // stages per group ring
+    int nslots;       // item scale slots per group
+    int ngroups;      // item groups in the CTA (consumer warps = 4 * ngroups, then the producer warp)
 };
 
 struct Pos {
@@ -64,7 +65,7 @@ struct Pos {
 }  // namespace db
 
 template <int FMT, int GMAX>
-__global__ void __launch_bounds__(db::kThreads, 1) decode_band_kernel(const GroupedArgs p, const db::Plan plan) {
+__global__ void __launch_bounds__(db::kMaxThreads, 1) decode_band_kernel(const GroupedArgs p, const db::Plan plan) {
     using namespace db;
     constexpr int SB = (FMT == FMT_NF4) ? 64 : 32;   // K elements per scale block
     constexpr int STEPS = SB / 16;                   // k16 MMA steps per block
@@ -72,13 +73,17 @@ __global__ void __launch_bounds__(db::kThreads, 1) decode_band_kernel(const Grou
     constexpr int XW = SB / 8;                       // bf16x2 words of x per lane per block
     constexpr int BPW = (kChunkK / SB) / kGroupWarps;  // blocks per warp per full chunk (2 or 4)
 
+    const int kGroups = plan.ngroups;
+    const int kConsumers = kGroups * kGroupWarps;
+    const int kThreads = (kConsumers + 1) * 32;
+
     extern __shared__ __align__(1024) uint8_t smem[];
     // [lut][rings: groups x stages x stage_bytes][scale slots: groups x stages x scale_bytes]
     // [red][barriers][abort, counts][active experts: id, first row, rows]
     uint8_t* lut = smem;                                            // [256][64] words
     uint8_t* rings = smem + kLutBytes;
     uint8_t* sslots = rings + kGroups * plan.nstages * plan.stage_bytes;
-    float4* red = reinterpret_cast<float4*>(sslots + kGroups * plan.nstages * plan.scale_bytes);
+    float4* red = reinterpret_cast<float4*>(sslots + kGroups * plan.nslots * plan.scale_bytes);
     uint64_t* bars = reinterpret_cast<uint64_t*>(red + kConsumers * GMAX * 32);   // full[g][s], empty[g][s]
     int* tailw = reinterpret_cast<int*>(bars + 2 * kGroups * plan.nstages);
     volatile int* abort_flag = tailw;
@@ -151,7 +156,7 @@ __global__ void __launch_bounds__(db::kThreads, 1) decode_band_kernel(const Grou
             uint64_t* full = bars + q * ns;
             uint64_t* empty = bars + kGroups * ns + q * ns;
             uint8_t* ring = rings + q * ns * plan.stage_bytes;
-            uint8_t* sring = sslots + q * ns * plan.scale_bytes;
+            uint8_t* sring = sslots + q * plan.nslots * plan.scale_bytes;
             const int ssz = FMT == FMT_NF4 ? 4 : 1;
             uint32_t ctr = 0, jitem = 0;
             for (Pos ps{i0 + q, 0, 0}; ps.item < i1; ps = advance(ps), ++ctr) {
@@ -171,7 +176,7 @@ __global__ void __launch_bounds__(db::kThreads, 1) decode_band_kernel(const Grou
                                           ((int64_t)e * p.N + n0) * nbk * ssz;
                     asm volatile(
                         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                        ::"r"(smem_addr(sring + (jitem % ns) * plan.scale_bytes)), "l"(ssrc),
+                        ::"r"(smem_addr(sring + (jitem % plan.nslots) * plan.scale_bytes)), "l"(ssrc),
                           "r"(sbytes), "r"(fb) : "memory");
                     ++jitem;
                 }
@@ -192,7 +197,7 @@ __global__ void __launch_bounds__(db::kThreads, 1) decode_band_kernel(const Grou
         uint64_t* full = bars + q * ns;
         uint64_t* empty = bars + kGroups * ns + q * ns;
         const uint8_t* ring = rings + q * ns * plan.stage_bytes;
-        const uint8_t* sring = sslots + q * ns * plan.scale_bytes;
+        const uint8_t* sring = sslots + q * plan.nslots * plan.scale_bytes;
         float4* gred = red + q * kGroupWarps * GMAX * 32;
         const uint32_t lane_sel = (uint32_t)lane * 4u;   // lut offset of this lane's copy
         uint32_t ctr = 0, jitem = 0;
@@ -253,7 +258,7 @@ __global__ void __launch_bounds__(db::kThreads, 1) decode_band_kernel(const Grou
             ++ctr;
             if (!mbar_wait_bounded(smem_addr(full + slot), ph, abort_flag, &g_decode_error, 2u)) break;
             const uint8_t* st = ring + slot * plan.stage_bytes;
-            const uint8_t* ss = sring + (jitem % ns) * plan.scale_bytes;
+            const uint8_t* ss = sring + (jitem % plan.nslots) * plan.scale_bytes;
             const int bg0 = cur.kc * (plan.kch / SB);     // first scale block of the chunk
 #pragma unroll
             for (int c = 0; c < BPW; ++c) {
@@ -366,15 +371,26 @@ static cudaError_t launch_db(const GroupedArgs& a, cudaStream_t s) {
     plan.stage_bytes = ((16 * plan.row_stride + 127) / 128) * 128;
     const int SB = (FMT == FMT_NF4) ? 64 : 32;
     plan.scale_bytes = ((16 * (a.K / SB) * (FMT == FMT_NF4 ? 4 : 1) + 127) / 128) * 128;
-    const int red_bytes = kConsumers * GMAX * 32 * (int)sizeof(float4);
+    // largest group count whose rings fit in shared memory
     const int tables = 32 + 16 * a.E;
-    const int fixed = kLutBytes + red_bytes + 2 * kGroups * 8 * 8 + tables;
-    int nst = (226 * 1024 - fixed) / (kGroups * (plan.stage_bytes + plan.scale_bytes));
-    if (nst > 8) nst = 8;
-    if (nst < 2) return cudaErrorInvalidValue;
-    plan.nstages = nst;
-    const int smem = kLutBytes + kGroups * nst * (plan.stage_bytes + plan.scale_bytes) + red_bytes +
-                     2 * kGroups * nst * 8 + tables;
+    int smem = 0;
+    plan.ngroups = 0;
+    for (int ng = kMaxGroups; ng >= 1 && plan.ngroups == 0; ng >>= 1) {
+        const int red_bytes = ng * kGroupWarps * GMAX * 32 * (int)sizeof(float4);
+        const int fixed = kLutBytes + red_bytes + 2 * ng * 8 * 8 + tables;
+        for (int nst = 8; nst >= 3; --nst) {
+            const int nsl = (nst - 1 + plan.nch - 1) / plan.nch + 1;   // items a group can have in flight
+            const int need = fixed + ng * (nst * plan.stage_bytes + nsl * plan.scale_bytes);
+            if (need <= 226 * 1024) {
+                plan.ngroups = ng;
+                plan.nstages = nst;
+                plan.nslots = nsl;
+                smem = need;
+                break;
+            }
+        }
+    }
+    if (plan.ngroups == 0) return cudaErrorInvalidValue;
     static int smem_set = 0;                 // largest dynamic shared memory opted in so far
     if (smem > smem_set) {
         cudaError_t e = cudaFuncSetAttribute(decode_band_kernel<FMT, GMAX>,
@@ -387,7 +403,7 @@ static cudaError_t launch_db(const GroupedArgs& a, cudaStream_t s) {
     int64_t grid = device_sm_count();
     if (items_max < grid) grid = items_max;
     if (grid < 1) return cudaSuccess;
-    decode_band_kernel<FMT, GMAX><<<(unsigned)grid, kThreads, smem, s>>>(a, plan);
+    decode_band_kernel<FMT, GMAX><<<(unsigned)grid, (plan.ngroups * kGroupWarps + 1) * 32, smem, s>>>(a, plan);
     return cudaGetLastError();
 }
 

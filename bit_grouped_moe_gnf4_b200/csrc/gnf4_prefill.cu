@@ -10,9 +10,9 @@
 // the tiles of every expert in the band, computed on the device from the
 // expert offsets. Roles (19 warps):
 //   warp 0      tensor-memory owner and MMA issuer (one thread)
-//   warp 1      activation loader: TMA tile loads of contiguous rows (one
-//               thread), or 16-byte cp.async of the rows named by row_token,
-//               both into the 128B-swizzled K-major layout
+//   warp 1      activation loader: TMA tile loads of contiguous rows, or TMA
+//               gather4 loads of the rows named by row_token, both into the
+//               128B-swizzled K-major layout
 //   warp 2      packed-weight loader: TMA loads of the tile's 128 rows x 32
 //               bytes per 64 K into a deep ring of its own
 //   warps 3-10  decoders: half a weight row per thread; nibbles -> bf16 by
@@ -125,6 +125,16 @@ __device__ __forceinline__ void tma_tile_2d(uint32_t dst, const CUtensorMap* map
         " [%0], [%1, {%2, %3}], [%4];"
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
 }
+// four rows (y0..y3) x one box of columns starting at x, written as four consecutive
+// 128-byte rows at dst (the tensor map's box is one row high)
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, int y0, int y1, int y2,
+                                            int y3, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar)
+        : "memory");
+}
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
@@ -183,9 +193,10 @@ __device__ __forceinline__ Tile tile_at(const GroupedArgs& p, const Sched& s, in
 }  // namespace pf
 
 template <int FMT>
-__global__ void __launch_bounds__(pf::kThreads, 1)
+__global__ void __maxnreg__(104)
 prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xmap,
-                    const __grid_constant__ CUtensorMap wmap, const int gather) {
+                    const __grid_constant__ CUtensorMap gmap, const __grid_constant__ CUtensorMap wmap,
+                    const int gather) {
     using namespace pf;
     constexpr int SB = (FMT == FMT_NF4) ? 64 : 32;      // scale block
     constexpr int SBPS = kKStage / SB;                  // scale blocks per stage (1 or 2)
@@ -247,7 +258,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
     } else if (warp == 2 && lane == 0) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(bar_afull + 8 * i, 32 * kDecWarps);
-            mbar_init(bar_bfull + 8 * i, gather ? 32 : 1);
+            mbar_init(bar_bfull + 8 * i, 1);
             mbar_init(bar_empty + 8 * i, 1);
         }
         for (int i = 0; i < kWStages; ++i) {
@@ -305,77 +316,41 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
     mma_done:
         __syncwarp();
     } else if (warp == 1) {
-        // ================= activation loader =================
-        if (!gather) {
-            // contiguous routed rows: TMA tile loads, 16 rows x 64 K per box, 128B-swizzled
+        // ================= activation loader (TMA) =================
+        // contiguous routed rows: tile loads of 16 rows x 64 K; rows named by row_token:
+        // gather4 loads of 4 rows x 64 K. Both land 128B-swizzled, as the MMA reads them.
+        int* s_rows = reinterpret_cast<int*>(smem + kOffRows);
+        uint32_t stage_ctr = 0;
+        for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
+            const Tile tl = tile_at(p, sch, t, nnt);
+            if (gather) {
+                // the tile's rows; padding rows repeat the tile's first row
+                __syncwarp();
+                for (int row = lane; row < tl.bn; row += 32)
+                    s_rows[row] = __ldg(p.row_token + tl.r0 + (row < tl.cnt ? row : 0));
+                __syncwarp();
+            }
             if (lane == 0) {
-                uint32_t stage_ctr = 0;
-                for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
-                    const Tile tl = tile_at(p, sch, t, nnt);
-                    for (int s = 0; s < nst; ++s, ++stage_ctr) {
-                        const uint32_t slot = stage_ctr % kStages, ph = ((stage_ctr / kStages) & 1u) ^ 1u;
-                        if (!mbar_wait_bounded(bar_empty + 8 * slot, ph, abort_flag, err, 8u)) goto load_done;
-                        const uint32_t full = bar_bfull + 8 * slot;
-                        const uint32_t dst = sbase + kOffB + slot * kBStageBytes;
-                        mbar_arrive_tx(full, (uint32_t)tl.bn * 128u);
+                for (int s = 0; s < nst; ++s, ++stage_ctr) {
+                    const uint32_t slot = stage_ctr % kStages, ph = ((stage_ctr / kStages) & 1u) ^ 1u;
+                    if (!mbar_wait_bounded(bar_empty + 8 * slot, ph, abort_flag, err, 8u)) goto load_done;
+                    const uint32_t full = bar_bfull + 8 * slot;
+                    const uint32_t dst = sbase + kOffB + slot * kBStageBytes;
+                    mbar_arrive_tx(full, (uint32_t)tl.bn * 128u);
+                    if (gather) {
+                        for (int j = 0; j < tl.bn; j += 4)
+                            tma_gather4(dst + j * 128, &gmap, s * kKStage, s_rows[j], s_rows[j + 1], s_rows[j + 2],
+                                        s_rows[j + 3], full);
+                    } else {
                         for (int j = 0; j < tl.bn; j += 16)
                             tma_tile_2d(dst + j * 128, &xmap, s * kKStage, (int)(tl.r0 + j), full);
                     }
                 }
+            } else {
+                stage_ctr += nst;
             }
-        } else {
-            // gathered rows (row_token): 16-byte cp.async per (row, chunk), written in the
-            // 128B-swizzled layout; each lane completes its copies of a stage, makes them
-            // visible to the tensor core (proxy fence) and arrives, two stages behind issue
-            const int c = lane & 7;                      // 16-byte chunk of the 128-byte row
-            const int rb = lane >> 3;                    // rows rb, rb + 4, ...
-            constexpr int kRowsPer = kBNMax / 4;
-            int* s_rows = reinterpret_cast<int*>(smem + kOffRows);
-            uint32_t stage_ctr = 0;
-            int npend = 0;
-            uint32_t pend0 = 0, pend1 = 0, pend2 = 0;
-            for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
-                const Tile tl = tile_at(p, sch, t, nnt);
-                __syncwarp();
-                for (int row = lane; row < kBNMax; row += 32)
-                    s_rows[row] = (row < tl.cnt) ? __ldg(p.row_token + tl.r0 + row) : -1;
-                __syncwarp();
-                for (int s = 0; s < nst; ++s, ++stage_ctr) {
-                    const uint32_t slot = stage_ctr % kStages, ph = ((stage_ctr / kStages) & 1u) ^ 1u;
-                    if (!mbar_wait_bounded(bar_empty + 8 * slot, ph, abort_flag, err, 8u)) goto load_done;
-                    const uint32_t dst = sbase + kOffB + slot * kBStageBytes;
-                    const int kx = s * kKStage + c * 8;
-                    if (kx < p.K) {
-#pragma unroll 4
-                        for (int j = 0; j < kRowsPer; ++j) {
-                            const int row = rb + 4 * j;
-                            const int tk = s_rows[row];
-                            if (tk >= 0)
-                                cp_async16(dst + row * 128 + ((c ^ (row & 7)) << 4), p.x + (int64_t)tk * p.K + kx);
-                        }
-                    }
-                    cp_async_commit();
-                    if (npend == 0) pend0 = slot;
-                    else if (npend == 1) pend1 = slot;
-                    else pend2 = slot;
-                    ++npend;
-                    if (npend == 3) {
-                        cp_async_wait<2>();
-                        fence_proxy_async();
-                        mbar_arrive(bar_bfull + 8 * pend0);
-                        pend0 = pend1;
-                        pend1 = pend2;
-                        npend = 2;
-                    }
-                }
-            }
-            cp_async_wait<0>();
-            fence_proxy_async();
-            if (npend >= 1) mbar_arrive(bar_bfull + 8 * pend0);
-            if (npend >= 2) mbar_arrive(bar_bfull + 8 * pend1);
         }
     load_done:
-        cp_async_wait<0>();
         __syncwarp();
     } else if (warp == 2) {
         // ================= packed-weight loader (TMA) =================
@@ -547,6 +522,18 @@ static cudaError_t launch_pf(const GroupedArgs& a, int64_t T_in, cudaStream_t s)
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     }
+    CUtensorMap gmap;
+    {
+        // activations for gather4: the same tensor, boxes of 64 K x 1 row, 128B swizzle
+        cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)T_in};
+        cuuint64_t strides[1] = {(cuuint64_t)a.K * 2};
+        cuuint32_t box[2] = {64, 1};
+        cuuint32_t estr[2] = {1, 1};
+        CUresult r = enc(&gmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.x), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    }
     {
         // packed weights: bytes [E*N, K/2], boxes of 32 bytes x 128 rows, no swizzle
         cuuint64_t dims[2] = {(cuuint64_t)(a.K / 2), (cuuint64_t)a.E * (cuuint64_t)a.N};
@@ -559,7 +546,7 @@ static cudaError_t launch_pf(const GroupedArgs& a, int64_t T_in, cudaStream_t s)
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     }
     const int grid = device_sm_count();
-    prefill_band_kernel<FMT><<<grid, pf::kThreads, pf::kSmemBytes, s>>>(a, xmap, wmap, gather);
+    prefill_band_kernel<FMT><<<grid, pf::kThreads, pf::kSmemBytes, s>>>(a, xmap, gmap, wmap, gather);
     return cudaGetLastError();
 }
 
