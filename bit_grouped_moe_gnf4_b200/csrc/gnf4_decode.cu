@@ -5,31 +5,35 @@
 // take the GEMV path).
 //
 // One persistent CTA per SM takes a contiguous run of work items; an item is
-// (active expert, 16 weight rows). The CTA's 16 consumer warps form 4 groups of
-// 4 warps; group q takes items q, q+4, ... of the run. A producer warp (one
-// lane per group) streams each item's packed rows, one K chunk of 512 at a
-// time, into the group's ring of shared-memory stages with 1-D bulk copies
-// (cp.async.bulk, completion counted on an mbarrier), several chunks ahead, so
-// HBM always has many bytes in flight per SM.
+// (active expert, ROWS = 64 weight rows; 32 when K is very large). A producer
+// thread streams each item's packed rows, one K chunk of 512 at a time, into a
+// ring of 16 KB shared-memory stages with 2-D TMA loads (boxes of 128 bytes x
+// ROWS rows, 128B-swizzled), several stages ahead; big requests are what lets
+// the copy engine keep HBM busy. The item's block scales (ROWS rows x all
+// blocks, one contiguous range) arrive with its first chunk by a 1-D bulk copy.
 //
-// The 4 warps of a group split each chunk's scale blocks. Nibble pairs are
-// decoded by a table in shared memory that maps each packed byte to its two
-// bf16 values (one bf16x2 word), replicated per lane so that 32 lookups never
-// conflict; a byte permute forms the lookup address. The products run on
-// warp-level bf16 MMAs with the 16 weight rows as the M side and up to 8 routed
-// rows per MMA as the N side. Every MMA chain covers exactly one scale block
-// (64 K for NF4, 32 K for MXFP4), so the block sum leaves the tensor core in
-// fp32 and is scaled and accumulated in fp32 outside it. After the last chunk
-// the group's 4 partial sums are added in a fixed order through shared memory
-// (deterministic), weighted, rounded to bf16 and stored at the destination rows.
+// 16 consumer warps split an item as (ROWS/16 row tiles) x (16/(ROWS/16)) K
+// splits of every chunk. Nibble pairs are decoded by a table in shared memory
+// that maps each packed byte to its two bf16 values (one bf16x2 word),
+// replicated per lane so that 32 lookups never conflict; a byte permute forms
+// the lookup address. The products run on warp-level bf16 MMAs with 16 weight
+// rows as the M side and up to 8 routed rows per MMA as the N side. Every MMA
+// chain covers exactly one scale block (64 K for NF4, 32 K for MXFP4), so the
+// block sum leaves the tensor core in fp32 and is scaled and accumulated in
+// fp32 outside it. At the end of an item the K splits' partial sums are added
+// in a fixed order through shared memory (deterministic), weighted, rounded to
+// bf16 and stored at the destination rows.
 //
 // MMA k-slot mapping: in m16n8k16, lane (g, t) supplies k-slots 2t, 2t+1,
 // 2t+8, 2t+9 of both operands. They are mapped to the four consecutive K
 // positions base + (SB/4)*t + 4*s + {0,1,2,3} of step s, the same for A and
 // B, so each lane reads contiguous bytes of the packed rows and of x.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
 #include <climits>
 #include <cstdint>
-#include <cuda_runtime.h>
 
 #include "gnf4_common.cuh"
 #include "gnf4_kernels.h"
@@ -40,52 +44,53 @@ __device__ unsigned g_decode_error;
 
 namespace db {
 
-constexpr int kMaxGroups = 4;                      // item groups per CTA (fewer when shared memory is short)
-constexpr int kGroupWarps = 4;                     // consumer warps per group (split of each chunk)
-constexpr int kMaxThreads = (kMaxGroups * kGroupWarps + 1) * 32;   // + one producer warp
-constexpr int kMaxExperts = 2048;
-constexpr int kChunkK = 512;                       // K per stage
+constexpr int kConsumers = 16;                     // consumer warps
+constexpr int kThreads = (kConsumers + 1) * 32;    // + one producer warp
+constexpr int kChunkK = 512;                       // K per stage: 256 packed bytes per row
+constexpr int kBoxBytes = 128;                     // TMA box width (one 128B swizzle row)
 constexpr int kLutBytes = 256 * 256;               // byte value b, lane l -> offset b*256 + l*4
 
 struct Plan {
-    int kch;          // K elements per stage
+    int rows;         // weight rows per item (64 or 32)
     int nch;          // stages per item pass
-    int row_stride;   // bytes per weight row in a stage (chunk bytes + 16 of padding)
-    int stage_bytes;  // 16 rows
-    int scale_bytes;  // slot for one item's scales (16 rows x all blocks, contiguous in memory), rounded to 128
-    int nstages;      // stages per group ring
-    int nslots;       // item scale slots per group
-    int ngroups;      // item groups in the CTA (consumer warps = 4 * ngroups, then the producer warp)
+    int stage_bytes;  // rows x 256 bytes
+    int scale_bytes;  // slot for one item's scales (rows x all blocks), rounded to 128
+    int nstages;      // ring stages
+    int nslots;       // item scale slots
 };
 
 struct Pos {
     int item, pass, kc;
 };
 
+__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+
 }  // namespace db
 
 template <int FMT, int GMAX>
-__global__ void __launch_bounds__(db::kMaxThreads, 1) decode_band_kernel(const GroupedArgs p, const db::Plan plan) {
+__global__ void __launch_bounds__(db::kThreads, 1)
+decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_constant__ CUtensorMap wmap) {
     using namespace db;
     constexpr int SB = (FMT == FMT_NF4) ? 64 : 32;   // K elements per scale block
     constexpr int STEPS = SB / 16;                   // k16 MMA steps per block
     constexpr int BPL = SB / 8;                      // packed bytes per lane per row per block (8 or 4)
     constexpr int XW = SB / 8;                       // bf16x2 words of x per lane per block
-    constexpr int BPW = (kChunkK / SB) / kGroupWarps;  // blocks per warp per full chunk (2 or 4)
+    constexpr int BPW = 4;                           // most blocks a warp takes from one chunk
 
-    const int kGroups = plan.ngroups;
-    const int kConsumers = kGroups * kGroupWarps;
-    const int kThreads = (kConsumers + 1) * 32;
-
-    extern __shared__ __align__(1024) uint8_t smem[];
-    // [lut][rings: groups x stages x stage_bytes][scale slots: groups x stages x scale_bytes]
-    // [red][barriers][abort, counts][active experts: id, first row, rows]
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // [lut][ring: stages x stage_bytes][scale slots][red][barriers][abort, count][experts]
     uint8_t* lut = smem;                                            // [256][64] words
-    uint8_t* rings = smem + kLutBytes;
-    uint8_t* sslots = rings + kGroups * plan.nstages * plan.stage_bytes;
-    float4* red = reinterpret_cast<float4*>(sslots + kGroups * plan.nslots * plan.scale_bytes);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(red + kConsumers * GMAX * 32);   // full[g][s], empty[g][s]
-    int* tailw = reinterpret_cast<int*>(bars + 2 * kGroups * plan.nstages);
+    uint8_t* ring = smem + kLutBytes;                               // 1024-aligned stages
+    uint8_t* sslots = ring + plan.nstages * plan.stage_bytes;
+    float4* red = reinterpret_cast<float4*>(sslots + plan.nslots * plan.scale_bytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(red + kConsumers * GMAX * 32);   // full[s], empty[s]
+    int* tailw = reinterpret_cast<int*>(bars + 2 * plan.nstages);
     volatile int* abort_flag = tailw;
     int* s_nact = tailw + 4;
     int64_t* s_r0 = reinterpret_cast<int64_t*>(tailw + 8);         // [E] first routed row
@@ -94,6 +99,7 @@ __global__ void __launch_bounds__(db::kMaxThreads, 1) decode_band_kernel(const G
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ns = plan.nstages;
+    const int ROWS = plan.rows;
 
     // byte -> bf16x2 table, one copy per lane
     for (int i = threadIdx.x; i < 256 * 32; i += kThreads) {
@@ -121,86 +127,76 @@ __global__ void __launch_bounds__(db::kMaxThreads, 1) decode_band_kernel(const G
         }
         if (lane == 0) s_nact[0] = count;
     } else if (warp == kConsumers && lane == 0) {
-        for (int i = 0; i < kGroups * ns; ++i) {
-            mbar_init(smem_addr(bars + i), 1);                                 // full: producer + tx bytes
-            mbar_init(smem_addr(bars + kGroups * ns + i), kGroupWarps);        // empty: the group's warps
+        for (int i = 0; i < ns; ++i) {
+            mbar_init(smem_addr(bars + i), 1);                 // full: producer + tx bytes
+            mbar_init(smem_addr(bars + ns + i), kConsumers);   // empty: every consumer warp
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
 
-    const int nt = p.N >> 4;
-    const int total = s_nact[0] * nt;
+    const int nit = (p.N + ROWS - 1) / ROWS;           // items per expert
+    const int total = s_nact[0] * nit;
     const int i0 = (int)((int64_t)blockIdx.x * total / gridDim.x);
     const int i1 = (int)((int64_t)(blockIdx.x + 1) * total / gridDim.x);
-    const int64_t rowbytes = p.K >> 1;
-    const int nbk = p.K / SB;                        // scale blocks per weight row
+    const int nbk = p.K / SB;                          // scale blocks per weight row
+    const int ssz = FMT == FMT_NF4 ? 4 : 1;
 
     auto advance = [&](Pos q) -> Pos {
         if (++q.kc == plan.nch) {
             q.kc = 0;
-            const int m = s_cnt[q.item / nt];
+            const int m = s_cnt[q.item / nit];
             if (++q.pass == (m + 8 * GMAX - 1) / (8 * GMAX)) {
                 q.pass = 0;
-                q.item += kGroups;
+                ++q.item;
             }
         }
         return q;
     };
 
     if (warp == kConsumers) {
-        // ================= producer: lane q feeds group q's ring =================
-        if (lane < kGroups) {
-            const int q = lane;
-            uint64_t* full = bars + q * ns;
-            uint64_t* empty = bars + kGroups * ns + q * ns;
-            uint8_t* ring = rings + q * ns * plan.stage_bytes;
-            uint8_t* sring = sslots + q * plan.nslots * plan.scale_bytes;
-            const int ssz = FMT == FMT_NF4 ? 4 : 1;
+        // ================= producer (one thread) =================
+        if (lane == 0) {
             uint32_t ctr = 0, jitem = 0;
-            for (Pos ps{i0 + q, 0, 0}; ps.item < i1; ps = advance(ps), ++ctr) {
+            for (Pos ps{i0, 0, 0}; ps.item < i1; ps = advance(ps), ++ctr) {
                 const uint32_t slot = ctr % ns, ph = ((ctr / ns) & 1u) ^ 1u;
-                if (!mbar_wait_bounded(smem_addr(empty + slot), ph, abort_flag, &g_decode_error, 1u)) break;
-                const int e = s_active[ps.item / nt];
-                const int n0 = (ps.item % nt) << 4;
-                const int kb = ps.kc * plan.kch;
-                const uint32_t bytes = (uint32_t)(min(plan.kch, p.K - kb) >> 1);
-                const uint32_t fb = smem_addr(full + slot);
+                if (!mbar_wait_bounded(smem_addr(bars + ns + slot), ph, abort_flag, &g_decode_error, 1u)) break;
+                const int a = ps.item / nit;
+                const int e = s_active[a];
+                const int n0 = (ps.item % nit) * ROWS;
+                const int xb = ps.kc * (kChunkK / 2);                 // first packed byte of the chunk
+                const int nbox = (p.K / 2 - xb) > kBoxBytes ? 2 : 1;  // the last chunk may be half
+                const uint32_t fb = smem_addr(bars + slot);
                 const bool first = ps.kc == 0 && ps.pass == 0;
-                const uint32_t sbytes = (uint32_t)(16 * nbk * ssz);      // exact, a multiple of 16
-                mbar_arrive_tx(fb, 16u * bytes + (first ? sbytes : 0u));
+                const int vrows = min(ROWS, p.N - n0);
+                const uint32_t sbytes = (uint32_t)(vrows * nbk * ssz);   // a multiple of 16
+                mbar_arrive_tx(fb, (uint32_t)(nbox * kBoxBytes * ROWS) + (first ? sbytes : 0u));
+                const uint32_t dst = smem_addr(ring + slot * plan.stage_bytes);
+                for (int bx = 0; bx < nbox; ++bx)
+                    tma_2d(dst + bx * kBoxBytes * ROWS, &wmap, xb + bx * kBoxBytes, e * p.N + n0, fb);
                 if (first) {
-                    // the item's scales: 16 rows x all blocks, one contiguous range
+                    // the item's scales: its rows x all blocks, one contiguous range
                     const uint8_t* ssrc = reinterpret_cast<const uint8_t*>(p.scales) +
                                           ((int64_t)e * p.N + n0) * nbk * ssz;
                     asm volatile(
                         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                        ::"r"(smem_addr(sring + (jitem % plan.nslots) * plan.scale_bytes)), "l"(ssrc),
+                        ::"r"(smem_addr(sslots + (jitem % plan.nslots) * plan.scale_bytes)), "l"(ssrc),
                           "r"(sbytes), "r"(fb) : "memory");
                     ++jitem;
                 }
-                const uint8_t* src = p.W + ((int64_t)e * p.N + n0) * rowbytes + (kb >> 1);
-                const uint32_t dst = smem_addr(ring + slot * plan.stage_bytes);
-                for (int r = 0; r < 16; ++r)
-                    asm volatile(
-                        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                        ::"r"(dst + r * plan.row_stride), "l"(src + r * rowbytes), "r"(bytes), "r"(fb)
-                        : "memory");
             }
         }
         __syncwarp();
     } else {
         // ================= consumers =================
-        const int q = warp / kGroupWarps, gw = warp % kGroupWarps;
+        const int nrt = ROWS / 16, nks = kConsumers / nrt;
+        const int rt = warp % nrt, ks = warp / nrt;     // row tile, K split
         const int g = lane >> 2, t = lane & 3;
-        uint64_t* full = bars + q * ns;
-        uint64_t* empty = bars + kGroups * ns + q * ns;
-        const uint8_t* ring = rings + q * ns * plan.stage_bytes;
-        const uint8_t* sring = sslots + q * plan.nslots * plan.scale_bytes;
-        float4* gred = red + q * kGroupWarps * GMAX * 32;
-        const uint32_t lane_sel = (uint32_t)lane * 4u;   // lut offset of this lane's copy
+        const int ra = rt * 16 + g, rb = ra + 8;        // the two item rows of this lane
+        const uint32_t lane_sel = (uint32_t)lane * 4u;  // lut offset of this lane's copy
         uint32_t ctr = 0, jitem = 0;
+        bool dead = false;   // set when a wait gives up: the warp then only keeps the barrier schedule
         float acc[GMAX][4];
         // activation row of this lane's token column g, per 8-row group (-1: none), for the
         // current and the next item; the next item's rows are prefetched into L1 early
@@ -209,7 +205,7 @@ __global__ void __launch_bounds__(db::kMaxThreads, 1) decode_band_kernel(const G
 #pragma unroll
             for (int j = 0; j < GMAX; ++j) tk[j] = -1;
             if (item >= i1) return;
-            const int a = item / nt;
+            const int a = item / nit;
             const int64_t r0 = s_r0[a];
             const int m = s_cnt[a];
             const int mc = pass * 8 * GMAX;
@@ -220,26 +216,25 @@ __global__ void __launch_bounds__(db::kMaxThreads, 1) decode_band_kernel(const G
             }
         };
         auto prefetch_x = [&](const int (&tk)[GMAX]) {
-            // this lane's 16-byte pieces of x for every block of this warp, all chunks
 #pragma unroll
             for (int j = 0; j < GMAX; ++j) {
                 if (tk[j] < 0) continue;
                 const uint16_t* xr = p.x + (int64_t)tk[j] * p.K + t * (SB / 4);
                 for (int kc = 0; kc < plan.nch; ++kc) {
-                    const int kb = kc * plan.kch;
-                    const int nbc = min(plan.kch, p.K - kb) / SB;
-                    for (int b = gw * nbc / kGroupWarps; b < (gw + 1) * nbc / kGroupWarps; ++b)
+                    const int kb = kc * kChunkK;
+                    const int nbc = min(kChunkK, p.K - kb) / SB;
+                    for (int b = ks * nbc / nks; b < (ks + 1) * nbc / nks; ++b)
                         asm volatile("prefetch.global.L1 [%0];" ::"l"(xr + kb + b * SB));
                 }
             }
         };
-        Pos cur{i0 + q, 0, 0};
+        Pos cur{i0, 0, 0};
         tokens_of(cur.item, 0, xtk);
         prefetch_x(xtk);
-        tokens_of(cur.item + kGroups, 0, ntk);
+        tokens_of(cur.item + 1, 0, ntk);
         while (cur.item < i1) {
-            const int a = cur.item / nt;
-            const int n0 = (cur.item % nt) << 4;
+            const int a = cur.item / nit;
+            const int n0 = (cur.item % nit) * ROWS;
             const int64_t r0 = s_r0[a];
             const int m = s_cnt[a];
             const int mc = cur.pass * 8 * GMAX;
@@ -250,32 +245,36 @@ __global__ void __launch_bounds__(db::kMaxThreads, 1) decode_band_kernel(const G
                 for (int j = 0; j < GMAX; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
                 if (cur.pass == 0) prefetch_x(ntk);       // next item's rows, one item ahead
             }
-            const int kb = cur.kc * plan.kch;
-            const int nbc = min(plan.kch, p.K - kb) / SB;
-            const int b0 = gw * nbc / kGroupWarps, b1 = (gw + 1) * nbc / kGroupWarps;
+            const int kb = cur.kc * kChunkK;
+            const int nbc = min(kChunkK, p.K - kb) / SB;
+            const int b0 = ks * nbc / nks, b1 = (ks + 1) * nbc / nks;
             const uint16_t* xbase = p.x + kb + t * (SB / 4);
             const uint32_t slot = ctr % ns, ph = (ctr / ns) & 1u;
             ++ctr;
-            if (!mbar_wait_bounded(smem_addr(full + slot), ph, abort_flag, &g_decode_error, 2u)) break;
+            if (!dead && !mbar_wait_bounded(smem_addr(bars + slot), ph, abort_flag, &g_decode_error, 2u)) dead = true;
             const uint8_t* st = ring + slot * plan.stage_bytes;
-            const uint8_t* ss = sring + (jitem % plan.nslots) * plan.scale_bytes;
-            const int bg0 = cur.kc * (plan.kch / SB);     // first scale block of the chunk
+            const uint8_t* ss = sslots + (jitem % plan.nslots) * plan.scale_bytes;
+            const int bg0 = cur.kc * (kChunkK / SB);      // first scale block of the chunk
 #pragma unroll
             for (int c = 0; c < BPW; ++c) {
-                if (b0 + c < b1) {
+                if (!dead && b0 + c < b1) {
                     const int b = b0 + c;
                     float s0, s1;
                     if constexpr (FMT == FMT_NF4) {
-                        s0 = reinterpret_cast<const float*>(ss)[g * nbk + bg0 + b];
-                        s1 = reinterpret_cast<const float*>(ss)[(g + 8) * nbk + bg0 + b];
+                        s0 = reinterpret_cast<const float*>(ss)[ra * nbk + bg0 + b];
+                        s1 = reinterpret_cast<const float*>(ss)[rb * nbk + bg0 + b];
                     } else {
-                        s0 = e8m0_to_f32(ss[g * nbk + bg0 + b]);
-                        s1 = e8m0_to_f32(ss[(g + 8) * nbk + bg0 + b]);
+                        s0 = e8m0_to_f32(ss[ra * nbk + bg0 + b]);
+                        s1 = e8m0_to_f32(ss[rb * nbk + bg0 + b]);
                     }
-                    // this lane's packed bytes of rows g and g+8
+                    // this lane's packed bytes of rows ra and rb: byte o of the row's 256-byte
+                    // chunk lives in box o/128, 16-byte piece ((o%128)/16) ^ (row%8)
+                    const int o = b * (SB / 2) + t * BPL;
+                    const uint8_t* bx = st + (o >> 7) * (kBoxBytes * ROWS);
+                    const int pc = (o & 127) >> 4, po = o & 15;
+                    const uint8_t* rp0 = bx + ra * kBoxBytes + ((pc ^ (ra & 7)) << 4) + po;
+                    const uint8_t* rp1 = bx + rb * kBoxBytes + ((pc ^ (rb & 7)) << 4) + po;
                     uint32_t w0[BPL / 4], w1[BPL / 4];
-                    const uint8_t* rp0 = st + g * plan.row_stride + b * (SB / 2) + t * BPL;
-                    const uint8_t* rp1 = rp0 + 8 * plan.row_stride;
                     if constexpr (BPL == 8) {
                         const uint2 u0 = *reinterpret_cast<const uint2*>(rp0);
                         const uint2 u1 = *reinterpret_cast<const uint2*>(rp1);
@@ -322,36 +321,37 @@ __global__ void __launch_bounds__(db::kMaxThreads, 1) decode_band_kernel(const G
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(empty + slot));
+            if (lane == 0) mbar_arrive(smem_addr(bars + ns + slot));
             if (cur.kc == plan.nch - 1) {
-                // the group's 4 partial sums, added in a fixed order, then the epilogue
+                // the K splits' partial sums, added in a fixed order, then the epilogue
 #pragma unroll
                 for (int j = 0; j < GMAX; ++j)
-                    if (j < G) gred[(gw * GMAX + j) * 32 + lane] = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
-                asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "n"(kGroupWarps * 32) : "memory");
-                const int tid = gw * 32 + lane;
-                for (int qq = tid; qq < G * 128; qq += kGroupWarps * 32) {
-                    const int j = qq >> 7, ln = (qq >> 2) & 31, i = qq & 3;
-                    float v = 0.f;
-#pragma unroll
-                    for (int w = 0; w < kGroupWarps; ++w)
-                        v += reinterpret_cast<const float*>(&gred[(w * GMAX + j) * 32 + ln])[i];
-                    const int row = mc + 8 * j + 2 * (ln & 3) + (i & 1);   // C column 2t (+1)
-                    if (row < m) {
+                    if (j < G) red[((ks * nrt + rt) * GMAX + j) * 32 + lane] =
+                                   make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+                asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");
+                const int vrows = min(ROWS, p.N - n0);
+                for (int qq = threadIdx.x; qq < nrt * G * 128; qq += kConsumers * 32) {
+                    const int i = qq & 3, ln = (qq >> 2) & 31, rest = qq >> 7;
+                    const int j = rest % G, rtt = rest / G;
+                    const int row = mc + 8 * j + 2 * (ln & 3) + (i & 1);     // C column 2t (+1)
+                    const int nr = rtt * 16 + (ln >> 2) + ((i & 2) ? 8 : 0);  // C row g (+8)
+                    if (row < m && nr < vrows) {
+                        float v = 0.f;
+                        for (int k2 = 0; k2 < nks; ++k2)
+                            v += reinterpret_cast<const float*>(&red[((k2 * nrt + rtt) * GMAX + j) * 32 + ln])[i];
                         const int64_t r = r0 + row;
                         if (p.row_weight) v *= __ldg(p.row_weight + r);
                         const int64_t dst = p.row_dest ? (int64_t)__ldg(p.row_dest + r) : r;
-                        const int n = n0 + (ln >> 2) + ((i & 2) ? 8 : 0);   // C row g (+8)
-                        p.out[dst * p.N + n] = f32_to_bf16_rne(v);
+                        p.out[dst * p.N + n0 + nr] = f32_to_bf16_rne(v);
                     }
                 }
-                asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "n"(kGroupWarps * 32) : "memory");
+                asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");
                 // next pass of this item, or the next item
                 if (nxt.item != cur.item) {
                     ++jitem;
 #pragma unroll
                     for (int j = 0; j < GMAX; ++j) xtk[j] = ntk[j];
-                    tokens_of(nxt.item + kGroups, 0, ntk);
+                    tokens_of(nxt.item + 1, 0, ntk);
                 } else {
                     tokens_of(nxt.item, nxt.pass, xtk);
                 }
@@ -361,28 +361,39 @@ __global__ void __launch_bounds__(db::kMaxThreads, 1) decode_band_kernel(const G
     }
 }
 
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn_db() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
 template <int FMT, int GMAX>
 static cudaError_t launch_db(const GroupedArgs& a, cudaStream_t s) {
     using namespace db;
-    Plan plan;
-    plan.kch = kChunkK < a.K ? kChunkK : a.K;
-    plan.nch = (a.K + plan.kch - 1) / plan.kch;
-    plan.row_stride = plan.kch / 2 + 16;
-    plan.stage_bytes = ((16 * plan.row_stride + 127) / 128) * 128;
     const int SB = (FMT == FMT_NF4) ? 64 : 32;
-    plan.scale_bytes = ((16 * (a.K / SB) * (FMT == FMT_NF4 ? 4 : 1) + 127) / 128) * 128;
-    // largest group count whose rings fit in shared memory
+    const int ssz = (FMT == FMT_NF4) ? 4 : 1;
+    Plan plan;
+    plan.nch = (a.K + kChunkK - 1) / kChunkK;
+    const int red_bytes = kConsumers * GMAX * 32 * (int)sizeof(float4);
     const int tables = 32 + 16 * a.E;
     int smem = 0;
-    plan.ngroups = 0;
-    for (int ng = kMaxGroups; ng >= 1 && plan.ngroups == 0; ng >>= 1) {
-        const int red_bytes = ng * kGroupWarps * GMAX * 32 * (int)sizeof(float4);
-        const int fixed = kLutBytes + red_bytes + 2 * ng * 8 * 8 + tables;
+    plan.rows = 0;
+    for (int rows = 64; rows >= 32 && plan.rows == 0; rows >>= 1) {
+        const int stage_bytes = rows * (kChunkK / 2);
+        const int scale_bytes = ((rows * (a.K / SB) * ssz + 127) / 128) * 128;
         for (int nst = 8; nst >= 3; --nst) {
-            const int nsl = (nst - 1 + plan.nch - 1) / plan.nch + 1;   // items a group can have in flight
-            const int need = fixed + ng * (nst * plan.stage_bytes + nsl * plan.scale_bytes);
+            const int nsl = (nst - 1 + plan.nch - 1) / plan.nch + 1;   // items in flight at once
+            const int need = 1024 + kLutBytes + nst * stage_bytes + nsl * scale_bytes + red_bytes + 2 * nst * 8 + tables;
             if (need <= 226 * 1024) {
-                plan.ngroups = ng;
+                plan.rows = rows;
+                plan.stage_bytes = stage_bytes;
+                plan.scale_bytes = scale_bytes;
                 plan.nstages = nst;
                 plan.nslots = nsl;
                 smem = need;
@@ -390,7 +401,7 @@ static cudaError_t launch_db(const GroupedArgs& a, cudaStream_t s) {
             }
         }
     }
-    if (plan.ngroups == 0) return cudaErrorInvalidValue;
+    if (plan.rows == 0) return cudaErrorInvalidValue;
     static int smem_set = 0;                 // largest dynamic shared memory opted in so far
     if (smem > smem_set) {
         cudaError_t e = cudaFuncSetAttribute(decode_band_kernel<FMT, GMAX>,
@@ -398,12 +409,24 @@ static cudaError_t launch_db(const GroupedArgs& a, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         smem_set = smem;
     }
+    auto enc = encode_fn_db();
+    if (!enc) return cudaErrorNotSupported;
+    // packed weights as bytes [E*N, K/2]: boxes of 128 bytes x rows, 128B swizzle
+    CUtensorMap wmap;
+    cuuint64_t dims[2] = {(cuuint64_t)(a.K / 2), (cuuint64_t)a.E * (cuuint64_t)a.N};
+    cuuint64_t strides[1] = {(cuuint64_t)(a.K / 2)};
+    cuuint32_t box[2] = {(cuuint32_t)kBoxBytes, (cuuint32_t)plan.rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.W), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     const int64_t groups_max = a.R < (int64_t)a.E ? a.R : (int64_t)a.E;
-    const int64_t items_max = groups_max * (a.N / 16);
+    const int64_t items_max = groups_max * ((a.N + plan.rows - 1) / plan.rows);
     int64_t grid = device_sm_count();
     if (items_max < grid) grid = items_max;
     if (grid < 1) return cudaSuccess;
-    decode_band_kernel<FMT, GMAX><<<(unsigned)grid, (plan.ngroups * kGroupWarps + 1) * 32, smem, s>>>(a, plan);
+    decode_band_kernel<FMT, GMAX><<<(unsigned)grid, kThreads, smem, s>>>(a, plan, wmap);
     return cudaGetLastError();
 }
 

@@ -193,7 +193,7 @@ __device__ __forceinline__ Tile tile_at(const GroupedArgs& p, const Sched& s, in
 }  // namespace pf
 
 template <int FMT>
-__global__ void __maxnreg__(104)
+__global__ void __maxnreg__(96)
 prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xmap,
                     const __grid_constant__ CUtensorMap gmap, const __grid_constant__ CUtensorMap wmap,
                     const int gather) {
@@ -317,7 +317,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
         __syncwarp();
     } else if (warp == 1) {
         // ================= activation loader (TMA) =================
-        // contiguous routed rows: tile loads of 16 rows x 64 K; rows named by row_token:
+        // contiguous routed rows: one tile load of 128 rows x 64 K; rows named by row_token:
         // gather4 loads of 4 rows x 64 K. Both land 128B-swizzled, as the MMA reads them.
         int* s_rows = reinterpret_cast<int*>(smem + kOffRows);
         uint32_t stage_ctr = 0;
@@ -336,14 +336,15 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
                     if (!mbar_wait_bounded(bar_empty + 8 * slot, ph, abort_flag, err, 8u)) goto load_done;
                     const uint32_t full = bar_bfull + 8 * slot;
                     const uint32_t dst = sbase + kOffB + slot * kBStageBytes;
-                    mbar_arrive_tx(full, (uint32_t)tl.bn * 128u);
                     if (gather) {
+                        mbar_arrive_tx(full, (uint32_t)tl.bn * 128u);
                         for (int j = 0; j < tl.bn; j += 4)
                             tma_gather4(dst + j * 128, &gmap, s * kKStage, s_rows[j], s_rows[j + 1], s_rows[j + 2],
                                         s_rows[j + 3], full);
                     } else {
-                        for (int j = 0; j < tl.bn; j += 16)
-                            tma_tile_2d(dst + j * 128, &xmap, s * kKStage, (int)(tl.r0 + j), full);
+                        // one box of 128 rows (rows past the tile are loaded and never used)
+                        mbar_arrive_tx(full, (uint32_t)kBStageBytes);
+                        tma_tile_2d(dst, &xmap, s * kKStage, (int)tl.r0, full);
                     }
                 }
             } else {
@@ -512,10 +513,10 @@ static cudaError_t launch_pf(const GroupedArgs& a, int64_t T_in, cudaStream_t s)
     const int gather = a.row_token != nullptr;
     CUtensorMap xmap, wmap;
     {
-        // activations: bf16 [T_in, K], boxes of 64 K x 16 rows, 128B swizzle
+        // activations: bf16 [T_in, K], boxes of 64 K x 128 rows, 128B swizzle
         cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)T_in};
         cuuint64_t strides[1] = {(cuuint64_t)a.K * 2};
-        cuuint32_t box[2] = {64, 16};
+        cuuint32_t box[2] = {64, (cuuint32_t)pf::kBNMax};
         cuuint32_t estr[2] = {1, 1};
         CUresult r = enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.x), dims, strides, box,
                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
