@@ -9,8 +9,12 @@
 // thread streams each item's packed rows, one K chunk of 512 at a time, into a
 // ring of 16 KB shared-memory stages with 2-D TMA loads (boxes of 128 bytes x
 // ROWS rows, 128B-swizzled), several stages ahead; big requests are what lets
-// the copy engine keep HBM busy. The item's block scales (ROWS rows x all
-// blocks, one contiguous range) arrive with its first chunk by a 1-D bulk copy.
+// the copy engine keep HBM busy. The same stage also carries the chunk of each
+// routed row's activations (1-D bulk copies, one per row), and the item's block
+// scales (ROWS rows x all blocks, one contiguous range) arrive with its first
+// chunk, so the consumers never wait on a global load. The CTA's routing
+// metadata (token, weight, destination of each of its routed rows) is staged in
+// shared memory once at the start.
 //
 // 16 consumer warps split an item as (ROWS/16 row tiles) x (16/(ROWS/16)) K
 // splits of every chunk. Nibble pairs are decoded by a table in shared memory
@@ -49,11 +53,14 @@ constexpr int kThreads = (kConsumers + 1) * 32;    // + one producer warp
 constexpr int kChunkK = 512;                       // K per stage: 256 packed bytes per row
 constexpr int kBoxBytes = 128;                     // TMA box width (one 128B swizzle row)
 constexpr int kLutBytes = 256 * 256;               // byte value b, lane l -> offset b*256 + l*4
+constexpr int kXStride = kChunkK * 2 + 16;         // bytes per staged activation row (padded)
+constexpr int kMaxTableRows = 1024;                // routed rows whose metadata fits the CTA's table
 
 struct Plan {
     int rows;         // weight rows per item (64 or 32)
     int nch;          // stages per item pass
-    int stage_bytes;  // rows x 256 bytes
+    int wbytes;       // packed-weight part of a stage: rows x 256 bytes
+    int stage_bytes;  // wbytes + activation rows (8*GMAX x kXStride)
     int scale_bytes;  // slot for one item's scales (rows x all blocks), rounded to 128
     int nstages;      // ring stages
     int nslots;       // item scale slots
@@ -96,6 +103,9 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
     int64_t* s_r0 = reinterpret_cast<int64_t*>(tailw + 8);         // [E] first routed row
     int* s_active = reinterpret_cast<int*>(s_r0 + p.E);            // [E] expert id
     int* s_cnt = s_active + p.E;                                   // [E] routed rows
+    int* t_tok = s_cnt + p.E;                                      // [kMaxTableRows] per routed row
+    float* t_wt = reinterpret_cast<float*>(t_tok + kMaxTableRows);
+    int* t_dst = reinterpret_cast<int*>(t_wt + kMaxTableRows);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ns = plan.nstages;
@@ -143,6 +153,27 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
     const int nbk = p.K / SB;                          // scale blocks per weight row
     const int ssz = FMT == FMT_NF4 ? 4 : 1;
 
+    // routed rows of this CTA's experts: one contiguous range [rlo, rhi)
+    int64_t rlo = 0, rhi = 0;
+    if (i0 < i1) {
+        const int a0 = i0 / nit, a1 = (i1 - 1) / nit;
+        rlo = s_r0[a0];
+        rhi = s_r0[a1] + s_cnt[a1];
+    }
+    const bool table = (rhi - rlo) <= kMaxTableRows;
+    if (table) {
+        for (int64_t r = rlo + threadIdx.x; r < rhi; r += kThreads) {
+            const int k = (int)(r - rlo);
+            t_tok[k] = p.row_token ? __ldg(p.row_token + r) : (int)r;
+            t_wt[k] = p.row_weight ? __ldg(p.row_weight + r) : 1.f;
+            t_dst[k] = p.row_dest ? __ldg(p.row_dest + r) : (int)r;
+        }
+    }
+    __syncthreads();
+    auto tok_of = [&](int64_t r) -> int {
+        return table ? t_tok[r - rlo] : (p.row_token ? __ldg(p.row_token + r) : (int)r);
+    };
+
     auto advance = [&](Pos q) -> Pos {
         if (++q.kc == plan.nch) {
             q.kc = 0;
@@ -171,10 +202,23 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
                 const bool first = ps.kc == 0 && ps.pass == 0;
                 const int vrows = min(ROWS, p.N - n0);
                 const uint32_t sbytes = (uint32_t)(vrows * nbk * ssz);   // a multiple of 16
-                mbar_arrive_tx(fb, (uint32_t)(nbox * kBoxBytes * ROWS) + (first ? sbytes : 0u));
+                // activation rows of this pass: their chunk of K, one bulk copy each
+                const int64_t r0 = s_r0[a];
+                const int mc = ps.pass * 8 * GMAX;
+                const int nx = min(8 * GMAX, s_cnt[a] - mc);
+                const int kb = ps.kc * kChunkK;
+                const uint32_t xbytes = (uint32_t)(min(kChunkK, p.K - kb) * 2);
+                mbar_arrive_tx(fb, (uint32_t)(nbox * kBoxBytes * ROWS) + (uint32_t)nx * xbytes + (first ? sbytes : 0u));
                 const uint32_t dst = smem_addr(ring + slot * plan.stage_bytes);
                 for (int bx = 0; bx < nbox; ++bx)
                     tma_2d(dst + bx * kBoxBytes * ROWS, &wmap, xb + bx * kBoxBytes, e * p.N + n0, fb);
+                for (int j = 0; j < nx; ++j) {
+                    const int tk = tok_of(r0 + mc + j);
+                    asm volatile(
+                        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                        ::"r"(dst + plan.wbytes + j * kXStride), "l"(p.x + (int64_t)tk * p.K + kb), "r"(xbytes),
+                          "r"(fb) : "memory");
+                }
                 if (first) {
                     // the item's scales: its rows x all blocks, one contiguous range
                     const uint8_t* ssrc = reinterpret_cast<const uint8_t*>(p.scales) +
@@ -198,40 +242,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
         uint32_t ctr = 0, jitem = 0;
         bool dead = false;   // set when a wait gives up: the warp then only keeps the barrier schedule
         float acc[GMAX][4];
-        // activation row of this lane's token column g, per 8-row group (-1: none), for the
-        // current and the next item; the next item's rows are prefetched into L1 early
-        int xtk[GMAX], ntk[GMAX];
-        auto tokens_of = [&](int item, int pass, int (&tk)[GMAX]) {
-#pragma unroll
-            for (int j = 0; j < GMAX; ++j) tk[j] = -1;
-            if (item >= i1) return;
-            const int a = item / nit;
-            const int64_t r0 = s_r0[a];
-            const int m = s_cnt[a];
-            const int mc = pass * 8 * GMAX;
-#pragma unroll
-            for (int j = 0; j < GMAX; ++j) {
-                const int rr = mc + 8 * j + g;
-                if (rr < m) tk[j] = p.row_token ? __ldg(p.row_token + r0 + rr) : (int)(r0 + rr);
-            }
-        };
-        auto prefetch_x = [&](const int (&tk)[GMAX]) {
-#pragma unroll
-            for (int j = 0; j < GMAX; ++j) {
-                if (tk[j] < 0) continue;
-                const uint16_t* xr = p.x + (int64_t)tk[j] * p.K + t * (SB / 4);
-                for (int kc = 0; kc < plan.nch; ++kc) {
-                    const int kb = kc * kChunkK;
-                    const int nbc = min(kChunkK, p.K - kb) / SB;
-                    for (int b = ks * nbc / nks; b < (ks + 1) * nbc / nks; ++b)
-                        asm volatile("prefetch.global.L1 [%0];" ::"l"(xr + kb + b * SB));
-                }
-            }
-        };
         Pos cur{i0, 0, 0};
-        tokens_of(cur.item, 0, xtk);
-        prefetch_x(xtk);
-        tokens_of(cur.item + 1, 0, ntk);
         while (cur.item < i1) {
             const int a = cur.item / nit;
             const int n0 = (cur.item % nit) * ROWS;
@@ -243,12 +254,10 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
             if (cur.kc == 0) {
 #pragma unroll
                 for (int j = 0; j < GMAX; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-                if (cur.pass == 0) prefetch_x(ntk);       // next item's rows, one item ahead
             }
             const int kb = cur.kc * kChunkK;
             const int nbc = min(kChunkK, p.K - kb) / SB;
             const int b0 = ks * nbc / nks, b1 = (ks + 1) * nbc / nks;
-            const uint16_t* xbase = p.x + kb + t * (SB / 4);
             const uint32_t slot = ctr % ns, ph = (ctr / ns) & 1u;
             ++ctr;
             if (!dead && !mbar_wait_bounded(smem_addr(bars + slot), ph, abort_flag, &g_decode_error, 2u)) dead = true;
@@ -295,17 +304,14 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
 #pragma unroll
                     for (int j = 0; j < GMAX; ++j) {
                         if (j < G) {
+                            // staged activations of routed row mc + 8j + g (rows past m hold stale
+                            // data and only feed output columns that are never stored)
                             uint32_t xw[XW];
-                            if (xtk[j] >= 0) {
+                            const uint8_t* xs = st + plan.wbytes + (8 * j + g) * kXStride + (b * SB + t * (SB / 4)) * 2;
 #pragma unroll
-                                for (int w = 0; w < XW / 4; ++w) {
-                                    const uint4 v = __ldg(reinterpret_cast<const uint4*>(
-                                        xbase + (int64_t)xtk[j] * p.K + b * SB) + w);
-                                    xw[4 * w] = v.x; xw[4 * w + 1] = v.y; xw[4 * w + 2] = v.z; xw[4 * w + 3] = v.w;
-                                }
-                            } else {
-#pragma unroll
-                                for (int w = 0; w < XW; ++w) xw[w] = 0u;
+                            for (int w = 0; w < XW / 4; ++w) {
+                                const uint4 v = *reinterpret_cast<const uint4*>(xs + 16 * w);
+                                xw[4 * w] = v.x; xw[4 * w + 1] = v.y; xw[4 * w + 2] = v.z; xw[4 * w + 3] = v.w;
                             }
                             float cb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -340,21 +346,20 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
                         for (int k2 = 0; k2 < nks; ++k2)
                             v += reinterpret_cast<const float*>(&red[((k2 * nrt + rtt) * GMAX + j) * 32 + ln])[i];
                         const int64_t r = r0 + row;
-                        if (p.row_weight) v *= __ldg(p.row_weight + r);
-                        const int64_t dst = p.row_dest ? (int64_t)__ldg(p.row_dest + r) : r;
-                        p.out[dst * p.N + n0 + nr] = f32_to_bf16_rne(v);
+                        float wgt;
+                        int64_t dst;
+                        if (table) {
+                            wgt = t_wt[r - rlo];
+                            dst = t_dst[r - rlo];
+                        } else {
+                            wgt = p.row_weight ? __ldg(p.row_weight + r) : 1.f;
+                            dst = p.row_dest ? (int64_t)__ldg(p.row_dest + r) : r;
+                        }
+                        p.out[dst * p.N + n0 + nr] = f32_to_bf16_rne(v * wgt);
                     }
                 }
                 asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");
-                // next pass of this item, or the next item
-                if (nxt.item != cur.item) {
-                    ++jitem;
-#pragma unroll
-                    for (int j = 0; j < GMAX; ++j) xtk[j] = ntk[j];
-                    tokens_of(nxt.item + 1, 0, ntk);
-                } else {
-                    tokens_of(nxt.item, nxt.pass, xtk);
-                }
+                if (nxt.item != cur.item) ++jitem;
             }
             cur = nxt;
         }
@@ -381,17 +386,19 @@ static cudaError_t launch_db(const GroupedArgs& a, cudaStream_t s) {
     Plan plan;
     plan.nch = (a.K + kChunkK - 1) / kChunkK;
     const int red_bytes = kConsumers * GMAX * 32 * (int)sizeof(float4);
-    const int tables = 32 + 16 * a.E;
+    const int tables = 32 + 16 * a.E + 12 * kMaxTableRows;
     int smem = 0;
     plan.rows = 0;
     for (int rows = 64; rows >= 32 && plan.rows == 0; rows >>= 1) {
-        const int stage_bytes = rows * (kChunkK / 2);
+        const int wbytes = rows * (kChunkK / 2);
+        const int stage_bytes = wbytes + ((8 * GMAX * kXStride + 1023) / 1024) * 1024;
         const int scale_bytes = ((rows * (a.K / SB) * ssz + 127) / 128) * 128;
-        for (int nst = 8; nst >= 3; --nst) {
+        for (int nst = 6; nst >= 3; --nst) {
             const int nsl = (nst - 1 + plan.nch - 1) / plan.nch + 1;   // items in flight at once
             const int need = 1024 + kLutBytes + nst * stage_bytes + nsl * scale_bytes + red_bytes + 2 * nst * 8 + tables;
             if (need <= 226 * 1024) {
                 plan.rows = rows;
+                plan.wbytes = wbytes;
                 plan.stage_bytes = stage_bytes;
                 plan.scale_bytes = scale_bytes;
                 plan.nstages = nst;
