@@ -170,14 +170,20 @@ __device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
 
 // bf16 bit pattern of one 4-bit code (NF4: 16-entry table; MXFP4: magnitude
 // table of codes 0..7 plus the sign bit 3)
+// (the plane word is chosen by selects, not by a runtime array index, so that
+// the tables stay in registers)
+__device__ __forceinline__ uint32_t plane_word(const uint32_t (&v)[4], uint32_t i) {
+    return i == 0u ? v[0] : i == 1u ? v[1] : i == 2u ? v[2] : v[3];
+}
 template <int FMT>
 __device__ __forceinline__ uint32_t code_bf16(uint32_t c, const LutPlanes& L) {
     if constexpr (FMT == FMT_NF4) {
         const uint32_t sh = 8u * (c & 3u);
-        return (((L.hi[c >> 2] >> sh) & 0xFFu) << 8) | ((L.lo[c >> 2] >> sh) & 0xFFu);
+        return (((plane_word(L.hi, c >> 2) >> sh) & 0xFFu) << 8) | ((plane_word(L.lo, c >> 2) >> sh) & 0xFFu);
     } else {
         const uint32_t m = c & 7u, sh = 8u * (m & 3u);
-        return (((L.hi[m >> 2] >> sh) & 0xFFu) << 8) | ((L.lo[m >> 2] >> sh) & 0xFFu) | ((c & 8u) << 12);
+        return (((plane_word(L.hi, m >> 2) >> sh) & 0xFFu) << 8) | ((plane_word(L.lo, m >> 2) >> sh) & 0xFFu) |
+               ((c & 8u) << 12);
     }
 }
 

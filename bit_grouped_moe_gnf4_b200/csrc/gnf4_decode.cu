@@ -6,27 +6,32 @@
 //
 // One persistent CTA per SM takes a contiguous run of work items; an item is
 // (active expert, ROWS = 64 weight rows; 32 when K is very large). A producer
-// thread streams each item's packed rows, one K chunk of 512 at a time, into a
-// ring of 16 KB shared-memory stages with 2-D TMA loads (boxes of 128 bytes x
-// ROWS rows, 128B-swizzled), several stages ahead; big requests are what lets
-// the copy engine keep HBM busy. The same stage also carries the chunk of each
-// routed row's activations (1-D bulk copies, one per row), and the item's block
-// scales (ROWS rows x all blocks, one contiguous range) arrive with its first
-// chunk, so the consumers never wait on a global load. The CTA's routing
+// thread streams each item's packed rows, one K chunk of 256 at a time, into a
+// ring of shared-memory stages with one 2-D TMA load per chunk (a box of 128
+// bytes x ROWS rows, 128B-swizzled), several stages ahead; big requests are what
+// lets the copy engine keep HBM busy. The same stage also carries the chunk of
+// each routed row's activations (1-D bulk copies, one per row), and the item's
+// block scales (ROWS rows x all blocks, one contiguous range) arrive with its
+// first chunk, so the consumers never wait on a global load. The CTA's routing
 // metadata (token, weight, destination of each of its routed rows) is staged in
 // shared memory once at the start.
 //
-// 16 consumer warps split an item as (ROWS/16 row tiles) x (16/(ROWS/16)) K
-// splits of every chunk. Nibble pairs are decoded by a table in shared memory
-// that maps each packed byte to its two bf16 values (one bf16x2 word),
-// replicated per lane so that 32 lookups never conflict; a byte permute forms
-// the lookup address. The products run on warp-level bf16 MMAs with 16 weight
-// rows as the M side and up to 8 routed rows per MMA as the N side. Every MMA
-// chain covers exactly one scale block (64 K for NF4, 32 K for MXFP4), so the
-// block sum leaves the tensor core in fp32 and is scaled and accumulated in
-// fp32 outside it. At the end of an item the K splits' partial sums are added
-// in a fixed order through shared memory (deterministic), weighted, rounded to
-// bf16 and stored at the destination rows.
+// 16 consumer warps: warp (rt, ks) owns row tile rt (16 rows of the item) and
+// every nks-th chunk of the CTA's stream (chunk counter % nks == ks), so each
+// stage is read by ROWS/16 warps and stages are consumed in parallel. Because
+// owners skip the stages of other warps, a ring slot carries a tag naming the
+// chunk that was last issued into it; an owner reads the slot's barrier only
+// once the tag shows its chunk, which keeps every parity wait within one phase. Nibbles are decoded two ways, to balance the
+// shared-memory and ALU pipes: one of the lane's two rows by a table in shared
+// memory that maps each packed byte to its two bf16 values (replicated per lane,
+// so 32 lookups never conflict; a byte permute forms the address), the other by
+// byte permutes on tables held in registers. The products run on warp-level
+// bf16 MMAs with 16 weight rows as the M side and up to 8 routed rows per MMA as
+// the N side. Every MMA chain covers exactly one scale block (64 K for NF4, 32 K
+// for MXFP4), so the block sum leaves the tensor core in fp32 and is scaled and
+// accumulated in fp32 outside it. At the end of an item the row tile's K-split
+// partial sums are added in a fixed order through shared memory
+// (deterministic), weighted, rounded to bf16 and stored at the destination rows.
 //
 // MMA k-slot mapping: in m16n8k16, lane (g, t) supplies k-slots 2t, 2t+1,
 // 2t+8, 2t+9 of both operands. They are mapped to the four consecutive K
@@ -50,8 +55,8 @@ namespace db {
 
 constexpr int kConsumers = 16;                     // consumer warps
 constexpr int kThreads = (kConsumers + 1) * 32;    // + one producer warp
-constexpr int kChunkK = 512;                       // K per stage: 256 packed bytes per row
-constexpr int kBoxBytes = 128;                     // TMA box width (one 128B swizzle row)
+constexpr int kChunkK = 256;                       // K per stage: 128 packed bytes per row = one TMA box
+constexpr int kBoxBytes = 128;
 constexpr int kLutBytes = 256 * 256;               // byte value b, lane l -> offset b*256 + l*4
 constexpr int kXStride = kChunkK * 2 + 16;         // bytes per staged activation row (padded)
 constexpr int kMaxTableRows = 1024;                // routed rows whose metadata fits the CTA's table
@@ -59,15 +64,11 @@ constexpr int kMaxTableRows = 1024;                // routed rows whose metadata
 struct Plan {
     int rows;         // weight rows per item (64 or 32)
     int nch;          // stages per item pass
-    int wbytes;       // packed-weight part of a stage: rows x 256 bytes
-    int stage_bytes;  // wbytes + activation rows (8*GMAX x kXStride)
+    int wbytes;       // packed-weight part of a stage: rows x 128 bytes
+    int stage_bytes;  // wbytes + activation rows (8*GMAX x kXStride), rounded to 1024
     int scale_bytes;  // slot for one item's scales (rows x all blocks), rounded to 128
     int nstages;      // ring stages
     int nslots;       // item scale slots
-};
-
-struct Pos {
-    int item, pass, kc;
 };
 
 __device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
@@ -75,6 +76,34 @@ __device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3}], [%4];"
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void bulk_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+// Wait until the ring slot's tag names chunk `want` (the producer has issued it,
+// so the slot's previous fill was consumed). Bounded like mbar_wait_bounded.
+__device__ __forceinline__ bool wait_tag(const int* tag, uint32_t want, volatile int* abort_flag, unsigned* err,
+                                         unsigned code) {
+    const uint32_t a = smem_addr(tag);
+    uint32_t v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    if (v == want) return true;
+    const long long t0 = clock64();
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(64);
+        asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+        if (v == want) return true;
+        if ((it & 7u) == 0u) {
+            if (*abort_flag) return false;
+            if (clock64() - t0 > kWaitTimeoutCycles) {
+                *abort_flag = 1;
+                atomicOr(err, code);
+                return false;
+            }
+        }
+    }
 }
 
 }  // namespace db
@@ -87,20 +116,22 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
     constexpr int STEPS = SB / 16;                   // k16 MMA steps per block
     constexpr int BPL = SB / 8;                      // packed bytes per lane per row per block (8 or 4)
     constexpr int XW = SB / 8;                       // bf16x2 words of x per lane per block
-    constexpr int BPW = 4;                           // most blocks a warp takes from one chunk
+    constexpr int NBC = kChunkK / SB;                // scale blocks in a full chunk (4 or 8)
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // [lut][ring: stages x stage_bytes][scale slots][red][barriers][abort, count][experts]
+    // [lut][ring: stages x stage_bytes][scale slots][red][barriers][abort, count][experts][row table]
     uint8_t* lut = smem;                                            // [256][64] words
     uint8_t* ring = smem + kLutBytes;                               // 1024-aligned stages
     uint8_t* sslots = ring + plan.nstages * plan.stage_bytes;
     float4* red = reinterpret_cast<float4*>(sslots + plan.nslots * plan.scale_bytes);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(red + kConsumers * GMAX * 32);   // full[s], empty[s]
-    int* tailw = reinterpret_cast<int*>(bars + 2 * plan.nstages);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(red + kConsumers * GMAX * 32);
+    // full[ns], empty[ns], scale slot free[nslots], scale slot full[nslots]
+    int* tailw = reinterpret_cast<int*>(bars + 2 * plan.nstages + 2 * plan.nslots);
     volatile int* abort_flag = tailw;
     int* s_nact = tailw + 4;
-    int64_t* s_r0 = reinterpret_cast<int64_t*>(tailw + 8);         // [E] first routed row
+    int* tags = tailw + 8;                                         // [ns] chunk counter last issued per slot
+    int64_t* s_r0 = reinterpret_cast<int64_t*>(tailw + 8 + ((plan.nstages + 1) & ~1)); // [E] first routed row
     int* s_active = reinterpret_cast<int*>(s_r0 + p.E);            // [E] expert id
     int* s_cnt = s_active + p.E;                                   // [E] routed rows
     int* t_tok = s_cnt + p.E;                                      // [kMaxTableRows] per routed row
@@ -108,13 +139,19 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
     int* t_dst = reinterpret_cast<int*>(t_wt + kMaxTableRows);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ns = plan.nstages;
+    const int ns = plan.nstages, nsl = plan.nslots;
     const int ROWS = plan.rows;
+    const int nrt = ROWS / 16, nks = kConsumers / nrt;
+    uint64_t* full = bars;
+    uint64_t* empty = bars + ns;
+    uint64_t* sfree = bars + 2 * ns;
+    uint64_t* sfull = bars + 2 * ns + nsl;
 
     // byte -> bf16x2 table, one copy per lane
+    const LutPlanes L = p.lut;                      // register copy (also for the permute decode)
     for (int i = threadIdx.x; i < 256 * 32; i += kThreads) {
         const int b = i >> 5, l = i & 31;
-        *reinterpret_cast<uint32_t*>(lut + b * 256 + l * 4) = byte_bf16x2<FMT>((uint32_t)b, p.lut);
+        *reinterpret_cast<uint32_t*>(lut + b * 256 + l * 4) = byte_bf16x2<FMT>((uint32_t)b, L);
     }
     if (warp == 0) {
         // experts of this band, in id order (every CTA derives the same list)
@@ -138,9 +175,14 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
         if (lane == 0) s_nact[0] = count;
     } else if (warp == kConsumers && lane == 0) {
         for (int i = 0; i < ns; ++i) {
-            mbar_init(smem_addr(bars + i), 1);                 // full: producer + tx bytes
-            mbar_init(smem_addr(bars + ns + i), kConsumers);   // empty: every consumer warp
+            mbar_init(smem_addr(full + i), 1);       // producer + tx bytes
+            mbar_init(smem_addr(empty + i), nrt);    // the warps that own the chunk
         }
+        for (int i = 0; i < nsl; ++i) {
+            mbar_init(smem_addr(sfree + i), kConsumers);
+            mbar_init(smem_addr(sfull + i), 1);
+        }
+        for (int i = 0; i < ns; ++i) tags[i] = -1;
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -170,181 +212,223 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
         }
     }
     __syncthreads();
-    auto tok_of = [&](int64_t r) -> int {
-        return table ? t_tok[r - rlo] : (p.row_token ? __ldg(p.row_token + r) : (int)r);
-    };
 
-    auto advance = [&](Pos q) -> Pos {
-        if (++q.kc == plan.nch) {
-            q.kc = 0;
-            const int m = s_cnt[q.item / nit];
-            if (++q.pass == (m + 8 * GMAX - 1) / (8 * GMAX)) {
-                q.pass = 0;
-                ++q.item;
-            }
-        }
-        return q;
-    };
-
+    const int nch = plan.nch;
     if (warp == kConsumers) {
         // ================= producer (one thread) =================
         if (lane == 0) {
-            uint32_t ctr = 0, jitem = 0;
-            for (Pos ps{i0, 0, 0}; ps.item < i1; ps = advance(ps), ++ctr) {
-                const uint32_t slot = ctr % ns, ph = ((ctr / ns) & 1u) ^ 1u;
-                if (!mbar_wait_bounded(smem_addr(bars + ns + slot), ph, abort_flag, &g_decode_error, 1u)) break;
-                const int a = ps.item / nit;
+            uint32_t ctr = 0, slot = 0, ph = 1;       // ring position; empty-barrier parity to wait on
+            uint32_t sslot = 0, sph = 1;              // scale slot; its free-barrier parity
+            int a = (i1 > i0) ? i0 / nit : 0, it = (i1 > i0) ? i0 % nit : 0;
+            bool ok = true;
+            for (int item = i0; item < i1 && ok; ++item) {
                 const int e = s_active[a];
-                const int n0 = (ps.item % nit) * ROWS;
-                const int xb = ps.kc * (kChunkK / 2);                 // first packed byte of the chunk
-                const int nbox = (p.K / 2 - xb) > kBoxBytes ? 2 : 1;  // the last chunk may be half
-                const uint32_t fb = smem_addr(bars + slot);
-                const bool first = ps.kc == 0 && ps.pass == 0;
-                const int vrows = min(ROWS, p.N - n0);
-                const uint32_t sbytes = (uint32_t)(vrows * nbk * ssz);   // a multiple of 16
-                // activation rows of this pass: their chunk of K, one bulk copy each
+                const int n0 = it * ROWS;
+                const int cnt = s_cnt[a];
                 const int64_t r0 = s_r0[a];
-                const int mc = ps.pass * 8 * GMAX;
-                const int nx = min(8 * GMAX, s_cnt[a] - mc);
-                const int kb = ps.kc * kChunkK;
-                const uint32_t xbytes = (uint32_t)(min(kChunkK, p.K - kb) * 2);
-                mbar_arrive_tx(fb, (uint32_t)(nbox * kBoxBytes * ROWS) + (uint32_t)nx * xbytes + (first ? sbytes : 0u));
-                const uint32_t dst = smem_addr(ring + slot * plan.stage_bytes);
-                for (int bx = 0; bx < nbox; ++bx)
-                    tma_2d(dst + bx * kBoxBytes * ROWS, &wmap, xb + bx * kBoxBytes, e * p.N + n0, fb);
-                for (int j = 0; j < nx; ++j) {
-                    const int tk = tok_of(r0 + mc + j);
-                    asm volatile(
-                        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                        ::"r"(dst + plan.wbytes + j * kXStride), "l"(p.x + (int64_t)tk * p.K + kb), "r"(xbytes),
-                          "r"(fb) : "memory");
-                }
-                if (first) {
-                    // the item's scales: its rows x all blocks, one contiguous range
+                const int npass = (cnt + 8 * GMAX - 1) / (8 * GMAX);
+                const int vrows = min(ROWS, p.N - n0);
+                // the item's scales: its rows x all blocks, one contiguous range (a multiple of 16 bytes)
+                if (!mbar_wait_bounded(smem_addr(sfree + sslot), sph, abort_flag, &g_decode_error, 4u)) break;
+                {
+                    const uint32_t sbytes = (uint32_t)(vrows * nbk * ssz);
                     const uint8_t* ssrc = reinterpret_cast<const uint8_t*>(p.scales) +
                                           ((int64_t)e * p.N + n0) * nbk * ssz;
-                    asm volatile(
-                        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                        ::"r"(smem_addr(sslots + (jitem % plan.nslots) * plan.scale_bytes)), "l"(ssrc),
-                          "r"(sbytes), "r"(fb) : "memory");
-                    ++jitem;
+                    const uint32_t sb = smem_addr(sfull + sslot);
+                    mbar_arrive_tx(sb, sbytes);
+                    bulk_1d(smem_addr(sslots + sslot * plan.scale_bytes), ssrc, sbytes, sb);
+                    if (++sslot == (uint32_t)nsl) {
+                        sslot = 0;
+                        sph ^= 1u;
+                    }
+                }
+                for (int pass = 0; pass < npass && ok; ++pass) {
+                    // activation rows of this pass: their chunk of K, one bulk copy each
+                    const int mc = pass * 8 * GMAX;
+                    const int nx = min(8 * GMAX, cnt - mc);
+                    for (int kc = 0; kc < nch; ++kc) {
+                        if (!mbar_wait_bounded(smem_addr(empty + slot), ph, abort_flag, &g_decode_error, 1u)) {
+                            ok = false;
+                            break;
+                        }
+                        // the slot's previous chunk is consumed: name the chunk it now receives
+                        asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_addr(tags + slot)), "r"(ctr)
+                                     : "memory");
+                        const int kb = kc * kChunkK;
+                        const uint32_t xbytes = (uint32_t)(min(kChunkK, p.K - kb) * 2);
+                        const uint32_t fb = smem_addr(full + slot);
+                        mbar_arrive_tx(fb, (uint32_t)(kBoxBytes * ROWS) + (uint32_t)nx * xbytes);
+                        const uint32_t dst = smem_addr(ring + slot * plan.stage_bytes);
+                        tma_2d(dst, &wmap, kb / 2, e * p.N + n0, fb);
+                        for (int j = 0; j < nx; ++j) {
+                            const int64_t r = r0 + mc + j;
+                            const int tk = table ? t_tok[r - rlo] : (p.row_token ? __ldg(p.row_token + r) : (int)r);
+                            bulk_1d(dst + plan.wbytes + j * kXStride, p.x + (int64_t)tk * p.K + kb, xbytes, fb);
+                        }
+                        ++ctr;
+                        if (++slot == (uint32_t)ns) {
+                            slot = 0;
+                            ph ^= 1u;
+                        }
+                    }
+                }
+                if (++it == nit) {
+                    it = 0;
+                    ++a;
                 }
             }
         }
         __syncwarp();
     } else {
         // ================= consumers =================
-        const int nrt = ROWS / 16, nks = kConsumers / nrt;
-        const int rt = warp % nrt, ks = warp / nrt;     // row tile, K split
+        const int rt = warp % nrt, ks = warp / nrt;     // row tile, K split (chunk counter % nks == ks)
         const int g = lane >> 2, t = lane & 3;
         const int ra = rt * 16 + g, rb = ra + 8;        // the two item rows of this lane
         const uint32_t lane_sel = (uint32_t)lane * 4u;  // lut offset of this lane's copy
-        uint32_t ctr = 0, jitem = 0;
+        const bool vec_scales = (FMT == FMT_NF4) && (nbk % 4 == 0);
+        const uint32_t kmask = (uint32_t)nks - 1u;      // nks is 4 or 8
         bool dead = false;   // set when a wait gives up: the warp then only keeps the barrier schedule
         float acc[GMAX][4];
-        Pos cur{i0, 0, 0};
-        while (cur.item < i1) {
-            const int a = cur.item / nit;
-            const int n0 = (cur.item % nit) * ROWS;
-            const int64_t r0 = s_r0[a];
+#pragma unroll
+        for (int j = 0; j < GMAX; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+        uint32_t base = 0;                              // chunk counter at the start of the pass
+        uint32_t sslot = 0, sph = 0;                    // scale slot; its full-barrier parity
+        int a = (i1 > i0) ? i0 / nit : 0, it = (i1 > i0) ? i0 % nit : 0;
+        for (int item = i0; item < i1; ++item) {
             const int m = s_cnt[a];
-            const int mc = cur.pass * 8 * GMAX;
-            const int G = min(GMAX, (m - mc + 7) >> 3);
-            const Pos nxt = advance(cur);
-            if (cur.kc == 0) {
-#pragma unroll
-                for (int j = 0; j < GMAX; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-            }
-            const int kb = cur.kc * kChunkK;
-            const int nbc = min(kChunkK, p.K - kb) / SB;
-            const int b0 = ks * nbc / nks, b1 = (ks + 1) * nbc / nks;
-            const uint32_t slot = ctr % ns, ph = (ctr / ns) & 1u;
-            ++ctr;
-            if (!dead && !mbar_wait_bounded(smem_addr(bars + slot), ph, abort_flag, &g_decode_error, 2u)) dead = true;
-            const uint8_t* st = ring + slot * plan.stage_bytes;
-            const uint8_t* ss = sslots + (jitem % plan.nslots) * plan.scale_bytes;
-            const int bg0 = cur.kc * (kChunkK / SB);      // first scale block of the chunk
-#pragma unroll
-            for (int c = 0; c < BPW; ++c) {
-                if (!dead && b0 + c < b1) {
-                    const int b = b0 + c;
-                    float s0, s1;
-                    if constexpr (FMT == FMT_NF4) {
-                        s0 = reinterpret_cast<const float*>(ss)[ra * nbk + bg0 + b];
-                        s1 = reinterpret_cast<const float*>(ss)[rb * nbk + bg0 + b];
-                    } else {
-                        s0 = e8m0_to_f32(ss[ra * nbk + bg0 + b]);
-                        s1 = e8m0_to_f32(ss[rb * nbk + bg0 + b]);
-                    }
-                    // this lane's packed bytes of rows ra and rb: byte o of the row's 256-byte
-                    // chunk lives in box o/128, 16-byte piece ((o%128)/16) ^ (row%8)
-                    const int o = b * (SB / 2) + t * BPL;
-                    const uint8_t* bx = st + (o >> 7) * (kBoxBytes * ROWS);
-                    const int pc = (o & 127) >> 4, po = o & 15;
-                    const uint8_t* rp0 = bx + ra * kBoxBytes + ((pc ^ (ra & 7)) << 4) + po;
-                    const uint8_t* rp1 = bx + rb * kBoxBytes + ((pc ^ (rb & 7)) << 4) + po;
-                    uint32_t w0[BPL / 4], w1[BPL / 4];
-                    if constexpr (BPL == 8) {
-                        const uint2 u0 = *reinterpret_cast<const uint2*>(rp0);
-                        const uint2 u1 = *reinterpret_cast<const uint2*>(rp1);
-                        w0[0] = u0.x; w0[BPL / 4 - 1] = u0.y;
-                        w1[0] = u1.x; w1[BPL / 4 - 1] = u1.y;
-                    } else {
-                        w0[0] = *reinterpret_cast<const uint32_t*>(rp0);
-                        w1[0] = *reinterpret_cast<const uint32_t*>(rp1);
-                    }
-                    // byte j -> bf16x2 word j (table lookup; address = byte*256 + lane*4)
-                    uint32_t d0[BPL], d1[BPL];
-#pragma unroll
-                    for (int j = 0; j < BPL; ++j) {
-                        const uint32_t sel = 0x5504u | ((uint32_t)(j & 3) << 4);
-                        d0[j] = *reinterpret_cast<const uint32_t*>(lut + prmt(w0[j >> 2], lane_sel, sel));
-                        d1[j] = *reinterpret_cast<const uint32_t*>(lut + prmt(w1[j >> 2], lane_sel, sel));
-                    }
-#pragma unroll
-                    for (int j = 0; j < GMAX; ++j) {
-                        if (j < G) {
-                            // staged activations of routed row mc + 8j + g (rows past m hold stale
-                            // data and only feed output columns that are never stored)
-                            uint32_t xw[XW];
-                            const uint8_t* xs = st + plan.wbytes + (8 * j + g) * kXStride + (b * SB + t * (SB / 4)) * 2;
-#pragma unroll
-                            for (int w = 0; w < XW / 4; ++w) {
-                                const uint4 v = *reinterpret_cast<const uint4*>(xs + 16 * w);
-                                xw[4 * w] = v.x; xw[4 * w + 1] = v.y; xw[4 * w + 2] = v.z; xw[4 * w + 3] = v.w;
+            const int n0 = it * ROWS;
+            const int64_t r0 = s_r0[a];
+            const int npass = (m + 8 * GMAX - 1) / (8 * GMAX);
+            const int vrows = min(ROWS, p.N - n0);
+            // every warp waits for the item's scales (also those that own no chunk of it)
+            if (!dead && !mbar_wait_bounded(smem_addr(sfull + sslot), sph, abort_flag, &g_decode_error, 8u))
+                dead = true;
+            const uint8_t* ss = sslots + sslot * plan.scale_bytes;
+            for (int pass = 0; pass < npass; ++pass) {
+                const int mc = pass * 8 * GMAX;
+                const int nvalid = min(8 * GMAX, m - mc);   // routed rows of this pass
+                int kc = (int)(((uint32_t)ks - base) & kmask);
+                uint32_t ctr = base + (uint32_t)kc;
+                uint32_t slot = ctr % (uint32_t)ns, ph = (ctr / (uint32_t)ns) & 1u;
+                for (; kc < nch; kc += nks) {
+                    if (!dead && !wait_tag(tags + slot, ctr, abort_flag, &g_decode_error, 16u)) dead = true;
+                    if (!dead && !mbar_wait_bounded(smem_addr(full + slot), ph, abort_flag, &g_decode_error, 2u))
+                        dead = true;
+                        const uint8_t* st = ring + slot * plan.stage_bytes;
+                        const int kb = kc * kChunkK;
+                        const int nbc = min(kChunkK, p.K - kb) / SB;
+                        const int bg0 = kc * NBC;                 // first scale block of the chunk
+                        // block scales of rows ra and rb for this chunk
+                        float sa[NBC], sb[NBC];
+                        if (!dead) {
+                            if (vec_scales && nbc == NBC) {
+                                const float4 va = *reinterpret_cast<const float4*>(ss + (ra * nbk + bg0) * 4);
+                                const float4 vb = *reinterpret_cast<const float4*>(ss + (rb * nbk + bg0) * 4);
+                                sa[0] = va.x; sa[1] = va.y; sa[2] = va.z; sa[3] = va.w;
+                                sb[0] = vb.x; sb[1] = vb.y; sb[2] = vb.z; sb[3] = vb.w;
+                            } else {
+        #pragma unroll
+                                for (int b = 0; b < NBC; ++b) {
+                                    if (b < nbc) {
+                                        if constexpr (FMT == FMT_NF4) {
+                                            sa[b] = reinterpret_cast<const float*>(ss)[ra * nbk + bg0 + b];
+                                            sb[b] = reinterpret_cast<const float*>(ss)[rb * nbk + bg0 + b];
+                                        } else {
+                                            sa[b] = e8m0_to_f32(ss[ra * nbk + bg0 + b]);
+                                            sb[b] = e8m0_to_f32(ss[rb * nbk + bg0 + b]);
+                                        }
+                                    } else {
+                                        sa[b] = sb[b] = 0.f;
+                                    }
+                                }
                             }
-                            float cb[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                            for (int s = 0; s < STEPS; ++s)
-                                mma_bf16_16816(cb, d0[2 * s], d1[2 * s], d0[2 * s + 1], d1[2 * s + 1], xw[2 * s],
-                                               xw[2 * s + 1]);
-                            acc[j][0] = fmaf(cb[0], s0, acc[j][0]);
-                            acc[j][1] = fmaf(cb[1], s0, acc[j][1]);
-                            acc[j][2] = fmaf(cb[2], s1, acc[j][2]);
-                            acc[j][3] = fmaf(cb[3], s1, acc[j][3]);
                         }
+        #pragma unroll
+                        for (int b = 0; b < NBC; ++b) {
+                            if (!dead && b < nbc) {
+                                // this lane's packed bytes of rows ra and rb: byte o of the row's 128-byte
+                                // chunk sits in 16-byte piece (o/16) ^ (row%8) of the swizzled box row
+                                const int o = b * (SB / 2) + t * BPL;
+                                const int pc = o >> 4, po = o & 15;
+                                const uint8_t* rp0 = st + ra * kBoxBytes + ((pc ^ (ra & 7)) << 4) + po;
+                                const uint8_t* rp1 = st + rb * kBoxBytes + ((pc ^ (rb & 7)) << 4) + po;
+                                uint32_t w0[BPL / 4], w1[BPL / 4];
+                                if constexpr (BPL == 8) {
+                                    const uint2 u0 = *reinterpret_cast<const uint2*>(rp0);
+                                    const uint2 u1 = *reinterpret_cast<const uint2*>(rp1);
+                                    w0[0] = u0.x; w0[BPL / 4 - 1] = u0.y;
+                                    w1[0] = u1.x; w1[BPL / 4 - 1] = u1.y;
+                                } else {
+                                    w0[0] = *reinterpret_cast<const uint32_t*>(rp0);
+                                    w1[0] = *reinterpret_cast<const uint32_t*>(rp1);
+                                }
+                                // row ra by the shared-memory table, row rb by register byte permutes
+                                uint32_t d0[BPL], d1[BPL];
+        #pragma unroll
+                                for (int j = 0; j < BPL; ++j) {
+                                    const uint32_t sel = 0x5504u | ((uint32_t)(j & 3) << 4);
+                                    d0[j] = *reinterpret_cast<const uint32_t*>(lut + prmt(w0[j >> 2], lane_sel, sel));
+                                }
+        #pragma unroll
+                                for (int q = 0; q < BPL / 4; ++q) {
+                                    uint32_t o4[4];
+                                    decode_word<FMT>(w1[q], L, o4);
+                                    d1[4 * q] = o4[0]; d1[4 * q + 1] = o4[1]; d1[4 * q + 2] = o4[2]; d1[4 * q + 3] = o4[3];
+                                }
+        #pragma unroll
+                                for (int j = 0; j < GMAX; ++j) {
+                                    if (8 * j < nvalid) {
+                                        // staged activations of routed row mc + 8j + g (lanes past the pass's
+                                        // rows feed output columns that are never stored)
+                                        uint32_t xw[XW];
+        #pragma unroll
+                                        for (int w = 0; w < XW; ++w) xw[w] = 0u;
+                                        if (8 * j + g < nvalid) {
+                                            const uint8_t* xs = st + plan.wbytes + (8 * j + g) * kXStride + (b * SB + t * (SB / 4)) * 2;
+        #pragma unroll
+                                            for (int w = 0; w < XW / 4; ++w) {
+                                                const uint4 v = *reinterpret_cast<const uint4*>(xs + 16 * w);
+                                                xw[4 * w] = v.x; xw[4 * w + 1] = v.y; xw[4 * w + 2] = v.z; xw[4 * w + 3] = v.w;
+                                            }
+                                        }
+                                        float cb[4] = {0.f, 0.f, 0.f, 0.f};
+        #pragma unroll
+                                        for (int s = 0; s < STEPS; ++s)
+                                            mma_bf16_16816(cb, d0[2 * s], d1[2 * s], d0[2 * s + 1], d1[2 * s + 1], xw[2 * s],
+                                                           xw[2 * s + 1]);
+                                        acc[j][0] = fmaf(cb[0], sa[b], acc[j][0]);
+                                        acc[j][1] = fmaf(cb[1], sa[b], acc[j][1]);
+                                        acc[j][2] = fmaf(cb[2], sb[b], acc[j][2]);
+                                        acc[j][3] = fmaf(cb[3], sb[b], acc[j][3]);
+                                    }
+                                }
+                            }
+                        }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_addr(empty + slot));
+                    ctr += (uint32_t)nks;
+                    slot += (uint32_t)nks;                      // nks <= ns: at most one wrap
+                    if (slot >= (uint32_t)ns) {
+                        slot -= (uint32_t)ns;
+                        ph ^= 1u;
                     }
                 }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(bars + ns + slot));
-            if (cur.kc == plan.nch - 1) {
-                // the K splits' partial sums, added in a fixed order, then the epilogue
+                base += (uint32_t)nch;
+                // end of a pass: the row tile's K-split partial sums, added in a fixed order
+                const int G = min(GMAX, (nvalid + 7) >> 3);
 #pragma unroll
                 for (int j = 0; j < GMAX; ++j)
-                    if (j < G) red[((ks * nrt + rt) * GMAX + j) * 32 + lane] =
+                    if (j < G) red[((rt * nks + ks) * GMAX + j) * 32 + lane] =
                                    make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
-                asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");
-                const int vrows = min(ROWS, p.N - n0);
-                for (int qq = threadIdx.x; qq < nrt * G * 128; qq += kConsumers * 32) {
-                    const int i = qq & 3, ln = (qq >> 2) & 31, rest = qq >> 7;
-                    const int j = rest % G, rtt = rest / G;
-                    const int row = mc + 8 * j + 2 * (ln & 3) + (i & 1);     // C column 2t (+1)
-                    const int nr = rtt * 16 + (ln >> 2) + ((i & 2) ? 8 : 0);  // C row g (+8)
+                asm volatile("bar.sync %0, %1;" ::"r"(1 + rt), "r"(nks * 32) : "memory");
+                for (int qq = ks * 32 + lane; qq < G * 128; qq += nks * 32) {
+                    const int i = qq & 3, ln = (qq >> 2) & 31, j = qq >> 7;
+                    const int row = mc + 8 * j + 2 * (ln & 3) + (i & 1);       // C column 2t (+1)
+                    const int nr = rt * 16 + (ln >> 2) + ((i & 2) ? 8 : 0);    // C row g (+8)
                     if (row < m && nr < vrows) {
                         float v = 0.f;
                         for (int k2 = 0; k2 < nks; ++k2)
-                            v += reinterpret_cast<const float*>(&red[((k2 * nrt + rtt) * GMAX + j) * 32 + ln])[i];
+                            v += reinterpret_cast<const float*>(&red[((rt * nks + k2) * GMAX + j) * 32 + ln])[i];
                         const int64_t r = r0 + row;
                         float wgt;
                         int64_t dst;
@@ -358,10 +442,21 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
                         p.out[dst * p.N + n0 + nr] = f32_to_bf16_rne(v * wgt);
                     }
                 }
-                asm volatile("bar.sync 1, %0;" ::"n"(kConsumers * 32) : "memory");
-                if (nxt.item != cur.item) ++jitem;
+                asm volatile("bar.sync %0, %1;" ::"r"(1 + rt), "r"(nks * 32) : "memory");
+#pragma unroll
+                for (int j = 0; j < GMAX; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
             }
-            cur = nxt;
+            // every warp is done with this item's scales
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(sfree + sslot));
+            if (++sslot == (uint32_t)nsl) {
+                sslot = 0;
+                sph ^= 1u;
+            }
+            if (++it == nit) {
+                it = 0;
+                ++a;
+            }
         }
     }
 }
@@ -390,22 +485,26 @@ static cudaError_t launch_db(const GroupedArgs& a, cudaStream_t s) {
     int smem = 0;
     plan.rows = 0;
     for (int rows = 64; rows >= 32 && plan.rows == 0; rows >>= 1) {
-        const int wbytes = rows * (kChunkK / 2);
-        const int stage_bytes = wbytes + ((8 * GMAX * kXStride + 1023) / 1024) * 1024;
+        const int wbytes = rows * kBoxBytes;
+        const int stage_bytes = ((wbytes + 8 * GMAX * kXStride + 1023) / 1024) * 1024;
         const int scale_bytes = ((rows * (a.K / SB) * ssz + 127) / 128) * 128;
-        for (int nst = 6; nst >= 3; --nst) {
-            const int nsl = (nst - 1 + plan.nch - 1) / plan.nch + 1;   // items in flight at once
-            const int need = 1024 + kLutBytes + nst * stage_bytes + nsl * scale_bytes + red_bytes + 2 * nst * 8 + tables;
-            if (need <= 226 * 1024) {
-                plan.rows = rows;
-                plan.wbytes = wbytes;
-                plan.stage_bytes = stage_bytes;
-                plan.scale_bytes = scale_bytes;
-                plan.nstages = nst;
-                plan.nslots = nsl;
-                smem = need;
-                break;
+        const int nks = kConsumers * 16 / rows;          // K-split warps per row tile: the ring holds at least one chunk each
+        for (int nst = 12; nst >= nks; --nst) {
+            for (int nsl = 3; nsl >= 2; --nsl) {
+                const int need = 1024 + kLutBytes + nst * stage_bytes + nsl * scale_bytes + red_bytes +
+                                 (2 * nst + 2 * nsl) * 8 + 4 * ((nst + 1) & ~1) + tables;
+                if (need <= 226 * 1024) {
+                    plan.rows = rows;
+                    plan.wbytes = wbytes;
+                    plan.stage_bytes = stage_bytes;
+                    plan.scale_bytes = scale_bytes;
+                    plan.nstages = nst;
+                    plan.nslots = nsl;
+                    smem = need;
+                    break;
+                }
             }
+            if (plan.rows) break;
         }
     }
     if (plan.rows == 0) return cudaErrorInvalidValue;

@@ -376,6 +376,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
         const int d = warp - kDecWarp0;
         const int i = (d & 3) * 32 + lane;                 // tile row
         const int hf = d >> 2;                             // 16-byte chunks 4hf .. 4hf+3 of the row
+        const LutPlanes L = p.lut;                         // decode tables in registers
         uint32_t stage_ctr = 0;
         for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
             for (int s = 0; s < nst; ++s, ++stage_ctr) {
@@ -388,7 +389,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
                 const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
                 uint32_t o[4][4];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) decode_word<FMT>(words[c], p.lut, o[c]);
+                for (int c = 0; c < 4; ++c) decode_word<FMT>(words[c], L, o[c]);
                 const uint32_t slot = stage_ctr % kStages, ph = ((stage_ctr / kStages) & 1u) ^ 1u;
                 if (!mbar_wait_bounded(bar_empty + 8 * slot, ph, abort_flag, err, 64u)) goto dec_done;
                 uint8_t* arow = smem + kOffA + slot * kAStageBytes + i * 128;
