@@ -10,28 +10,33 @@
 // ring of shared-memory stages with one 2-D TMA load per chunk (a box of 128
 // bytes x ROWS rows, 128B-swizzled), several stages ahead; big requests are what
 // lets the copy engine keep HBM busy. The same stage also carries the chunk of
-// each routed row's activations (1-D bulk copies, one per row), and the item's
-// block scales (ROWS rows x all blocks, one contiguous range) arrive with its
-// first chunk, so the consumers never wait on a global load. The CTA's routing
-// metadata (token, weight, destination of each of its routed rows) is staged in
-// shared memory once at the start.
+// each routed row's activations (1-D bulk copies, one per row). The item's block
+// scales (ROWS rows x all blocks, one contiguous range) land in a scale slot
+// with a barrier of their own. The CTA's routing metadata (token, weight,
+// destination of each of its routed rows) is staged in shared memory once.
 //
 // 16 consumer warps: warp (rt, ks) owns row tile rt (16 rows of the item) and
 // every nks-th chunk of the CTA's stream (chunk counter % nks == ks), so each
 // stage is read by ROWS/16 warps and stages are consumed in parallel. Because
 // owners skip the stages of other warps, a ring slot carries a tag naming the
 // chunk that was last issued into it; an owner reads the slot's barrier only
-// once the tag shows its chunk, which keeps every parity wait within one phase. Nibbles are decoded two ways, to balance the
-// shared-memory and ALU pipes: one of the lane's two rows by a table in shared
-// memory that maps each packed byte to its two bf16 values (replicated per lane,
-// so 32 lookups never conflict; a byte permute forms the address), the other by
-// byte permutes on tables held in registers. The products run on warp-level
-// bf16 MMAs with 16 weight rows as the M side and up to 8 routed rows per MMA as
-// the N side. Every MMA chain covers exactly one scale block (64 K for NF4, 32 K
-// for MXFP4), so the block sum leaves the tensor core in fp32 and is scaled and
-// accumulated in fp32 outside it. At the end of an item the row tile's K-split
-// partial sums are added in a fixed order through shared memory
-// (deterministic), weighted, rounded to bf16 and stored at the destination rows.
+// once the tag shows its chunk, which keeps every parity wait within one phase.
+//
+// Nibbles are decoded two ways, to balance the shared-memory and ALU pipes: one
+// of the lane's two rows by a table in shared memory that maps each packed byte
+// to its two bf16 values (replicated per lane, so 32 lookups never conflict; a
+// byte permute forms the address), the other by byte permutes on tables held in
+// registers. The products run on warp-level bf16 MMAs with 16 weight rows as
+// the M side and up to 8 routed rows per MMA as the N side. Every MMA chain
+// covers part of exactly one scale block (64 K for NF4, 32 K for MXFP4), so the
+// block sums leave the tensor core in fp32 and are scaled and accumulated in
+// fp32 outside it.
+//
+// At the end of each pass over an item the consumer warps hand their fp32
+// partial sums to an epilogue warp through double-buffered slots (kept in the
+// unused half of every 256-byte row of the lookup table) and go on; the
+// epilogue warp adds the K splits in a fixed order (deterministic), applies the
+// routing weight, rounds to bf16 and stores at the destination rows.
 //
 // MMA k-slot mapping: in m16n8k16, lane (g, t) supplies k-slots 2t, 2t+1,
 // 2t+8, 2t+9 of both operands. They are mapped to the four consecutive K
@@ -54,12 +59,15 @@ __device__ unsigned g_decode_error;
 namespace db {
 
 constexpr int kConsumers = 16;                     // consumer warps
-constexpr int kThreads = (kConsumers + 1) * 32;    // + one producer warp
+constexpr int kProducerWarp = kConsumers;          // one thread issues all copies
+constexpr int kEpilogueWarp = kConsumers + 1;      // reduces and stores the partial sums
+constexpr int kThreads = (kConsumers + 2) * 32;
 constexpr int kChunkK = 256;                       // K per stage: 128 packed bytes per row = one TMA box
 constexpr int kBoxBytes = 128;
 constexpr int kLutBytes = 256 * 256;               // byte value b, lane l -> offset b*256 + l*4
 constexpr int kXStride = kChunkK * 2 + 16;         // bytes per staged activation row (padded)
 constexpr int kMaxTableRows = 1024;                // routed rows whose metadata fits the CTA's table
+constexpr int kMaxRowTiles = 4;                    // ROWS / 16 for ROWS = 64
 
 struct Plan {
     int rows;         // weight rows per item (64 or 32)
@@ -106,6 +114,121 @@ __device__ __forceinline__ bool wait_tag(const int* tag, uint32_t want, volatile
     }
 }
 
+// Partial-sum slot of unit u (= ((buffer * row tiles + rt) * nks + ks) * GMAX + j)
+// for one lane: 512 bytes per unit, spread over four 128-byte holes of the lookup
+// table (bytes 128..255 of each 256-byte row, which the table leaves unused).
+__device__ __forceinline__ float4* red_slot(uint8_t* lut, int u, int lane) {
+    return reinterpret_cast<float4*>(lut + (u * 4 + (lane >> 3)) * 256 + 128 + (lane & 7) * 16);
+}
+
+// The MMAs of one chunk for one consumer warp: 16 weight rows (ra = row g, rb =
+// row g + 8 of the row tile) x NG groups of 8 routed rows x NBC scale blocks
+// (only the first nbc when the chunk is the ragged end of K).
+template <int FMT, int GMAX, int NG, bool FULL>
+__device__ __forceinline__ void chunk_mma(const uint8_t* __restrict__ st, const uint8_t* __restrict__ ss,
+                                          const uint8_t* __restrict__ lut, uint32_t lane_sel, const LutPlanes& L,
+                                          int ra, int rb, int g, int t, int nbk, int kc, int nbc, int wbytes,
+                                          bool vec_scales, float (&acc)[GMAX][4]) {
+    constexpr int SB = (FMT == FMT_NF4) ? 64 : 32;   // K elements per scale block
+    constexpr int STEPS = SB / 16;                   // k16 MMA steps per block
+    constexpr int BPL = SB / 8;                      // packed bytes per lane per row per block (8 or 4)
+    constexpr int XW = SB / 8;                       // bf16x2 words of x per lane per block
+    constexpr int NBC = kChunkK / SB;                // scale blocks in a full chunk (4 or 8)
+    const int bg0 = kc * NBC;                        // first scale block of the chunk
+    // block scales of rows ra and rb for this chunk
+    float sa[NBC], sb[NBC];
+    if (FULL && vec_scales) {
+        if constexpr (FMT == FMT_NF4) {
+            const float4 va = *reinterpret_cast<const float4*>(ss + (ra * nbk + bg0) * 4);
+            const float4 vb = *reinterpret_cast<const float4*>(ss + (rb * nbk + bg0) * 4);
+            sa[0] = va.x; sa[1] = va.y; sa[2] = va.z; sa[3] = va.w;
+            sb[0] = vb.x; sb[1] = vb.y; sb[2] = vb.z; sb[3] = vb.w;
+        } else {
+            const uint2 va = *reinterpret_cast<const uint2*>(ss + ra * nbk + bg0);
+            const uint2 vb = *reinterpret_cast<const uint2*>(ss + rb * nbk + bg0);
+#pragma unroll
+            for (int b = 0; b < NBC; ++b) {
+                sa[b] = e8m0_to_f32(((b < 4 ? va.x : va.y) >> (8 * (b & 3))) & 0xFFu);
+                sb[b] = e8m0_to_f32(((b < 4 ? vb.x : vb.y) >> (8 * (b & 3))) & 0xFFu);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int b = 0; b < NBC; ++b) {
+            if (FULL || b < nbc) {
+                if constexpr (FMT == FMT_NF4) {
+                    sa[b] = reinterpret_cast<const float*>(ss)[ra * nbk + bg0 + b];
+                    sb[b] = reinterpret_cast<const float*>(ss)[rb * nbk + bg0 + b];
+                } else {
+                    sa[b] = e8m0_to_f32(ss[ra * nbk + bg0 + b]);
+                    sb[b] = e8m0_to_f32(ss[rb * nbk + bg0 + b]);
+                }
+            } else {
+                sa[b] = sb[b] = 0.f;
+            }
+        }
+    }
+#pragma unroll
+    for (int b = 0; b < NBC; ++b) {
+        if (FULL || b < nbc) {
+            // this lane's packed bytes of rows ra and rb: byte o of the row's 128-byte
+            // chunk sits in 16-byte piece (o/16) ^ (row%8) of the swizzled box row
+            const int o = b * (SB / 2) + t * BPL;
+            const int pc = o >> 4, po = o & 15;
+            const uint8_t* rp0 = st + ra * kBoxBytes + ((pc ^ (ra & 7)) << 4) + po;
+            const uint8_t* rp1 = st + rb * kBoxBytes + ((pc ^ (rb & 7)) << 4) + po;
+            uint32_t w0[BPL / 4], w1[BPL / 4];
+            if constexpr (BPL == 8) {
+                const uint2 u0 = *reinterpret_cast<const uint2*>(rp0);
+                const uint2 u1 = *reinterpret_cast<const uint2*>(rp1);
+                w0[0] = u0.x; w0[BPL / 4 - 1] = u0.y;
+                w1[0] = u1.x; w1[BPL / 4 - 1] = u1.y;
+            } else {
+                w0[0] = *reinterpret_cast<const uint32_t*>(rp0);
+                w1[0] = *reinterpret_cast<const uint32_t*>(rp1);
+            }
+            // row ra by the shared-memory table, row rb by register byte permutes
+            uint32_t d0[BPL], d1[BPL];
+#pragma unroll
+            for (int j = 0; j < BPL; ++j) {
+                const uint32_t sel = 0x5504u | ((uint32_t)(j & 3) << 4);
+                d0[j] = *reinterpret_cast<const uint32_t*>(lut + prmt(w0[j >> 2], lane_sel, sel));
+            }
+#pragma unroll
+            for (int q = 0; q < BPL / 4; ++q) {
+                uint32_t o4[4];
+                decode_word<FMT>(w1[q], L, o4);
+                d1[4 * q] = o4[0]; d1[4 * q + 1] = o4[1]; d1[4 * q + 2] = o4[2]; d1[4 * q + 3] = o4[3];
+            }
+#pragma unroll
+            for (int j = 0; j < NG; ++j) {
+                // staged activations of routed row 8j + g of the pass (rows past the pass's
+                // end hold stale bytes; they only feed output columns that are never stored)
+                uint32_t xw[XW];
+                const uint8_t* xs = st + wbytes + (8 * j + g) * kXStride + (b * SB + t * (SB / 4)) * 2;
+#pragma unroll
+                for (int w = 0; w < XW / 4; ++w) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(xs + 16 * w);
+                    xw[4 * w] = v.x; xw[4 * w + 1] = v.y; xw[4 * w + 2] = v.z; xw[4 * w + 3] = v.w;
+                }
+                // two independent MMA chains per block (first and second half of its steps)
+                float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int s = 0; s < STEPS; ++s) {
+                    if (s < STEPS / 2)
+                        mma_bf16_16816(c0, d0[2 * s], d1[2 * s], d0[2 * s + 1], d1[2 * s + 1], xw[2 * s], xw[2 * s + 1]);
+                    else
+                        mma_bf16_16816(c1, d0[2 * s], d1[2 * s], d0[2 * s + 1], d1[2 * s + 1], xw[2 * s], xw[2 * s + 1]);
+                }
+                acc[j][0] = fmaf(c0[0] + c1[0], sa[b], acc[j][0]);
+                acc[j][1] = fmaf(c0[1] + c1[1], sa[b], acc[j][1]);
+                acc[j][2] = fmaf(c0[2] + c1[2], sb[b], acc[j][2]);
+                acc[j][3] = fmaf(c0[3] + c1[3], sb[b], acc[j][3]);
+            }
+        }
+    }
+}
+
 }  // namespace db
 
 template <int FMT, int GMAX>
@@ -113,21 +236,18 @@ __global__ void __launch_bounds__(db::kThreads, 1)
 decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_constant__ CUtensorMap wmap) {
     using namespace db;
     constexpr int SB = (FMT == FMT_NF4) ? 64 : 32;   // K elements per scale block
-    constexpr int STEPS = SB / 16;                   // k16 MMA steps per block
-    constexpr int BPL = SB / 8;                      // packed bytes per lane per row per block (8 or 4)
-    constexpr int XW = SB / 8;                       // bf16x2 words of x per lane per block
-    constexpr int NBC = kChunkK / SB;                // scale blocks in a full chunk (4 or 8)
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // [lut][ring: stages x stage_bytes][scale slots][red][barriers][abort, count][experts][row table]
+    // [lut (+ partial-sum slots in its holes)][ring: stages x stage_bytes][scale slots][barriers]
+    // [abort, count, tags][experts][row table]
     uint8_t* lut = smem;                                            // [256][64] words
     uint8_t* ring = smem + kLutBytes;                               // 1024-aligned stages
     uint8_t* sslots = ring + plan.nstages * plan.stage_bytes;
-    float4* red = reinterpret_cast<float4*>(sslots + plan.nslots * plan.scale_bytes);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(red + kConsumers * GMAX * 32);
-    // full[ns], empty[ns], scale slot free[nslots], scale slot full[nslots]
-    int* tailw = reinterpret_cast<int*>(bars + 2 * plan.nstages + 2 * plan.nslots);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sslots + plan.nslots * plan.scale_bytes);
+    // full[ns], empty[ns], scale slot free[nslots], scale slot full[nslots],
+    // partials ready[2][kMaxRowTiles], partial slots free[2][kMaxRowTiles]
+    int* tailw = reinterpret_cast<int*>(bars + 2 * plan.nstages + 2 * plan.nslots + 4 * kMaxRowTiles);
     volatile int* abort_flag = tailw;
     int* s_nact = tailw + 4;
     int* tags = tailw + 8;                                         // [ns] chunk counter last issued per slot
@@ -146,6 +266,8 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
     uint64_t* empty = bars + ns;
     uint64_t* sfree = bars + 2 * ns;
     uint64_t* sfull = bars + 2 * ns + nsl;
+    uint64_t* rready = bars + 2 * ns + 2 * nsl;                   // [buffer * kMaxRowTiles + rt]
+    uint64_t* rfree = rready + 2 * kMaxRowTiles;
 
     // byte -> bf16x2 table, one copy per lane
     const LutPlanes L = p.lut;                      // register copy (also for the permute decode)
@@ -173,7 +295,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
             count += __popc(bal);
         }
         if (lane == 0) s_nact[0] = count;
-    } else if (warp == kConsumers && lane == 0) {
+    } else if (warp == kProducerWarp && lane == 0) {
         for (int i = 0; i < ns; ++i) {
             mbar_init(smem_addr(full + i), 1);       // producer + tx bytes
             mbar_init(smem_addr(empty + i), nrt);    // the warps that own the chunk
@@ -181,6 +303,10 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
         for (int i = 0; i < nsl; ++i) {
             mbar_init(smem_addr(sfree + i), kConsumers);
             mbar_init(smem_addr(sfull + i), 1);
+        }
+        for (int i = 0; i < 2 * kMaxRowTiles; ++i) {
+            mbar_init(smem_addr(rready + i), nks);   // the K-split warps of the row tile
+            mbar_init(smem_addr(rfree + i), 1);      // the epilogue warp
         }
         for (int i = 0; i < ns; ++i) tags[i] = -1;
         *abort_flag = 0;
@@ -214,7 +340,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
     __syncthreads();
 
     const int nch = plan.nch;
-    if (warp == kConsumers) {
+    if (warp == kProducerWarp) {
         // ================= producer (one thread) =================
         if (lane == 0) {
             uint32_t ctr = 0, slot = 0, ph = 1;       // ring position; empty-barrier parity to wait on
@@ -279,20 +405,10 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
             }
         }
         __syncwarp();
-    } else {
-        // ================= consumers =================
-        const int rt = warp % nrt, ks = warp / nrt;     // row tile, K split (chunk counter % nks == ks)
-        const int g = lane >> 2, t = lane & 3;
-        const int ra = rt * 16 + g, rb = ra + 8;        // the two item rows of this lane
-        const uint32_t lane_sel = (uint32_t)lane * 4u;  // lut offset of this lane's copy
-        const bool vec_scales = (FMT == FMT_NF4) && (nbk % 4 == 0);
-        const uint32_t kmask = (uint32_t)nks - 1u;      // nks is 4 or 8
-        bool dead = false;   // set when a wait gives up: the warp then only keeps the barrier schedule
-        float acc[GMAX][4];
-#pragma unroll
-        for (int j = 0; j < GMAX; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-        uint32_t base = 0;                              // chunk counter at the start of the pass
-        uint32_t sslot = 0, sph = 0;                    // scale slot; its full-barrier parity
+    } else if (warp == kEpilogueWarp) {
+        // ================= epilogue: fixed-order K-split sums, weight, bf16, scatter =================
+        bool dead = false;
+        uint32_t P = 0;                                 // pass counter of the CTA
         int a = (i1 > i0) ? i0 / nit : 0, it = (i1 > i0) ? i0 % nit : 0;
         for (int item = i0; item < i1; ++item) {
             const int m = s_cnt[a];
@@ -300,13 +416,78 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
             const int64_t r0 = s_r0[a];
             const int npass = (m + 8 * GMAX - 1) / (8 * GMAX);
             const int vrows = min(ROWS, p.N - n0);
+            for (int pass = 0; pass < npass; ++pass, ++P) {
+                const int mc = pass * 8 * GMAX;
+                const int nvalid = min(8 * GMAX, m - mc);
+                const int G = (nvalid + 7) >> 3;
+                const uint32_t buf = P & 1u, ph = (P >> 1) & 1u;
+                for (int rt = 0; rt < nrt; ++rt) {
+                    const int bi = (int)buf * kMaxRowTiles + rt;
+                    if (!dead && !mbar_wait_bounded(smem_addr(rready + bi), ph, abort_flag, &g_decode_error, 32u))
+                        dead = true;
+                    if (!dead) {
+                        for (int q = lane; q < G * 32; q += 32) {
+                            const int j = q >> 5, ln = q & 31;
+                            float4 v = *red_slot(lut, (((int)buf * nrt + rt) * nks + 0) * GMAX + j, ln);
+                            for (int k2 = 1; k2 < nks; ++k2) {
+                                const float4 w = *red_slot(lut, (((int)buf * nrt + rt) * nks + k2) * GMAX + j, ln);
+                                v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+                            }
+                            const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int row = mc + 8 * j + 2 * (ln & 3) + (i & 1);       // C column 2t (+1)
+                                const int nr = rt * 16 + (ln >> 2) + ((i & 2) ? 8 : 0);    // C row g (+8)
+                                if (row < m && nr < vrows) {
+                                    const int64_t r = r0 + row;
+                                    float wgt;
+                                    int64_t dst;
+                                    if (table) {
+                                        wgt = t_wt[r - rlo];
+                                        dst = t_dst[r - rlo];
+                                    } else {
+                                        wgt = p.row_weight ? __ldg(p.row_weight + r) : 1.f;
+                                        dst = p.row_dest ? (int64_t)__ldg(p.row_dest + r) : r;
+                                    }
+                                    p.out[dst * p.N + n0 + nr] = f32_to_bf16_rne(vv[i] * wgt);
+                                }
+                            }
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_addr(rfree + bi));
+                }
+            }
+            if (++it == nit) {
+                it = 0;
+                ++a;
+            }
+        }
+    } else {
+        // ================= consumers =================
+        const int rt = warp % nrt, ks = warp / nrt;     // row tile, K split (chunk counter % nks == ks)
+        const int g = lane >> 2, t = lane & 3;
+        const int ra = rt * 16 + g, rb = ra + 8;        // the two item rows of this lane
+        const uint32_t lane_sel = (uint32_t)lane * 4u;  // lut offset of this lane's copy
+        const bool vec_scales = (FMT == FMT_NF4) ? (nbk % 4 == 0) : (nbk % 8 == 0);
+        const uint32_t kmask = (uint32_t)nks - 1u;      // nks is 4 or 8
+        bool dead = false;   // set when a wait gives up: the warp then only keeps the barrier schedule
+        float acc[GMAX][4];
+#pragma unroll
+        for (int j = 0; j < GMAX; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+        uint32_t base = 0;                              // chunk counter at the start of the pass
+        uint32_t P = 0;                                 // pass counter of the CTA
+        uint32_t sslot = 0, sph = 0;                    // scale slot; its full-barrier parity
+        int a = (i1 > i0) ? i0 / nit : 0, it = (i1 > i0) ? i0 % nit : 0;
+        for (int item = i0; item < i1; ++item) {
+            const int m = s_cnt[a];
+            const int npass = (m + 8 * GMAX - 1) / (8 * GMAX);
             // every warp waits for the item's scales (also those that own no chunk of it)
             if (!dead && !mbar_wait_bounded(smem_addr(sfull + sslot), sph, abort_flag, &g_decode_error, 8u))
                 dead = true;
             const uint8_t* ss = sslots + sslot * plan.scale_bytes;
-            for (int pass = 0; pass < npass; ++pass) {
-                const int mc = pass * 8 * GMAX;
-                const int nvalid = min(8 * GMAX, m - mc);   // routed rows of this pass
+            for (int pass = 0; pass < npass; ++pass, ++P) {
+                const int nvalid = min(8 * GMAX, m - pass * 8 * GMAX);   // routed rows of this pass
                 int kc = (int)(((uint32_t)ks - base) & kmask);
                 uint32_t ctr = base + (uint32_t)kc;
                 uint32_t slot = ctr % (uint32_t)ns, ph = (ctr / (uint32_t)ns) & 1u;
@@ -314,96 +495,22 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
                     if (!dead && !wait_tag(tags + slot, ctr, abort_flag, &g_decode_error, 16u)) dead = true;
                     if (!dead && !mbar_wait_bounded(smem_addr(full + slot), ph, abort_flag, &g_decode_error, 2u))
                         dead = true;
+                    if (!dead) {
                         const uint8_t* st = ring + slot * plan.stage_bytes;
                         const int kb = kc * kChunkK;
-                        const int nbc = min(kChunkK, p.K - kb) / SB;
-                        const int bg0 = kc * NBC;                 // first scale block of the chunk
-                        // block scales of rows ra and rb for this chunk
-                        float sa[NBC], sb[NBC];
-                        if (!dead) {
-                            if (vec_scales && nbc == NBC) {
-                                const float4 va = *reinterpret_cast<const float4*>(ss + (ra * nbk + bg0) * 4);
-                                const float4 vb = *reinterpret_cast<const float4*>(ss + (rb * nbk + bg0) * 4);
-                                sa[0] = va.x; sa[1] = va.y; sa[2] = va.z; sa[3] = va.w;
-                                sb[0] = vb.x; sb[1] = vb.y; sb[2] = vb.z; sb[3] = vb.w;
-                            } else {
-        #pragma unroll
-                                for (int b = 0; b < NBC; ++b) {
-                                    if (b < nbc) {
-                                        if constexpr (FMT == FMT_NF4) {
-                                            sa[b] = reinterpret_cast<const float*>(ss)[ra * nbk + bg0 + b];
-                                            sb[b] = reinterpret_cast<const float*>(ss)[rb * nbk + bg0 + b];
-                                        } else {
-                                            sa[b] = e8m0_to_f32(ss[ra * nbk + bg0 + b]);
-                                            sb[b] = e8m0_to_f32(ss[rb * nbk + bg0 + b]);
-                                        }
-                                    } else {
-                                        sa[b] = sb[b] = 0.f;
-                                    }
-                                }
-                            }
+                        if (p.K - kb >= kChunkK) {
+                            if (GMAX == 2 && nvalid > 8)
+                                chunk_mma<FMT, GMAX, (GMAX == 2 ? 2 : 1), true>(st, ss, lut, lane_sel, L, ra, rb, g, t, nbk, kc,
+                                                                                0, plan.wbytes, vec_scales, acc);
+                            else
+                                chunk_mma<FMT, GMAX, 1, true>(st, ss, lut, lane_sel, L, ra, rb, g, t, nbk, kc, 0,
+                                                              plan.wbytes, vec_scales, acc);
+                        } else {
+                            const int nbc = (p.K - kb) / SB;
+                            chunk_mma<FMT, GMAX, GMAX, false>(st, ss, lut, lane_sel, L, ra, rb, g, t, nbk, kc, nbc,
+                                                              plan.wbytes, vec_scales, acc);
                         }
-        #pragma unroll
-                        for (int b = 0; b < NBC; ++b) {
-                            if (!dead && b < nbc) {
-                                // this lane's packed bytes of rows ra and rb: byte o of the row's 128-byte
-                                // chunk sits in 16-byte piece (o/16) ^ (row%8) of the swizzled box row
-                                const int o = b * (SB / 2) + t * BPL;
-                                const int pc = o >> 4, po = o & 15;
-                                const uint8_t* rp0 = st + ra * kBoxBytes + ((pc ^ (ra & 7)) << 4) + po;
-                                const uint8_t* rp1 = st + rb * kBoxBytes + ((pc ^ (rb & 7)) << 4) + po;
-                                uint32_t w0[BPL / 4], w1[BPL / 4];
-                                if constexpr (BPL == 8) {
-                                    const uint2 u0 = *reinterpret_cast<const uint2*>(rp0);
-                                    const uint2 u1 = *reinterpret_cast<const uint2*>(rp1);
-                                    w0[0] = u0.x; w0[BPL / 4 - 1] = u0.y;
-                                    w1[0] = u1.x; w1[BPL / 4 - 1] = u1.y;
-                                } else {
-                                    w0[0] = *reinterpret_cast<const uint32_t*>(rp0);
-                                    w1[0] = *reinterpret_cast<const uint32_t*>(rp1);
-                                }
-                                // row ra by the shared-memory table, row rb by register byte permutes
-                                uint32_t d0[BPL], d1[BPL];
-        #pragma unroll
-                                for (int j = 0; j < BPL; ++j) {
-                                    const uint32_t sel = 0x5504u | ((uint32_t)(j & 3) << 4);
-                                    d0[j] = *reinterpret_cast<const uint32_t*>(lut + prmt(w0[j >> 2], lane_sel, sel));
-                                }
-        #pragma unroll
-                                for (int q = 0; q < BPL / 4; ++q) {
-                                    uint32_t o4[4];
-                                    decode_word<FMT>(w1[q], L, o4);
-                                    d1[4 * q] = o4[0]; d1[4 * q + 1] = o4[1]; d1[4 * q + 2] = o4[2]; d1[4 * q + 3] = o4[3];
-                                }
-        #pragma unroll
-                                for (int j = 0; j < GMAX; ++j) {
-                                    if (8 * j < nvalid) {
-                                        // staged activations of routed row mc + 8j + g (lanes past the pass's
-                                        // rows feed output columns that are never stored)
-                                        uint32_t xw[XW];
-        #pragma unroll
-                                        for (int w = 0; w < XW; ++w) xw[w] = 0u;
-                                        if (8 * j + g < nvalid) {
-                                            const uint8_t* xs = st + plan.wbytes + (8 * j + g) * kXStride + (b * SB + t * (SB / 4)) * 2;
-        #pragma unroll
-                                            for (int w = 0; w < XW / 4; ++w) {
-                                                const uint4 v = *reinterpret_cast<const uint4*>(xs + 16 * w);
-                                                xw[4 * w] = v.x; xw[4 * w + 1] = v.y; xw[4 * w + 2] = v.z; xw[4 * w + 3] = v.w;
-                                            }
-                                        }
-                                        float cb[4] = {0.f, 0.f, 0.f, 0.f};
-        #pragma unroll
-                                        for (int s = 0; s < STEPS; ++s)
-                                            mma_bf16_16816(cb, d0[2 * s], d1[2 * s], d0[2 * s + 1], d1[2 * s + 1], xw[2 * s],
-                                                           xw[2 * s + 1]);
-                                        acc[j][0] = fmaf(cb[0], sa[b], acc[j][0]);
-                                        acc[j][1] = fmaf(cb[1], sa[b], acc[j][1]);
-                                        acc[j][2] = fmaf(cb[2], sb[b], acc[j][2]);
-                                        acc[j][3] = fmaf(cb[3], sb[b], acc[j][3]);
-                                    }
-                                }
-                            }
-                        }
+                    }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_addr(empty + slot));
                     ctr += (uint32_t)nks;
@@ -414,35 +521,19 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
                     }
                 }
                 base += (uint32_t)nch;
-                // end of a pass: the row tile's K-split partial sums, added in a fixed order
-                const int G = min(GMAX, (nvalid + 7) >> 3);
+                // end of a pass: hand the partial sums to the epilogue warp
+                const uint32_t buf = P & 1u, fph = ((P >> 1) & 1u) ^ 1u;
+                const int bi = (int)buf * kMaxRowTiles + rt;
+                if (!dead && !mbar_wait_bounded(smem_addr(rfree + bi), fph, abort_flag, &g_decode_error, 64u))
+                    dead = true;
+                if (!dead) {
 #pragma unroll
-                for (int j = 0; j < GMAX; ++j)
-                    if (j < G) red[((rt * nks + ks) * GMAX + j) * 32 + lane] =
-                                   make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
-                asm volatile("bar.sync %0, %1;" ::"r"(1 + rt), "r"(nks * 32) : "memory");
-                for (int qq = ks * 32 + lane; qq < G * 128; qq += nks * 32) {
-                    const int i = qq & 3, ln = (qq >> 2) & 31, j = qq >> 7;
-                    const int row = mc + 8 * j + 2 * (ln & 3) + (i & 1);       // C column 2t (+1)
-                    const int nr = rt * 16 + (ln >> 2) + ((i & 2) ? 8 : 0);    // C row g (+8)
-                    if (row < m && nr < vrows) {
-                        float v = 0.f;
-                        for (int k2 = 0; k2 < nks; ++k2)
-                            v += reinterpret_cast<const float*>(&red[((rt * nks + k2) * GMAX + j) * 32 + ln])[i];
-                        const int64_t r = r0 + row;
-                        float wgt;
-                        int64_t dst;
-                        if (table) {
-                            wgt = t_wt[r - rlo];
-                            dst = t_dst[r - rlo];
-                        } else {
-                            wgt = p.row_weight ? __ldg(p.row_weight + r) : 1.f;
-                            dst = p.row_dest ? (int64_t)__ldg(p.row_dest + r) : r;
-                        }
-                        p.out[dst * p.N + n0 + nr] = f32_to_bf16_rne(v * wgt);
-                    }
+                    for (int j = 0; j < GMAX; ++j)
+                        *red_slot(lut, (((int)buf * nrt + rt) * nks + ks) * GMAX + j, lane) =
+                            make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
                 }
-                asm volatile("bar.sync %0, %1;" ::"r"(1 + rt), "r"(nks * 32) : "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(rready + bi));
 #pragma unroll
                 for (int j = 0; j < GMAX; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
             }
@@ -480,7 +571,6 @@ static cudaError_t launch_db(const GroupedArgs& a, cudaStream_t s) {
     const int ssz = (FMT == FMT_NF4) ? 4 : 1;
     Plan plan;
     plan.nch = (a.K + kChunkK - 1) / kChunkK;
-    const int red_bytes = kConsumers * GMAX * 32 * (int)sizeof(float4);
     const int tables = 32 + 16 * a.E + 12 * kMaxTableRows;
     int smem = 0;
     plan.rows = 0;
@@ -491,8 +581,8 @@ static cudaError_t launch_db(const GroupedArgs& a, cudaStream_t s) {
         const int nks = kConsumers * 16 / rows;          // K-split warps per row tile: the ring holds at least one chunk each
         for (int nst = 12; nst >= nks; --nst) {
             for (int nsl = 3; nsl >= 2; --nsl) {
-                const int need = 1024 + kLutBytes + nst * stage_bytes + nsl * scale_bytes + red_bytes +
-                                 (2 * nst + 2 * nsl) * 8 + 4 * ((nst + 1) & ~1) + tables;
+                const int need = 1024 + kLutBytes + nst * stage_bytes + nsl * scale_bytes +
+                                 (2 * nst + 2 * nsl + 4 * kMaxRowTiles) * 8 + 4 * ((nst + 1) & ~1) + tables;
                 if (need <= 226 * 1024) {
                     plan.rows = rows;
                     plan.wbytes = wbytes;
