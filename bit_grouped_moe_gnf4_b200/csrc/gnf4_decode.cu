@@ -7,30 +7,30 @@
 // One persistent CTA per SM takes a contiguous run of work items; an item is
 // (active expert, ROWS = 64 weight rows; 32 when K is very large). A producer
 // thread streams each item's packed rows, one K chunk of 256 at a time, into a
-// ring of shared-memory stages with one 2-D TMA load per chunk (a box of 128
-// bytes x ROWS rows, 128B-swizzled), several stages ahead; big requests are what
-// lets the copy engine keep HBM busy. The same stage also carries the chunk of
-// each routed row's activations (1-D bulk copies, one per row). The item's block
-// scales (ROWS rows x all blocks, one contiguous range) land in a scale slot
-// with a barrier of their own. The CTA's routing metadata (token, weight,
-// destination of each of its routed rows) is staged in shared memory once.
+// ring of 8 KB shared-memory stages with one 2-D TMA load per chunk (a box of
+// 128 bytes x ROWS rows, 128B-swizzled); the stage holds nothing else, so the
+// producer issues one copy per stage and the copy engine keeps HBM busy. The
+// item's block scales (ROWS rows x all blocks, one contiguous range) land in a
+// scale slot with a barrier of their own, issued one item ahead.
 //
-// 16 consumer warps: warp (rt, ks) owns row tile rt (16 rows of the item) and
-// every nks-th chunk of the CTA's stream (chunk counter % nks == ks), so each
-// stage is read by ROWS/16 warps and stages are consumed in parallel. Because
-// owners skip the stages of other warps, a ring slot carries a tag naming the
-// chunk that was last issued into it; an owner reads the slot's barrier only
-// once the tag shows its chunk, which keeps every parity wait within one phase.
+// 12 consumer warps: warp (rt, ks) owns row tile rt (16 rows of the item) and
+// every nks-th chunk of the CTA's stream (chunk counter % nks == ks; nks = 3
+// for 64-row items), so each stage is read by ROWS/16 warps and stages are
+// consumed in parallel. Because owners skip the stages of other warps, a ring
+// slot carries a tag naming the chunk that was last issued into it; an owner
+// reads the slot's barrier only once the tag shows its chunk, which keeps
+// every parity wait within one phase.
 //
-// Nibbles are decoded two ways, to balance the shared-memory and ALU pipes: one
-// of the lane's two rows by a table in shared memory that maps each packed byte
-// to its two bf16 values (replicated per lane, so 32 lookups never conflict; a
-// byte permute forms the address), the other by byte permutes on tables held in
-// registers. The products run on warp-level bf16 MMAs with 16 weight rows as
-// the M side and up to 8 routed rows per MMA as the N side. Every MMA chain
-// covers part of exactly one scale block (64 K for NF4, 32 K for MXFP4), so the
-// block sums leave the tensor core in fp32 and are scaled and accumulated in
-// fp32 outside it.
+// The activations of the routed rows are small and shared by every item of an
+// expert, so the consumers read them straight from global memory through L1
+// (prefetched into L1 before the wait for the chunk's weights). Nibbles are
+// decoded by a table in shared memory that maps each packed byte to its two
+// bf16 values (replicated per lane, so 32 lookups never conflict; a byte
+// permute forms the address). The products run on warp-level bf16 MMAs with 16
+// weight rows as the M side and up to 8 routed rows per MMA as the N side.
+// Every MMA chain covers exactly one scale block (64 K for NF4, 32 K for
+// MXFP4), so the block sum leaves the tensor core in fp32 and is scaled and
+// accumulated in fp32 outside it.
 //
 // At the end of each pass over an item the consumer warps hand their fp32
 // partial sums to an epilogue warp through double-buffered slots (kept in the
@@ -58,22 +58,21 @@ __device__ unsigned g_decode_error;
 
 namespace db {
 
-constexpr int kConsumers = 16;                     // consumer warps
+constexpr int kConsumers = 12;                     // consumer warps: 4 row tiles x 3 K-split owners
 constexpr int kProducerWarp = kConsumers;          // one thread issues all copies
 constexpr int kEpilogueWarp = kConsumers + 1;      // reduces and stores the partial sums
-constexpr int kThreads = (kConsumers + 2) * 32;
+constexpr int kThreads = (kConsumers + 2) * 32;    // 14 warps: at most 4 per SM sub-partition,
+constexpr int kRegBound = 512;                     // so 128 registers a thread (bounds for 16 warps)
 constexpr int kChunkK = 256;                       // K per stage: 128 packed bytes per row = one TMA box
 constexpr int kBoxBytes = 128;
 constexpr int kLutBytes = 256 * 256;               // byte value b, lane l -> offset b*256 + l*4
-constexpr int kXStride = kChunkK * 2 + 16;         // bytes per staged activation row (padded)
 constexpr int kMaxTableRows = 1024;                // routed rows whose metadata fits the CTA's table
 constexpr int kMaxRowTiles = 4;                    // ROWS / 16 for ROWS = 64
 
 struct Plan {
     int rows;         // weight rows per item (64 or 32)
     int nch;          // stages per item pass
-    int wbytes;       // packed-weight part of a stage: rows x 128 bytes
-    int stage_bytes;  // wbytes + activation rows (8*GMAX x kXStride), rounded to 1024
+    int stage_bytes;  // rows x 128 bytes (a multiple of 1024)
     int scale_bytes;  // slot for one item's scales (rows x all blocks), rounded to 128
     int nstages;      // ring stages
     int nslots;       // item scale slots
@@ -114,6 +113,10 @@ __device__ __forceinline__ bool wait_tag(const int* tag, uint32_t want, volatile
     }
 }
 
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
 // Partial-sum slot of unit u (= ((buffer * row tiles + rt) * nks + ks) * GMAX + j)
 // for one lane: 512 bytes per unit, spread over four 128-byte holes of the lookup
 // table (bytes 128..255 of each 256-byte row, which the table leaves unused).
@@ -126,51 +129,52 @@ __device__ __forceinline__ float4* red_slot(uint8_t* lut, int u, int lane) {
 // (only the first nbc when the chunk is the ragged end of K).
 template <int FMT, int GMAX, int NG, bool FULL>
 __device__ __forceinline__ void chunk_mma(const uint8_t* __restrict__ st, const uint8_t* __restrict__ ss,
-                                          const uint8_t* __restrict__ lut, uint32_t lane_sel, const LutPlanes& L,
-                                          int ra, int rb, int g, int t, int nbk, int kc, int nbc, int wbytes,
-                                          bool vec_scales, float (&acc)[GMAX][4]) {
+                                          const uint8_t* __restrict__ lut, uint32_t lane_sel,
+                                          const uint16_t* xr0, const uint16_t* xr1, int ra, int rb, int t, int nbk,
+                                          int kc, int nbc, bool vec_scales, float (&acc)[GMAX][4]) {
     constexpr int SB = (FMT == FMT_NF4) ? 64 : 32;   // K elements per scale block
     constexpr int STEPS = SB / 16;                   // k16 MMA steps per block
     constexpr int BPL = SB / 8;                      // packed bytes per lane per row per block (8 or 4)
     constexpr int XW = SB / 8;                       // bf16x2 words of x per lane per block
     constexpr int NBC = kChunkK / SB;                // scale blocks in a full chunk (4 or 8)
     const int bg0 = kc * NBC;                        // first scale block of the chunk
-    // block scales of rows ra and rb for this chunk
-    float sa[NBC], sb[NBC];
-    if (FULL && vec_scales) {
+    // block scales of rows ra and rb for this chunk: one vector load per row when the
+    // rows' blocks are aligned for it, picked per block by selects (no local arrays)
+    float4 va4 = make_float4(0.f, 0.f, 0.f, 0.f), vb4 = va4;
+    uint2 va2 = make_uint2(0u, 0u), vb2 = va2;
+    const bool vec = FULL && vec_scales;
+    if (vec) {
         if constexpr (FMT == FMT_NF4) {
-            const float4 va = *reinterpret_cast<const float4*>(ss + (ra * nbk + bg0) * 4);
-            const float4 vb = *reinterpret_cast<const float4*>(ss + (rb * nbk + bg0) * 4);
-            sa[0] = va.x; sa[1] = va.y; sa[2] = va.z; sa[3] = va.w;
-            sb[0] = vb.x; sb[1] = vb.y; sb[2] = vb.z; sb[3] = vb.w;
+            va4 = *reinterpret_cast<const float4*>(ss + (ra * nbk + bg0) * 4);
+            vb4 = *reinterpret_cast<const float4*>(ss + (rb * nbk + bg0) * 4);
         } else {
-            const uint2 va = *reinterpret_cast<const uint2*>(ss + ra * nbk + bg0);
-            const uint2 vb = *reinterpret_cast<const uint2*>(ss + rb * nbk + bg0);
-#pragma unroll
-            for (int b = 0; b < NBC; ++b) {
-                sa[b] = e8m0_to_f32(((b < 4 ? va.x : va.y) >> (8 * (b & 3))) & 0xFFu);
-                sb[b] = e8m0_to_f32(((b < 4 ? vb.x : vb.y) >> (8 * (b & 3))) & 0xFFu);
-            }
-        }
-    } else {
-#pragma unroll
-        for (int b = 0; b < NBC; ++b) {
-            if (FULL || b < nbc) {
-                if constexpr (FMT == FMT_NF4) {
-                    sa[b] = reinterpret_cast<const float*>(ss)[ra * nbk + bg0 + b];
-                    sb[b] = reinterpret_cast<const float*>(ss)[rb * nbk + bg0 + b];
-                } else {
-                    sa[b] = e8m0_to_f32(ss[ra * nbk + bg0 + b]);
-                    sb[b] = e8m0_to_f32(ss[rb * nbk + bg0 + b]);
-                }
-            } else {
-                sa[b] = sb[b] = 0.f;
-            }
+            va2 = *reinterpret_cast<const uint2*>(ss + ra * nbk + bg0);
+            vb2 = *reinterpret_cast<const uint2*>(ss + rb * nbk + bg0);
         }
     }
-#pragma unroll
+#pragma unroll 2
     for (int b = 0; b < NBC; ++b) {
         if (FULL || b < nbc) {
+            float sa, sb;
+            if (vec) {
+                if constexpr (FMT == FMT_NF4) {
+                    const int i = b & 3;
+                    sa = i == 0 ? va4.x : i == 1 ? va4.y : i == 2 ? va4.z : va4.w;
+                    sb = i == 0 ? vb4.x : i == 1 ? vb4.y : i == 2 ? vb4.z : vb4.w;
+                } else {
+                    const uint32_t sh = 8u * (uint32_t)(b & 3);
+                    sa = e8m0_to_f32(((b < 4 ? va2.x : va2.y) >> sh) & 0xFFu);
+                    sb = e8m0_to_f32(((b < 4 ? vb2.x : vb2.y) >> sh) & 0xFFu);
+                }
+            } else {
+                if constexpr (FMT == FMT_NF4) {
+                    sa = reinterpret_cast<const float*>(ss)[ra * nbk + bg0 + b];
+                    sb = reinterpret_cast<const float*>(ss)[rb * nbk + bg0 + b];
+                } else {
+                    sa = e8m0_to_f32(ss[ra * nbk + bg0 + b]);
+                    sb = e8m0_to_f32(ss[rb * nbk + bg0 + b]);
+                }
+            }
             // this lane's packed bytes of rows ra and rb: byte o of the row's 128-byte
             // chunk sits in 16-byte piece (o/16) ^ (row%8) of the swizzled box row
             const int o = b * (SB / 2) + t * BPL;
@@ -187,29 +191,29 @@ __device__ __forceinline__ void chunk_mma(const uint8_t* __restrict__ st, const 
                 w0[0] = *reinterpret_cast<const uint32_t*>(rp0);
                 w1[0] = *reinterpret_cast<const uint32_t*>(rp1);
             }
-            // row ra by the shared-memory table, row rb by register byte permutes
+            // both rows by the shared-memory table
             uint32_t d0[BPL], d1[BPL];
 #pragma unroll
             for (int j = 0; j < BPL; ++j) {
                 const uint32_t sel = 0x5504u | ((uint32_t)(j & 3) << 4);
                 d0[j] = *reinterpret_cast<const uint32_t*>(lut + prmt(w0[j >> 2], lane_sel, sel));
-            }
-#pragma unroll
-            for (int q = 0; q < BPL / 4; ++q) {
-                uint32_t o4[4];
-                decode_word<FMT>(w1[q], L, o4);
-                d1[4 * q] = o4[0]; d1[4 * q + 1] = o4[1]; d1[4 * q + 2] = o4[2]; d1[4 * q + 3] = o4[3];
+                d1[j] = *reinterpret_cast<const uint32_t*>(lut + prmt(w1[j >> 2], lane_sel, sel));
             }
 #pragma unroll
             for (int j = 0; j < NG; ++j) {
-                // staged activations of routed row 8j + g of the pass (rows past the pass's
-                // end hold stale bytes; they only feed output columns that are never stored)
+                // activations of routed row 8j + g of the pass, from global memory (L1);
+                // lanes past the pass's rows feed zeros to output columns never stored
                 uint32_t xw[XW];
-                const uint8_t* xs = st + wbytes + (8 * j + g) * kXStride + (b * SB + t * (SB / 4)) * 2;
 #pragma unroll
-                for (int w = 0; w < XW / 4; ++w) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(xs + 16 * w);
-                    xw[4 * w] = v.x; xw[4 * w + 1] = v.y; xw[4 * w + 2] = v.z; xw[4 * w + 3] = v.w;
+                for (int w = 0; w < XW; ++w) xw[w] = 0u;
+                const uint16_t* xr = (j == 0) ? xr0 : xr1;
+                if (xr != nullptr) {
+                    const uint4* xs = reinterpret_cast<const uint4*>(xr + kc * kChunkK + b * SB + t * (SB / 4));
+#pragma unroll
+                    for (int w = 0; w < XW / 4; ++w) {
+                        const uint4 v = __ldg(xs + w);
+                        xw[4 * w] = v.x; xw[4 * w + 1] = v.y; xw[4 * w + 2] = v.z; xw[4 * w + 3] = v.w;
+                    }
                 }
                 // two independent MMA chains per block (first and second half of its steps)
                 float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
@@ -220,10 +224,10 @@ __device__ __forceinline__ void chunk_mma(const uint8_t* __restrict__ st, const 
                     else
                         mma_bf16_16816(c1, d0[2 * s], d1[2 * s], d0[2 * s + 1], d1[2 * s + 1], xw[2 * s], xw[2 * s + 1]);
                 }
-                acc[j][0] = fmaf(c0[0] + c1[0], sa[b], acc[j][0]);
-                acc[j][1] = fmaf(c0[1] + c1[1], sa[b], acc[j][1]);
-                acc[j][2] = fmaf(c0[2] + c1[2], sb[b], acc[j][2]);
-                acc[j][3] = fmaf(c0[3] + c1[3], sb[b], acc[j][3]);
+                acc[j][0] = fmaf(c0[0] + c1[0], sa, acc[j][0]);
+                acc[j][1] = fmaf(c0[1] + c1[1], sa, acc[j][1]);
+                acc[j][2] = fmaf(c0[2] + c1[2], sb, acc[j][2]);
+                acc[j][3] = fmaf(c0[3] + c1[3], sb, acc[j][3]);
             }
         }
     }
@@ -232,7 +236,7 @@ __device__ __forceinline__ void chunk_mma(const uint8_t* __restrict__ st, const 
 }  // namespace db
 
 template <int FMT, int GMAX>
-__global__ void __launch_bounds__(db::kThreads, 1)
+__global__ void __launch_bounds__(db::kRegBound, 1)
 decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_constant__ CUtensorMap wmap) {
     using namespace db;
     constexpr int SB = (FMT == FMT_NF4) ? 64 : 32;   // K elements per scale block
@@ -240,7 +244,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     // [lut (+ partial-sum slots in its holes)][ring: stages x stage_bytes][scale slots][barriers]
-    // [abort, count, tags][experts][row table]
+    // [abort, count, warp counts, tags][experts][row table]
     uint8_t* lut = smem;                                            // [256][64] words
     uint8_t* ring = smem + kLutBytes;                               // 1024-aligned stages
     uint8_t* sslots = ring + plan.nstages * plan.stage_bytes;
@@ -249,9 +253,9 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
     // partials ready[2][kMaxRowTiles], partial slots free[2][kMaxRowTiles]
     int* tailw = reinterpret_cast<int*>(bars + 2 * plan.nstages + 2 * plan.nslots + 4 * kMaxRowTiles);
     volatile int* abort_flag = tailw;
-    int* s_nact = tailw + 4;
-    int* tags = tailw + 8;                                         // [ns] chunk counter last issued per slot
-    int64_t* s_r0 = reinterpret_cast<int64_t*>(tailw + 8 + ((plan.nstages + 1) & ~1)); // [E] first routed row
+    int* s_wcnt = tailw + 8;                                       // [16] active experts per warp (scan)
+    int* tags = tailw + 24;                                        // [ns] chunk counter last issued per slot
+    int64_t* s_r0 = reinterpret_cast<int64_t*>(tailw + 24 + ((plan.nstages + 1) & ~1)); // [E] first routed row
     int* s_active = reinterpret_cast<int*>(s_r0 + p.E);            // [E] expert id
     int* s_cnt = s_active + p.E;                                   // [E] routed rows
     int* t_tok = s_cnt + p.E;                                      // [kMaxTableRows] per routed row
@@ -269,33 +273,16 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
     uint64_t* rready = bars + 2 * ns + 2 * nsl;                   // [buffer * kMaxRowTiles + rt]
     uint64_t* rfree = rready + 2 * kMaxRowTiles;
 
-    // byte -> bf16x2 table, one copy per lane
-    const LutPlanes L = p.lut;                      // register copy (also for the permute decode)
-    for (int i = threadIdx.x; i < 256 * 32; i += kThreads) {
-        const int b = i >> 5, l = i & 31;
-        *reinterpret_cast<uint32_t*>(lut + b * 256 + l * 4) = byte_bf16x2<FMT>((uint32_t)b, L);
-    }
-    if (warp == 0) {
-        // experts of this band, in id order (every CTA derives the same list)
-        int count = 0;
-        for (int e0 = 0; e0 < p.E; e0 += 32) {
-            const int e = e0 + lane;
-            bool act = false;
-            if (e < p.E) {
-                const int64_t m = p.offsets[e + 1] - p.offsets[e];
-                act = (m >= p.m_lo) && (m <= p.m_hi);
-            }
-            const unsigned bal = __ballot_sync(0xffffffffu, act);
-            if (act) {
-                const int idx = count + __popc(bal & ((1u << lane) - 1u));
-                s_active[idx] = e;
-                s_r0[idx] = p.offsets[e];
-                s_cnt[idx] = (int)(p.offsets[e + 1] - p.offsets[e]);
-            }
-            count += __popc(bal);
+    // byte -> bf16x2 table, one copy per lane: 8 sixteen-byte pieces per byte value
+    {
+        const LutPlanes L = p.lut;
+        for (int i = threadIdx.x; i < 256 * 8; i += kThreads) {
+            const int b = i >> 3, q = i & 7;
+            const uint32_t v = byte_bf16x2<FMT>((uint32_t)b, L);
+            *reinterpret_cast<uint4*>(lut + b * 256 + q * 16) = make_uint4(v, v, v, v);
         }
-        if (lane == 0) s_nact[0] = count;
-    } else if (warp == kProducerWarp && lane == 0) {
+    }
+    if (warp == kProducerWarp && lane == 0) {
         for (int i = 0; i < ns; ++i) {
             mbar_init(smem_addr(full + i), 1);       // producer + tx bytes
             mbar_init(smem_addr(empty + i), nrt);    // the warps that own the chunk
@@ -312,10 +299,39 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    __syncthreads();
+    // experts of this band, in id order (every CTA derives the same list): one
+    // expert per thread, a ballot per warp, a prefix over the warps
+    int nact = 0;
+    for (int e0 = 0; e0 < p.E; e0 += kThreads) {
+        const int e = e0 + (int)threadIdx.x;
+        bool act = false;
+        int64_t o0 = 0, o1 = 0;
+        if (e < p.E) {
+            o0 = p.offsets[e];
+            o1 = p.offsets[e + 1];
+            act = (o1 - o0 >= p.m_lo) && (o1 - o0 <= p.m_hi);
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, act);
+        if (lane == 0) s_wcnt[warp] = __popc(bal);
+        __syncthreads();
+        int before = nact, total = 0;
+        for (int w = 0; w < kThreads / 32; ++w) {
+            const int c = s_wcnt[w];
+            if (w < warp) before += c;
+            total += c;
+        }
+        if (act) {
+            const int idx = before + __popc(bal & ((1u << lane) - 1u));
+            s_active[idx] = e;
+            s_r0[idx] = o0;
+            s_cnt[idx] = (int)(o1 - o0);
+        }
+        nact += total;
+        __syncthreads();
+    }
 
     const int nit = (p.N + ROWS - 1) / ROWS;           // items per expert
-    const int total = s_nact[0] * nit;
+    const int total = nact * nit;
     const int i0 = (int)((int64_t)blockIdx.x * total / gridDim.x);
     const int i1 = (int)((int64_t)(blockIdx.x + 1) * total / gridDim.x);
     const int nbk = p.K / SB;                          // scale blocks per weight row
@@ -329,37 +345,29 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
         rhi = s_r0[a1] + s_cnt[a1];
     }
     const bool table = (rhi - rlo) <= kMaxTableRows;
-    if (table) {
-        for (int64_t r = rlo + threadIdx.x; r < rhi; r += kThreads) {
-            const int k = (int)(r - rlo);
-            t_tok[k] = p.row_token ? __ldg(p.row_token + r) : (int)r;
-            t_wt[k] = p.row_weight ? __ldg(p.row_weight + r) : 1.f;
-            t_dst[k] = p.row_dest ? __ldg(p.row_dest + r) : (int)r;
-        }
-    }
-    __syncthreads();
 
     const int nch = plan.nch;
     if (warp == kProducerWarp) {
-        // ================= producer (one thread) =================
+        // ================= producer (one thread): starts right away =================
         if (lane == 0) {
             uint32_t ctr = 0, slot = 0, ph = 1;       // ring position; empty-barrier parity to wait on
-            uint32_t sslot = 0, sph = 1;              // scale slot; its free-barrier parity
-            int a = (i1 > i0) ? i0 / nit : 0, it = (i1 > i0) ? i0 % nit : 0;
+            uint32_t sslot = 0, sph = 1;              // next scale slot to fill; its free-barrier parity
+            int sa_ = (i1 > i0) ? i0 / nit : 0, sit = (i1 > i0) ? i0 % nit : 0;   // next item whose scales go out
+            int s_next = i0;
+            int a = sa_, it = sit;
             bool ok = true;
             for (int item = i0; item < i1 && ok; ++item) {
-                const int e = s_active[a];
-                const int n0 = it * ROWS;
-                const int cnt = s_cnt[a];
-                const int64_t r0 = s_r0[a];
-                const int npass = (cnt + 8 * GMAX - 1) / (8 * GMAX);
-                const int vrows = min(ROWS, p.N - n0);
-                // the item's scales: its rows x all blocks, one contiguous range (a multiple of 16 bytes)
-                if (!mbar_wait_bounded(smem_addr(sfree + sslot), sph, abort_flag, &g_decode_error, 4u)) break;
-                {
-                    const uint32_t sbytes = (uint32_t)(vrows * nbk * ssz);
-                    const uint8_t* ssrc = reinterpret_cast<const uint8_t*>(p.scales) +
-                                          ((int64_t)e * p.N + n0) * nbk * ssz;
+                // scales go out one item ahead: those of this item and of the next
+                while (s_next < i1 && s_next <= item + 1) {
+                    // an item's scales: its rows x all blocks, one contiguous range (a multiple of 16 bytes)
+                    if (!mbar_wait_bounded(smem_addr(sfree + sslot), sph, abort_flag, &g_decode_error, 4u)) {
+                        ok = false;
+                        break;
+                    }
+                    const int se = s_active[sa_];
+                    const int sn0 = sit * ROWS;
+                    const uint32_t sbytes = (uint32_t)(min(ROWS, p.N - sn0) * nbk * ssz);
+                    const uint8_t* ssrc = reinterpret_cast<const uint8_t*>(p.scales) + ((int64_t)se * p.N + sn0) * nbk * ssz;
                     const uint32_t sb = smem_addr(sfull + sslot);
                     mbar_arrive_tx(sb, sbytes);
                     bulk_1d(smem_addr(sslots + sslot * plan.scale_bytes), ssrc, sbytes, sb);
@@ -367,11 +375,16 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
                         sslot = 0;
                         sph ^= 1u;
                     }
+                    if (++sit == nit) {
+                        sit = 0;
+                        ++sa_;
+                    }
+                    ++s_next;
                 }
+                const int e = s_active[a];
+                const int n0 = it * ROWS;
+                const int npass = (s_cnt[a] + 8 * GMAX - 1) / (8 * GMAX);
                 for (int pass = 0; pass < npass && ok; ++pass) {
-                    // activation rows of this pass: their chunk of K, one bulk copy each
-                    const int mc = pass * 8 * GMAX;
-                    const int nx = min(8 * GMAX, cnt - mc);
                     for (int kc = 0; kc < nch; ++kc) {
                         if (!mbar_wait_bounded(smem_addr(empty + slot), ph, abort_flag, &g_decode_error, 1u)) {
                             ok = false;
@@ -380,17 +393,9 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
                         // the slot's previous chunk is consumed: name the chunk it now receives
                         asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_addr(tags + slot)), "r"(ctr)
                                      : "memory");
-                        const int kb = kc * kChunkK;
-                        const uint32_t xbytes = (uint32_t)(min(kChunkK, p.K - kb) * 2);
                         const uint32_t fb = smem_addr(full + slot);
-                        mbar_arrive_tx(fb, (uint32_t)(kBoxBytes * ROWS) + (uint32_t)nx * xbytes);
-                        const uint32_t dst = smem_addr(ring + slot * plan.stage_bytes);
-                        tma_2d(dst, &wmap, kb / 2, e * p.N + n0, fb);
-                        for (int j = 0; j < nx; ++j) {
-                            const int64_t r = r0 + mc + j;
-                            const int tk = table ? t_tok[r - rlo] : (p.row_token ? __ldg(p.row_token + r) : (int)r);
-                            bulk_1d(dst + plan.wbytes + j * kXStride, p.x + (int64_t)tk * p.K + kb, xbytes, fb);
-                        }
+                        mbar_arrive_tx(fb, (uint32_t)(kBoxBytes * ROWS));
+                        tma_2d(smem_addr(ring + slot * plan.stage_bytes), &wmap, kc * (kChunkK / 2), e * p.N + n0, fb);
                         ++ctr;
                         if (++slot == (uint32_t)ns) {
                             slot = 0;
@@ -405,7 +410,22 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
             }
         }
         __syncwarp();
-    } else if (warp == kEpilogueWarp) {
+        return;
+    }
+
+    // consumers and the epilogue warp: stage the routing metadata of the CTA's rows
+    if (table) {
+        for (int64_t r = rlo + threadIdx.x; r < rhi; r += kConsumers * 32)
+            if (threadIdx.x < kConsumers * 32) {
+                const int k = (int)(r - rlo);
+                t_tok[k] = p.row_token ? __ldg(p.row_token + r) : (int)r;
+                t_wt[k] = p.row_weight ? __ldg(p.row_weight + r) : 1.f;
+                t_dst[k] = p.row_dest ? __ldg(p.row_dest + r) : (int)r;
+            }
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"((kConsumers + 1) * 32) : "memory");
+
+    if (warp == kEpilogueWarp) {
         // ================= epilogue: fixed-order K-split sums, weight, bf16, scatter =================
         bool dead = false;
         uint32_t P = 0;                                 // pass counter of the CTA
@@ -463,91 +483,117 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
                 ++a;
             }
         }
-    } else {
-        // ================= consumers =================
-        const int rt = warp % nrt, ks = warp / nrt;     // row tile, K split (chunk counter % nks == ks)
-        const int g = lane >> 2, t = lane & 3;
-        const int ra = rt * 16 + g, rb = ra + 8;        // the two item rows of this lane
-        const uint32_t lane_sel = (uint32_t)lane * 4u;  // lut offset of this lane's copy
-        const bool vec_scales = (FMT == FMT_NF4) ? (nbk % 4 == 0) : (nbk % 8 == 0);
-        const uint32_t kmask = (uint32_t)nks - 1u;      // nks is 4 or 8
-        bool dead = false;   // set when a wait gives up: the warp then only keeps the barrier schedule
-        float acc[GMAX][4];
+        return;
+    }
+
+    // ================= consumers =================
+    const int rt = warp % nrt, ks = warp / nrt;     // row tile, K split (chunk counter % nks == ks)
+    const int g = lane >> 2, t = lane & 3;
+    const int ra = rt * 16 + g, rb = ra + 8;        // the two item rows of this lane
+    const uint32_t lane_sel = (uint32_t)lane * 4u;  // lut offset of this lane's copy
+    const bool vec_scales = (FMT == FMT_NF4) ? (nbk % 4 == 0) : (nbk % 8 == 0);
+    const uint32_t nch_mod = (uint32_t)(nch % nks);
+    bool dead = false;   // set when a wait gives up: the warp then only keeps the barrier schedule
+    float acc[GMAX][4];
 #pragma unroll
-        for (int j = 0; j < GMAX; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-        uint32_t base = 0;                              // chunk counter at the start of the pass
-        uint32_t P = 0;                                 // pass counter of the CTA
-        uint32_t sslot = 0, sph = 0;                    // scale slot; its full-barrier parity
-        int a = (i1 > i0) ? i0 / nit : 0, it = (i1 > i0) ? i0 % nit : 0;
-        for (int item = i0; item < i1; ++item) {
-            const int m = s_cnt[a];
-            const int npass = (m + 8 * GMAX - 1) / (8 * GMAX);
-            // every warp waits for the item's scales (also those that own no chunk of it)
-            if (!dead && !mbar_wait_bounded(smem_addr(sfull + sslot), sph, abort_flag, &g_decode_error, 8u))
-                dead = true;
-            const uint8_t* ss = sslots + sslot * plan.scale_bytes;
-            for (int pass = 0; pass < npass; ++pass, ++P) {
-                const int nvalid = min(8 * GMAX, m - pass * 8 * GMAX);   // routed rows of this pass
-                int kc = (int)(((uint32_t)ks - base) & kmask);
-                uint32_t ctr = base + (uint32_t)kc;
-                uint32_t slot = ctr % (uint32_t)ns, ph = (ctr / (uint32_t)ns) & 1u;
-                for (; kc < nch; kc += nks) {
-                    if (!dead && !wait_tag(tags + slot, ctr, abort_flag, &g_decode_error, 16u)) dead = true;
-                    if (!dead && !mbar_wait_bounded(smem_addr(full + slot), ph, abort_flag, &g_decode_error, 2u))
-                        dead = true;
-                    if (!dead) {
-                        const uint8_t* st = ring + slot * plan.stage_bytes;
-                        const int kb = kc * kChunkK;
-                        if (p.K - kb >= kChunkK) {
-                            if (GMAX == 2 && nvalid > 8)
-                                chunk_mma<FMT, GMAX, (GMAX == 2 ? 2 : 1), true>(st, ss, lut, lane_sel, L, ra, rb, g, t, nbk, kc,
-                                                                                0, plan.wbytes, vec_scales, acc);
-                            else
-                                chunk_mma<FMT, GMAX, 1, true>(st, ss, lut, lane_sel, L, ra, rb, g, t, nbk, kc, 0,
-                                                              plan.wbytes, vec_scales, acc);
-                        } else {
-                            const int nbc = (p.K - kb) / SB;
-                            chunk_mma<FMT, GMAX, GMAX, false>(st, ss, lut, lane_sel, L, ra, rb, g, t, nbk, kc, nbc,
-                                                              plan.wbytes, vec_scales, acc);
-                        }
-                    }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_addr(empty + slot));
-                    ctr += (uint32_t)nks;
-                    slot += (uint32_t)nks;                      // nks <= ns: at most one wrap
-                    if (slot >= (uint32_t)ns) {
-                        slot -= (uint32_t)ns;
-                        ph ^= 1u;
-                    }
+    for (int j = 0; j < GMAX; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+    uint32_t base = 0;                              // chunk counter at the start of the pass
+    uint32_t bmod = 0;                              // base % nks
+    uint32_t P = 0;                                 // pass counter of the CTA
+    uint32_t sslot = 0, sph = 0;                    // scale slot; its full-barrier parity
+    int a = (i1 > i0) ? i0 / nit : 0, it = (i1 > i0) ? i0 % nit : 0;
+    for (int item = i0; item < i1; ++item) {
+        const int m = s_cnt[a];
+        const int64_t r0 = s_r0[a];
+        const int npass = (m + 8 * GMAX - 1) / (8 * GMAX);
+        // every warp waits for the item's scales (also those that own no chunk of it)
+        if (!dead && !mbar_wait_bounded(smem_addr(sfull + sslot), sph, abort_flag, &g_decode_error, 8u))
+            dead = true;
+        const uint8_t* ss = sslots + sslot * plan.scale_bytes;
+        for (int pass = 0; pass < npass; ++pass, ++P) {
+            const int mc = pass * 8 * GMAX;
+            const int nvalid = min(8 * GMAX, m - mc);   // routed rows of this pass
+            // x rows of this lane's routed rows (8j + g of the pass), or null past the pass's end
+            const uint16_t* xr0 = nullptr;
+            const uint16_t* xr1 = nullptr;
+            if (g < nvalid) {
+                const int64_t r = r0 + mc + g;
+                const int tk = table ? t_tok[r - rlo] : (p.row_token ? __ldg(p.row_token + r) : (int)r);
+                xr0 = p.x + (int64_t)tk * p.K;
+            }
+            if (GMAX == 2 && 8 + g < nvalid) {
+                const int64_t r = r0 + mc + 8 + g;
+                const int tk = table ? t_tok[r - rlo] : (p.row_token ? __ldg(p.row_token + r) : (int)r);
+                xr1 = p.x + (int64_t)tk * p.K;
+            }
+            int kc = ks - (int)bmod;
+            if (kc < 0) kc += nks;
+            uint32_t ctr = base + (uint32_t)kc;
+            uint32_t slot = ctr % (uint32_t)ns, ph = (ctr / (uint32_t)ns) & 1u;
+            for (; kc < nch; kc += nks) {
+                // bring this chunk's activations into L1 while the weights are on their way
+                // (lane t of row g: the t-th 128-byte line of the row's 512-byte chunk)
+                if (kc * kChunkK + t * 64 < p.K) {
+                    if (xr0 != nullptr) prefetch_l1(xr0 + kc * kChunkK + t * 64);
+                    if (xr1 != nullptr) prefetch_l1(xr1 + kc * kChunkK + t * 64);
                 }
-                base += (uint32_t)nch;
-                // end of a pass: hand the partial sums to the epilogue warp
-                const uint32_t buf = P & 1u, fph = ((P >> 1) & 1u) ^ 1u;
-                const int bi = (int)buf * kMaxRowTiles + rt;
-                if (!dead && !mbar_wait_bounded(smem_addr(rfree + bi), fph, abort_flag, &g_decode_error, 64u))
+                if (!dead && !wait_tag(tags + slot, ctr, abort_flag, &g_decode_error, 16u)) dead = true;
+                if (!dead && !mbar_wait_bounded(smem_addr(full + slot), ph, abort_flag, &g_decode_error, 2u))
                     dead = true;
                 if (!dead) {
-#pragma unroll
-                    for (int j = 0; j < GMAX; ++j)
-                        *red_slot(lut, (((int)buf * nrt + rt) * nks + ks) * GMAX + j, lane) =
-                            make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+                    const uint8_t* st = ring + slot * plan.stage_bytes;
+                    const int kb = kc * kChunkK;
+                    if (p.K - kb >= kChunkK) {
+                        if (GMAX == 2 && nvalid > 8)
+                            chunk_mma<FMT, GMAX, (GMAX == 2 ? 2 : 1), true>(st, ss, lut, lane_sel, xr0, xr1, ra, rb, t, nbk, kc,
+                                                                            0, vec_scales, acc);
+                        else
+                            chunk_mma<FMT, GMAX, 1, true>(st, ss, lut, lane_sel, xr0, xr1, ra, rb, t, nbk, kc, 0, vec_scales,
+                                                          acc);
+                    } else {
+                        const int nbc = (p.K - kb) / SB;
+                        chunk_mma<FMT, GMAX, GMAX, false>(st, ss, lut, lane_sel, xr0, xr1, ra, rb, t, nbk, kc, nbc, vec_scales,
+                                                          acc);
+                    }
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(rready + bi));
+                if (lane == 0) mbar_arrive(smem_addr(empty + slot));
+                ctr += (uint32_t)nks;
+                slot += (uint32_t)nks;                      // nks <= ns: at most one wrap
+                if (slot >= (uint32_t)ns) {
+                    slot -= (uint32_t)ns;
+                    ph ^= 1u;
+                }
+            }
+            base += (uint32_t)nch;
+            bmod += nch_mod;
+            if (bmod >= (uint32_t)nks) bmod -= (uint32_t)nks;
+            // end of a pass: hand the partial sums to the epilogue warp
+            const uint32_t buf = P & 1u, fph = ((P >> 1) & 1u) ^ 1u;
+            const int bi = (int)buf * kMaxRowTiles + rt;
+            if (!dead && !mbar_wait_bounded(smem_addr(rfree + bi), fph, abort_flag, &g_decode_error, 64u))
+                dead = true;
+            if (!dead) {
 #pragma unroll
-                for (int j = 0; j < GMAX; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+                for (int j = 0; j < GMAX; ++j)
+                    *red_slot(lut, (((int)buf * nrt + rt) * nks + ks) * GMAX + j, lane) =
+                        make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
             }
-            // every warp is done with this item's scales
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(sfree + sslot));
-            if (++sslot == (uint32_t)nsl) {
-                sslot = 0;
-                sph ^= 1u;
-            }
-            if (++it == nit) {
-                it = 0;
-                ++a;
-            }
+            if (lane == 0) mbar_arrive(smem_addr(rready + bi));
+#pragma unroll
+            for (int j = 0; j < GMAX; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+        }
+        // every warp is done with this item's scales
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(sfree + sslot));
+        if (++sslot == (uint32_t)nsl) {
+            sslot = 0;
+            sph ^= 1u;
+        }
+        if (++it == nit) {
+            it = 0;
+            ++a;
         }
     }
 }
@@ -571,21 +617,19 @@ static cudaError_t launch_db(const GroupedArgs& a, cudaStream_t s) {
     const int ssz = (FMT == FMT_NF4) ? 4 : 1;
     Plan plan;
     plan.nch = (a.K + kChunkK - 1) / kChunkK;
-    const int tables = 32 + 16 * a.E + 12 * kMaxTableRows;
+    const int tables = 96 + 16 * a.E + 12 * kMaxTableRows;
     int smem = 0;
     plan.rows = 0;
     for (int rows = 64; rows >= 32 && plan.rows == 0; rows >>= 1) {
-        const int wbytes = rows * kBoxBytes;
-        const int stage_bytes = ((wbytes + 8 * GMAX * kXStride + 1023) / 1024) * 1024;
+        const int stage_bytes = rows * kBoxBytes;       // 8 KB or 4 KB: multiples of 1024
         const int scale_bytes = ((rows * (a.K / SB) * ssz + 127) / 128) * 128;
         const int nks = kConsumers * 16 / rows;          // K-split warps per row tile: the ring holds at least one chunk each
-        for (int nst = 12; nst >= nks; --nst) {
+        for (int nst = 12; nst >= nks && plan.rows == 0; --nst) {
             for (int nsl = 3; nsl >= 2; --nsl) {
                 const int need = 1024 + kLutBytes + nst * stage_bytes + nsl * scale_bytes +
                                  (2 * nst + 2 * nsl + 4 * kMaxRowTiles) * 8 + 4 * ((nst + 1) & ~1) + tables;
                 if (need <= 226 * 1024) {
                     plan.rows = rows;
-                    plan.wbytes = wbytes;
                     plan.stage_bytes = stage_bytes;
                     plan.scale_bytes = scale_bytes;
                     plan.nstages = nst;
@@ -594,7 +638,6 @@ static cudaError_t launch_db(const GroupedArgs& a, cudaStream_t s) {
                     break;
                 }
             }
-            if (plan.rows) break;
         }
     }
     if (plan.rows == 0) return cudaErrorInvalidValue;
