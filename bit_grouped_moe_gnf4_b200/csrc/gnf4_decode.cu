@@ -14,9 +14,10 @@
 // scale slot with a barrier of their own, issued one item ahead.
 //
 // 12 consumer warps: warp (rt, ks) owns row tile rt (16 rows of the item) and
-// every nks-th chunk of the CTA's stream (chunk counter % nks == ks; nks = 3
-// for 64-row items), so each stage is read by ROWS/16 warps and stages are
-// consumed in parallel. Because owners skip the stages of other warps, a ring
+// the K chunks kc with kc % nks == ks (nks = 3 for 64-row items), so each stage
+// is read by ROWS/16 warps and stages are consumed in parallel. Ownership goes
+// by K position only, so the fp32 grouping of a row's sum never depends on the
+// other rows of the call. Because owners skip the stages of other warps, a ring
 // slot carries a tag naming the chunk that was last issued into it; an owner
 // reads the slot's barrier only once the tag shows its chunk, which keeps
 // every parity wait within one phase.
@@ -487,18 +488,16 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
     }
 
     // ================= consumers =================
-    const int rt = warp % nrt, ks = warp / nrt;     // row tile, K split (chunk counter % nks == ks)
+    const int rt = warp % nrt, ks = warp / nrt;     // row tile, K split (chunks kc % nks == ks)
     const int g = lane >> 2, t = lane & 3;
     const int ra = rt * 16 + g, rb = ra + 8;        // the two item rows of this lane
     const uint32_t lane_sel = (uint32_t)lane * 4u;  // lut offset of this lane's copy
     const bool vec_scales = (FMT == FMT_NF4) ? (nbk % 4 == 0) : (nbk % 8 == 0);
-    const uint32_t nch_mod = (uint32_t)(nch % nks);
     bool dead = false;   // set when a wait gives up: the warp then only keeps the barrier schedule
     float acc[GMAX][4];
 #pragma unroll
     for (int j = 0; j < GMAX; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
     uint32_t base = 0;                              // chunk counter at the start of the pass
-    uint32_t bmod = 0;                              // base % nks
     uint32_t P = 0;                                 // pass counter of the CTA
     uint32_t sslot = 0, sph = 0;                    // scale slot; its full-barrier parity
     int a = (i1 > i0) ? i0 / nit : 0, it = (i1 > i0) ? i0 % nit : 0;
@@ -526,8 +525,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
                 const int tk = table ? t_tok[r - rlo] : (p.row_token ? __ldg(p.row_token + r) : (int)r);
                 xr1 = p.x + (int64_t)tk * p.K;
             }
-            int kc = ks - (int)bmod;
-            if (kc < 0) kc += nks;
+            int kc = ks;                                // chunks kc = ks, ks + nks, ...
             uint32_t ctr = base + (uint32_t)kc;
             uint32_t slot = ctr % (uint32_t)ns, ph = (ctr / (uint32_t)ns) & 1u;
             for (; kc < nch; kc += nks) {
@@ -566,8 +564,6 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
                 }
             }
             base += (uint32_t)nch;
-            bmod += nch_mod;
-            if (bmod >= (uint32_t)nks) bmod -= (uint32_t)nks;
             // end of a pass: hand the partial sums to the epilogue warp
             const uint32_t buf = P & 1u, fph = ((P >> 1) & 1u) ^ 1u;
             const int bi = (int)buf * kMaxRowTiles + rt;

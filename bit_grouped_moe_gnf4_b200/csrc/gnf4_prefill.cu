@@ -10,9 +10,9 @@
 // the tiles of every expert in the band, computed on the device from the
 // expert offsets. Roles (19 warps):
 //   warp 0      tensor-memory owner and MMA issuer (one thread)
-//   warp 1      activation loader: TMA tile loads of contiguous rows, or TMA
-//               gather4 loads of the rows named by row_token, both into the
-//               128B-swizzled K-major layout
+//   warp 1      activation loader: TMA tile loads of contiguous rows, or
+//               16-byte cp.async copies (all 32 lanes) of the rows named by
+//               row_token, both into the 128B-swizzled K-major layout
 //   warp 2      packed-weight loader: TMA loads of the tile's 128 rows x 32
 //               bytes per 64 K into a deep ring of its own
 //   warps 3-10  decoders: half a weight row per thread; nibbles -> bf16 by
@@ -127,14 +127,15 @@ __device__ __forceinline__ void tma_tile_2d(uint32_t dst, const CUtensorMap* map
 }
 // four rows (y0..y3) x one box of columns starting at x, written as four consecutive
 // 128-byte rows at dst (the tensor map's box is one row high)
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, int y0, int y1, int y2,
-                                            int y3, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar)
-        : "memory");
+// 16-byte asynchronous copy global -> shared; bytes past src_bytes (0 or 16) are zero-filled
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
+// arrive on the barrier once this thread's earlier cp.async copies have landed
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
@@ -195,7 +196,7 @@ __device__ __forceinline__ Tile tile_at(const GroupedArgs& p, const Sched& s, in
 template <int FMT>
 __global__ void __maxnreg__(96)
 prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xmap,
-                    const __grid_constant__ CUtensorMap gmap, const __grid_constant__ CUtensorMap wmap,
+                    const __grid_constant__ CUtensorMap wmap,
                     const int gather) {
     using namespace pf;
     constexpr int SB = (FMT == FMT_NF4) ? 64 : 32;      // scale block
@@ -257,8 +258,8 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
         }
     } else if (warp == 2 && lane == 0) {
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(bar_afull + 8 * i, 32 * kDecWarps);
-            mbar_init(bar_bfull + 8 * i, 1);
+            mbar_init(bar_afull + 8 * i, kDecWarps);            // one arrival per decoder warp
+            mbar_init(bar_bfull + 8 * i, gather ? 32 : 1);   // gather: one arrival per loader lane
             mbar_init(bar_empty + 8 * i, 1);
         }
         for (int i = 0; i < kWStages; ++i) {
@@ -271,7 +272,12 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    } else if (warp == 0) {
+    }
+    __syncthreads();
+    // a CTA without a tile (no group of the band, or more CTAs than tiles) leaves
+    // before it takes tensor memory
+    if ((int)blockIdx.x >= s_count[1]) return;
+    if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;"
                      ::"r"(smem_addr(tmem_slot)) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -293,6 +299,8 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
                     const uint32_t slot = stage_ctr % kStages, ph = (stage_ctr / kStages) & 1u;
                     if (!mbar_wait_bounded(bar_afull + 8 * slot, ph, abort_flag, err, 1u)) goto mma_done;
                     if (!mbar_wait_bounded(bar_bfull + 8 * slot, ph, abort_flag, err, 2u)) goto mma_done;
+                    // gathered rows were written by cp.async (generic proxy): order them before the MMA reads
+                    if (gather) fence_proxy_async();
                     tc_fence_after();
                     const uint32_t a_addr = sbase + kOffA + slot * kAStageBytes;
                     const uint32_t b_addr = sbase + kOffB + slot * kBStageBytes;
@@ -316,9 +324,11 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
     mma_done:
         __syncwarp();
     } else if (warp == 1) {
-        // ================= activation loader (TMA) =================
-        // contiguous routed rows: one tile load of 128 rows x 64 K; rows named by row_token:
-        // gather4 loads of 4 rows x 64 K. Both land 128B-swizzled, as the MMA reads them.
+        // ================= activation loader =================
+        // contiguous routed rows: one TMA tile load of 128 rows x 64 K. Rows named by
+        // row_token: the warp's 32 lanes copy 16-byte pieces with cp.async (TMA gathers of
+        // 128-byte rows are bound by their request rate). Both land 128B-swizzled, as the
+        // MMA reads them.
         int* s_rows = reinterpret_cast<int*>(smem + kOffRows);
         uint32_t stage_ctr = 0;
         for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
@@ -329,23 +339,28 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
                 for (int row = lane; row < tl.bn; row += 32)
                     s_rows[row] = __ldg(p.row_token + tl.r0 + (row < tl.cnt ? row : 0));
                 __syncwarp();
-            }
-            if (lane == 0) {
                 for (int s = 0; s < nst; ++s, ++stage_ctr) {
                     const uint32_t slot = stage_ctr % kStages, ph = ((stage_ctr / kStages) & 1u) ^ 1u;
                     if (!mbar_wait_bounded(bar_empty + 8 * slot, ph, abort_flag, err, 8u)) goto load_done;
-                    const uint32_t full = bar_bfull + 8 * slot;
                     const uint32_t dst = sbase + kOffB + slot * kBStageBytes;
-                    if (gather) {
-                        mbar_arrive_tx(full, (uint32_t)tl.bn * 128u);
-                        for (int j = 0; j < tl.bn; j += 4)
-                            tma_gather4(dst + j * 128, &gmap, s * kKStage, s_rows[j], s_rows[j + 1], s_rows[j + 2],
-                                        s_rows[j + 3], full);
-                    } else {
-                        // one box of 128 rows (rows past the tile are loaded and never used)
-                        mbar_arrive_tx(full, (uint32_t)kBStageBytes);
-                        tma_tile_2d(dst, &xmap, s * kKStage, (int)tl.r0, full);
+                    const int kk = s * kKStage;
+                    const int kvalid = min(kKStage, p.K - kk);       // 64, or 32 at an MXFP4 tail
+                    for (int q = lane; q < tl.bn * 8; q += 32) {      // piece c of row r: K elements 8c .. 8c+7
+                        const int r = q >> 3, c = q & 7;
+                        const bool in = c * 8 < kvalid;
+                        const uint16_t* src = p.x + (int64_t)s_rows[r] * p.K + kk + (in ? c * 8 : 0);
+                        cp_async16(dst + r * 128 + ((c ^ (r & 7)) << 4), src, in ? 16u : 0u);
                     }
+                    cp_async_arrive(bar_bfull + 8 * slot);
+                }
+            } else if (lane == 0) {
+                for (int s = 0; s < nst; ++s, ++stage_ctr) {
+                    const uint32_t slot = stage_ctr % kStages, ph = ((stage_ctr / kStages) & 1u) ^ 1u;
+                    if (!mbar_wait_bounded(bar_empty + 8 * slot, ph, abort_flag, err, 8u)) goto load_done;
+                    // one box of 128 rows (rows past the tile are loaded and never used)
+                    const uint32_t full = bar_bfull + 8 * slot;
+                    mbar_arrive_tx(full, (uint32_t)kBStageBytes);
+                    tma_tile_2d(sbase + kOffB + slot * kBStageBytes, &xmap, s * kKStage, (int)tl.r0, full);
                 }
             } else {
                 stage_ctr += nst;
@@ -399,7 +414,8 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
                     *reinterpret_cast<uint4*>(arow + ((cc ^ (i & 7)) << 4)) = make_uint4(o[c][0], o[c][1], o[c][2], o[c][3]);
                 }
                 fence_proxy_async();
-                mbar_arrive(bar_afull + 8 * slot);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_afull + 8 * slot);
             }
         }
     dec_done:;
@@ -524,18 +540,6 @@ static cudaError_t launch_pf(const GroupedArgs& a, int64_t T_in, cudaStream_t s)
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     }
-    CUtensorMap gmap;
-    {
-        // activations for gather4: the same tensor, boxes of 64 K x 1 row, 128B swizzle
-        cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)T_in};
-        cuuint64_t strides[1] = {(cuuint64_t)a.K * 2};
-        cuuint32_t box[2] = {64, 1};
-        cuuint32_t estr[2] = {1, 1};
-        CUresult r = enc(&gmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.x), dims, strides, box,
-                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    }
     {
         // packed weights: bytes [E*N, K/2], boxes of 32 bytes x 128 rows, no swizzle
         cuuint64_t dims[2] = {(cuuint64_t)(a.K / 2), (cuuint64_t)a.E * (cuuint64_t)a.N};
@@ -547,8 +551,13 @@ static cudaError_t launch_pf(const GroupedArgs& a, int64_t T_in, cudaStream_t s)
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     }
-    const int grid = device_sm_count();
-    prefill_band_kernel<FMT><<<grid, pf::kThreads, pf::kSmemBytes, s>>>(a, xmap, gmap, wmap, gather);
+    // no more CTAs than the R routed rows can form tiles: groups of more than m_lo - 1
+    // rows number at most R / m_lo, and their token tiles at most R / kBNMax + R / m_lo
+    const int64_t mlo = a.m_lo > 1 ? a.m_lo : 1;
+    const int64_t max_tiles = (int64_t)((a.N + pf::kBM - 1) / pf::kBM) * (a.R / pf::kBNMax + a.R / mlo + 1);
+    int grid = device_sm_count();
+    if (max_tiles < grid) grid = (int)max_tiles;
+    prefill_band_kernel<FMT><<<grid, pf::kThreads, pf::kSmemBytes, s>>>(a, xmap, wmap, gather);
     return cudaGetLastError();
 }
 
