@@ -182,8 +182,11 @@ def oracle_sample(wl, calls, budget_s=15.0, seed=0):
             Wh[e], Sh[e] = q(G.expert_weights(seed, int(e), proj.N, proj.K))
         if proj.name == "gate_up":
             x = synth.activations_bf16(seed, T, proj.K)
+            tok = b.row_token
+            if wl.gate_up_input == "a_cat":
+                x, tok = x[b.row_token], None          # rows already in routed order
             t1 = time.perf_counter()
-            O.grouped_gemm(wl.fmt, x, Wh, Sh, b.offsets, b.row_token, None, None, T_out=b.R)
+            O.grouped_gemm(wl.fmt, x, Wh, Sh, b.offsets, tok, None, None, T_out=b.R)
         else:
             x = synth.activations_bf16(seed, b.R, proj.K, tag="x_down")
             t1 = time.perf_counter()
@@ -293,6 +296,8 @@ def run_ours(args, wl):
         if proj.name == "gate_up":
             xb = synth.activations_bf16(args.seed, T, proj.K)
             tok, wt, dst, T_out = b.row_token, None, None, b.R
+            if wl.gate_up_input == "a_cat":
+                xb, tok = np.ascontiguousarray(xb[b.row_token]), None   # rows already in routed order
         else:
             xb = synth.activations_bf16(args.seed, b.R, proj.K, tag="x_down")
             tok, wt, dst, T_out = None, b.row_weight, b.row_dest, T * b.k

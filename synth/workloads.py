@@ -26,6 +26,10 @@ class Workload:
     T: Tuple[int, ...]
     projections: Tuple[Projection, ...]
     routing: str = "softmax"       # "softmax" | "zipf"
+    # how gate_up receives its activations: "gather" = x [T, K] plus row_token (the
+    # kernel reads the token rows itself); "a_cat" = the rows already in routed order,
+    # [R, K] (the pages' gemm_4bit_grouped(a_cat, ...) interface, sorted outside)
+    gate_up_input: str = "gather"
     note: str = field(default="", compare=False)
 
 
@@ -43,7 +47,8 @@ WORKLOADS = {
         "qwen3_prefill_nf4", "nf4", E=128, top_k=(8,), T=(4096,),
         projections=(Projection("gate_up", K=2048, N=1536),
                      Projection("down", K=768, N=2048)),
-        note="Qwen3-30B-A3B-shaped prefill: hidden 2048, moe_intermediate 768"),
+        gate_up_input="a_cat",
+        note="Qwen3-30B-A3B-shaped prefill: hidden 2048, moe_intermediate 768; gate_up reads a_cat [R, K]"),
     "gptoss_mxfp4": Workload(
         "gptoss_mxfp4", "mxfp4", E=128, top_k=(4,), T=(1, 8, 64),
         projections=(Projection("gate_up", K=2880, N=5760),
