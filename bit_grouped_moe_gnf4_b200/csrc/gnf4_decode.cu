@@ -5,7 +5,7 @@
 // take the GEMV path).
 //
 // One persistent CTA per SM takes a contiguous run of work items; an item is
-// (active expert, ROWS = 64 weight rows; 32 when K is very large). A producer
+// (active expert, ROWS = 48 weight rows; fewer when K is very large). A producer
 // thread streams each item's packed rows, one K chunk of 256 at a time, into a
 // ring of 8 KB shared-memory stages with one 2-D TMA load per chunk (a box of
 // 128 bytes x ROWS rows, 128B-swizzled); the stage holds nothing else, so the
@@ -14,8 +14,9 @@
 // scale slot with a barrier of their own, issued one item ahead.
 //
 // 12 consumer warps: warp (rt, ks) owns row tile rt (16 rows of the item) and
-// the K chunks kc with kc % nks == ks (nks = 3 for 64-row items), so each stage
-// is read by ROWS/16 warps and stages are consumed in parallel. Ownership goes
+// the K chunks kc with kc % nks == ks (nks = 4 for 48-row items, so K chunks
+// of any multiple of 1024 split evenly), so each stage is read by ROWS/16 warps
+// and stages are consumed in parallel. Ownership goes
 // by K position only, so the fp32 grouping of a row's sum never depends on the
 // other rows of the call. Because owners skip the stages of other warps, a ring
 // slot carries a tag naming the chunk that was last issued into it; an owner
@@ -27,7 +28,9 @@
 // (prefetched into L1 before the wait for the chunk's weights). Nibbles are
 // decoded by a table in shared memory that maps each packed byte to its two
 // bf16 values (replicated per lane, so 32 lookups never conflict; a byte
-// permute forms the address). The products run on warp-level bf16 MMAs with 16
+// permute forms the address); for MXFP4, whose register decode is short, one
+// of the lane's two rows goes through byte permutes on register tables instead,
+// to spread the work over the shared-memory and ALU pipes. The products run on warp-level bf16 MMAs with 16
 // weight rows as the M side and up to 8 routed rows per MMA as the N side.
 // Every MMA chain covers exactly one scale block (64 K for NF4, 32 K for
 // MXFP4), so the block sum leaves the tensor core in fp32 and is scaled and
@@ -68,10 +71,10 @@ constexpr int kChunkK = 256;                       // K per stage: 128 packed by
 constexpr int kBoxBytes = 128;
 constexpr int kLutBytes = 256 * 256;               // byte value b, lane l -> offset b*256 + l*4
 constexpr int kMaxTableRows = 1024;                // routed rows whose metadata fits the CTA's table
-constexpr int kMaxRowTiles = 4;                    // ROWS / 16 for ROWS = 64
+constexpr int kMaxRowTiles = 4;                    // ROWS / 16 is at most 3
 
 struct Plan {
-    int rows;         // weight rows per item (64 or 32)
+    int rows;         // weight rows per item (48, 32 or 16)
     int nch;          // stages per item pass
     int stage_bytes;  // rows x 128 bytes (a multiple of 1024)
     int scale_bytes;  // slot for one item's scales (rows x all blocks), rounded to 128
@@ -130,7 +133,7 @@ __device__ __forceinline__ float4* red_slot(uint8_t* lut, int u, int lane) {
 // (only the first nbc when the chunk is the ragged end of K).
 template <int FMT, int GMAX, int NG, bool FULL>
 __device__ __forceinline__ void chunk_mma(const uint8_t* __restrict__ st, const uint8_t* __restrict__ ss,
-                                          const uint8_t* __restrict__ lut, uint32_t lane_sel,
+                                          const uint8_t* __restrict__ lut, uint32_t lane_sel, const LutPlanes& L,
                                           const uint16_t* xr0, const uint16_t* xr1, int ra, int rb, int t, int nbk,
                                           int kc, int nbc, bool vec_scales, float (&acc)[GMAX][4]) {
     constexpr int SB = (FMT == FMT_NF4) ? 64 : 32;   // K elements per scale block
@@ -192,13 +195,23 @@ __device__ __forceinline__ void chunk_mma(const uint8_t* __restrict__ st, const 
                 w0[0] = *reinterpret_cast<const uint32_t*>(rp0);
                 w1[0] = *reinterpret_cast<const uint32_t*>(rp1);
             }
-            // both rows by the shared-memory table
+            // row ra by the shared-memory table; row rb by the table too (NF4) or by
+            // byte permutes on register tables (MXFP4)
             uint32_t d0[BPL], d1[BPL];
 #pragma unroll
             for (int j = 0; j < BPL; ++j) {
                 const uint32_t sel = 0x5504u | ((uint32_t)(j & 3) << 4);
                 d0[j] = *reinterpret_cast<const uint32_t*>(lut + prmt(w0[j >> 2], lane_sel, sel));
-                d1[j] = *reinterpret_cast<const uint32_t*>(lut + prmt(w1[j >> 2], lane_sel, sel));
+                if constexpr (FMT == FMT_NF4)
+                    d1[j] = *reinterpret_cast<const uint32_t*>(lut + prmt(w1[j >> 2], lane_sel, sel));
+            }
+            if constexpr (FMT == FMT_MXFP4) {
+#pragma unroll
+                for (int q = 0; q < BPL / 4; ++q) {
+                    uint32_t o4[4];
+                    decode_word<FMT>(w1[q], L, o4);
+                    d1[4 * q] = o4[0]; d1[4 * q + 1] = o4[1]; d1[4 * q + 2] = o4[2]; d1[4 * q + 3] = o4[3];
+                }
             }
 #pragma unroll
             for (int j = 0; j < NG; ++j) {
@@ -274,15 +287,6 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
     uint64_t* rready = bars + 2 * ns + 2 * nsl;                   // [buffer * kMaxRowTiles + rt]
     uint64_t* rfree = rready + 2 * kMaxRowTiles;
 
-    // byte -> bf16x2 table, one copy per lane: 8 sixteen-byte pieces per byte value
-    {
-        const LutPlanes L = p.lut;
-        for (int i = threadIdx.x; i < 256 * 8; i += kThreads) {
-            const int b = i >> 3, q = i & 7;
-            const uint32_t v = byte_bf16x2<FMT>((uint32_t)b, L);
-            *reinterpret_cast<uint4*>(lut + b * 256 + q * 16) = make_uint4(v, v, v, v);
-        }
-    }
     if (warp == kProducerWarp && lane == 0) {
         for (int i = 0; i < ns; ++i) {
             mbar_init(smem_addr(full + i), 1);       // producer + tx bytes
@@ -414,7 +418,17 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
         return;
     }
 
-    // consumers and the epilogue warp: stage the routing metadata of the CTA's rows
+    // consumers and the epilogue warp, while the producer's first copies are in flight:
+    // the byte -> bf16x2 table (one copy per lane: 8 sixteen-byte pieces per byte value)
+    // and the routing metadata of the CTA's rows
+    if (threadIdx.x < kConsumers * 32) {
+        const LutPlanes Lt = p.lut;
+        for (int i = threadIdx.x; i < 256 * 8; i += kConsumers * 32) {
+            const int b = i >> 3, q = i & 7;
+            const uint32_t v = byte_bf16x2<FMT>((uint32_t)b, Lt);
+            *reinterpret_cast<uint4*>(lut + b * 256 + q * 16) = make_uint4(v, v, v, v);
+        }
+    }
     if (table) {
         for (int64_t r = rlo + threadIdx.x; r < rhi; r += kConsumers * 32)
             if (threadIdx.x < kConsumers * 32) {
@@ -492,6 +506,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
     const int g = lane >> 2, t = lane & 3;
     const int ra = rt * 16 + g, rb = ra + 8;        // the two item rows of this lane
     const uint32_t lane_sel = (uint32_t)lane * 4u;  // lut offset of this lane's copy
+    const LutPlanes L = p.lut;                      // register tables for the permute decode
     const bool vec_scales = (FMT == FMT_NF4) ? (nbk % 4 == 0) : (nbk % 8 == 0);
     bool dead = false;   // set when a wait gives up: the warp then only keeps the barrier schedule
     float acc[GMAX][4];
@@ -543,14 +558,14 @@ decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_consta
                     const int kb = kc * kChunkK;
                     if (p.K - kb >= kChunkK) {
                         if (GMAX == 2 && nvalid > 8)
-                            chunk_mma<FMT, GMAX, (GMAX == 2 ? 2 : 1), true>(st, ss, lut, lane_sel, xr0, xr1, ra, rb, t, nbk, kc,
+                            chunk_mma<FMT, GMAX, (GMAX == 2 ? 2 : 1), true>(st, ss, lut, lane_sel, L, xr0, xr1, ra, rb, t, nbk, kc,
                                                                             0, vec_scales, acc);
                         else
-                            chunk_mma<FMT, GMAX, 1, true>(st, ss, lut, lane_sel, xr0, xr1, ra, rb, t, nbk, kc, 0, vec_scales,
+                            chunk_mma<FMT, GMAX, 1, true>(st, ss, lut, lane_sel, L, xr0, xr1, ra, rb, t, nbk, kc, 0, vec_scales,
                                                           acc);
                     } else {
                         const int nbc = (p.K - kb) / SB;
-                        chunk_mma<FMT, GMAX, GMAX, false>(st, ss, lut, lane_sel, xr0, xr1, ra, rb, t, nbk, kc, nbc, vec_scales,
+                        chunk_mma<FMT, GMAX, GMAX, false>(st, ss, lut, lane_sel, L, xr0, xr1, ra, rb, t, nbk, kc, nbc, vec_scales,
                                                           acc);
                     }
                 }
@@ -616,8 +631,8 @@ static cudaError_t launch_db(const GroupedArgs& a, cudaStream_t s) {
     const int tables = 96 + 16 * a.E + 12 * kMaxTableRows;
     int smem = 0;
     plan.rows = 0;
-    for (int rows = 64; rows >= 32 && plan.rows == 0; rows >>= 1) {
-        const int stage_bytes = rows * kBoxBytes;       // 8 KB or 4 KB: multiples of 1024
+    for (int rows = 48; rows >= 16 && plan.rows == 0; rows -= 16) {
+        const int stage_bytes = rows * kBoxBytes;       // 6, 4 or 2 KB: multiples of 1024
         const int scale_bytes = ((rows * (a.K / SB) * ssz + 127) / 128) * 128;
         const int nks = kConsumers * 16 / rows;          // K-split warps per row tile: the ring holds at least one chunk each
         for (int nst = 12; nst >= nks && plan.rows == 0; --nst) {
