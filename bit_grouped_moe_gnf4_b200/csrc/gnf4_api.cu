@@ -14,6 +14,10 @@ namespace gnf4 {
 // Groups with more than this many routed rows go to the prefill (tensor-core)
 // band; the rest to the decode band.
 constexpr int kDecodeMaxRows = 64;
+// at most this many routed rows in the whole call: every group runs in the decode band
+// (at most one group can exceed kDecodeMaxRows, and a second launch costs more than
+// the decode band's extra passes over that group)
+constexpr int64_t kDecodeOnlyRows = 2 * kDecodeMaxRows;
 
 static thread_local char g_err[512] = "";
 
@@ -188,6 +192,7 @@ static gnf4_status grouped(int fmt, const void* x, const uint8_t* W, const void*
 
     // band split by rows per group; decided on the device from the offsets
     int split = kDecodeMaxRows;
+    if (R <= kDecodeOnlyRows) split = INT_MAX;
     if (flags & GNF4_FORCE_DECODE) split = INT_MAX;
     if (flags & GNF4_FORCE_PREFILL) split = 0;
 #ifndef GNF4_HAVE_PREFILL
@@ -274,7 +279,7 @@ int gnf4_grouped_gemm_launches(int64_t R, int flags) {
 #ifdef GNF4_HAVE_PREFILL
     if (flags & GNF4_FORCE_DECODE) return n + 1;
     if (flags & GNF4_FORCE_PREFILL) return n + 1;
-    return n + 1 + (R > kDecodeMaxRows ? 1 : 0);
+    return n + 1 + (R > kDecodeOnlyRows ? 1 : 0);
 #else
     return n + 1;
 #endif

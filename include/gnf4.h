@@ -110,6 +110,10 @@ gnf4_status gnf4_quantize_mxfp4(const float* w, int64_t rows, int64_t K,
  * Offsets are 64-bit everywhere inside, so stacks past 2^31 bytes are addressed
  * correctly (the int64-offset rule under "Supported scope" / "Limitations").
  * flags: 0, or GNF4_CHECK / GNF4_FORCE_DECODE / GNF4_FORCE_PREFILL (above).
+ * Bands: groups of at most 64 rows run in the decode band, larger groups in the
+ * prefill band (tensor cores); a call with R <= 128 runs every group in the
+ * decode band (one launch). Results are deterministic for a given call; a row
+ * computed in different bands may differ in the last bits (fp32 summation order).
  * Results are deterministic: the same inputs give the same bits on every call.
  */
 gnf4_status gnf4_grouped_gemm_nf4(const void* x, const uint8_t* W, const float* absmax,

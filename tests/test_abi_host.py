@@ -41,6 +41,10 @@ def test_version_and_launch_count():
     assert lib.gnf4_grouped_gemm_launches(0, 0) == 0
     assert lib.gnf4_grouped_gemm_launches(1, 0) == 1
     assert lib.gnf4_grouped_gemm_launches(1, _lib.GNF4_CHECK) == 2
+    # calls of at most 128 routed rows run every group in the decode band: one launch
+    assert lib.gnf4_grouped_gemm_launches(128, 0) == 1
+    assert lib.gnf4_grouped_gemm_launches(129, 0) == 2
+    assert lib.gnf4_grouped_gemm_launches(129, _lib.GNF4_FORCE_DECODE) == 1
 
 
 FAKE = 0x7f0000001000          # 16-byte aligned, never dereferenced: validation fails first
