@@ -8,8 +8,7 @@
 // Tile = 128 weight rows (the MMA's M side, one tensor-memory lane each) x up
 // to 128 routed rows of one expert (the N side), all of K. Persistent CTAs walk
 // the tiles of every expert in the band, computed on the device from the
-// expert offsets. Roles (15 warps: at most four per SM sub-partition, so 128
-// registers a thread):
+// expert offsets. Roles (23 warps, 80 registers a thread):
 //   warp 0      tensor-memory owner and MMA issuer (one thread)
 //   warp 1      activation loader: TMA tile loads of contiguous rows, or
 //               16-byte cp.async copies (all 32 lanes) of the rows named by
@@ -19,11 +18,12 @@
 //   warps 3-6   decoders: one weight row per thread; nibbles -> bf16 by byte
 //               permutes, written to shared memory in the 128B-swizzled
 //               K-major layout the MMA reads
-//   warps 7-14  rescale epilogue: per scale block, read the block's fp32 sums
-//               from tensor memory (two loads in flight per wait), multiply by
-//               the block scale (fetched eight blocks ahead) and add into fp32
-//               running sums held in registers; at the end of a tile, weight,
-//               round to bf16 and store (scatter) the outputs
+//   warps 7-22  rescale epilogue, four warps per tensor-memory lane quadrant, 32
+//               of the tile's columns each: per scale block, read the block's
+//               fp32 sums from tensor memory, multiply by the block scale
+//               (fetched four blocks ahead)
+//               and add into fp32 running sums held in registers; at the end of
+//               a tile, weight, round to bf16 and store (scatter) the outputs
 // The MMA chain of each scale block (64 K for NF4, 32 K for MXFP4) goes to
 // one of four tensor-memory buffers, so the scale is applied in fp32 outside
 // the MMA while the tensor core fills the next buffers.
@@ -46,7 +46,7 @@ __device__ unsigned g_prefill_error;
 
 namespace pf {
 
-constexpr int kThreads = 15 * 32;  // see the role list above
+constexpr int kThreads = 23 * 32;  // see the role list above
 constexpr int kBM = 128;             // weight rows per tile
 constexpr int kBNMax = 128;          // routed rows per tile (MMA N)
 constexpr int kStages = 4;           // A (decoded weights) + B (activations) stages
@@ -59,8 +59,9 @@ constexpr int kWStageBytes = kBM * 32;
 constexpr int kMaxExperts = 2048;
 constexpr int kDecWarp0 = 3;         // decoders: warps 3-6
 constexpr int kDecWarps = 4;
-constexpr int kEpiWarp0 = 7;         // epilogue: warps 7-14
-constexpr int kScaleAhead = 8;       // block scales held ahead in epilogue registers
+constexpr int kEpiWarp0 = 7;         // epilogue: warps 7-22
+constexpr int kEpiWarps = 16;
+constexpr int kScaleAhead = 4;       // block scales held ahead in epilogue registers
 
 // shared memory map (offsets from a 1024-aligned base)
 constexpr int kOffA = 0;
@@ -196,7 +197,7 @@ __device__ __forceinline__ Tile tile_at(const GroupedArgs& p, const Sched& s, in
 }  // namespace pf
 
 template <int FMT>
-__global__ void __maxnreg__(128)
+__global__ void __maxnreg__(80)
 prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xmap,
                     const __grid_constant__ CUtensorMap wmap,
                     const int gather) {
@@ -270,7 +271,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
         }
         for (int i = 0; i < kAccBufs; ++i) {
             mbar_init(bar_accfull + 8 * i, 1);
-            mbar_init(bar_accempty + 8 * i, 8);
+            mbar_init(bar_accempty + 8 * i, kEpiWarps);
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -403,16 +404,22 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
                 const uint4 c1 = *reinterpret_cast<const uint4*>(wrow + 16);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_wempty + 8 * wslot);
-                const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                uint32_t o[8][4];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) decode_word<FMT>(words[c], L, o[c]);
                 const uint32_t slot = stage_ctr % kStages, ph = ((stage_ctr / kStages) & 1u) ^ 1u;
-                if (!mbar_wait_bounded(bar_empty + 8 * slot, ph, abort_flag, err, 64u)) goto dec_done;
                 uint8_t* arow = smem + kOffA + slot * kAStageBytes + i * 128;
 #pragma unroll
-                for (int c = 0; c < 8; ++c)            // 16-byte chunk c: K elements 8c .. 8c+7
-                    *reinterpret_cast<uint4*>(arow + ((c ^ (i & 7)) << 4)) = make_uint4(o[c][0], o[c][1], o[c][2], o[c][3]);
+                for (int hh = 0; hh < 2; ++hh) {       // the row in two halves of 32 K (fewer live registers)
+                    const uint4 cw = hh == 0 ? c0 : c1;
+                    const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+                    uint32_t o[4][4];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) decode_word<FMT>(words[c], L, o[c]);
+                    if (hh == 0 && !mbar_wait_bounded(bar_empty + 8 * slot, ph, abort_flag, err, 64u)) goto dec_done;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {       // 16-byte chunk cc: K elements 8cc .. 8cc+7
+                        const int cc = 4 * hh + c;
+                        *reinterpret_cast<uint4*>(arow + ((cc ^ (i & 7)) << 4)) = make_uint4(o[c][0], o[c][1], o[c][2], o[c][3]);
+                    }
+                }
                 fence_proxy_async();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_afull + 8 * slot);
@@ -422,11 +429,11 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
     } else if (warp >= kEpiWarp0) {
         // ================= rescale epilogue =================
         const int q4 = warp & 3;                      // tensor-memory lane quadrant
-        const int half = (warp - kEpiWarp0) >> 2;     // which 16-column chunks: half, half+2, ...
+        const int cq = (warp - kEpiWarp0) >> 2;       // its 16-column chunks: cq and cq + 4
         const int i = q4 * 32 + lane;                 // tile row = tensor-memory lane
         const int nsbk = p.K / SB;                    // scale blocks per row
         uint32_t acc_ctr = 0;
-        float acc[kBNMax / 32][16];
+        float acc[2][16];
         for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
             const Tile tl = tile_at(p, sch, t, nnt);
             const int n = tl.n0 + i;
@@ -434,7 +441,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
             const int64_t srow = ((int64_t)tl.e * p.N + (valid ? n : 0)) * nsbk;
             const int nck = tl.bn >> 4;
 #pragma unroll
-            for (int j = 0; j < kBNMax / 32; ++j)
+            for (int j = 0; j < 2; ++j)
 #pragma unroll
                 for (int c = 0; c < 16; ++c) acc[j][c] = 0.f;
             float sring[kScaleAhead];                 // scales of blocks b .. b+kScaleAhead-1
@@ -453,20 +460,15 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
                         tc_fence_after();
                         const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16) + buf * kBNMax;
 #pragma unroll
-                        for (int j = 0; j < kBNMax / 32; j += 2) {
-                            // two 16-column chunks per wait (warp-uniform conditions)
-                            const int ca = half + 2 * j, cb = half + 2 * (j + 1);
-                            uint32_t va[16], vb[16];
-                            if (ca < nck) tmem_ld16(taddr + ca * 16, va);
-                            if (cb < nck) tmem_ld16(taddr + cb * 16, vb);
-                            tmem_wait_ld();
-                            if (ca < nck) {
+                        for (int j = 0; j < 2; ++j) {
+                            // 16-column chunk cq + 4j (warp-uniform condition)
+                            const int cc = cq + 4 * j;
+                            if (cc < nck) {
+                                uint32_t v[16];
+                                tmem_ld16(taddr + cc * 16, v);
+                                tmem_wait_ld();
 #pragma unroll
-                                for (int c = 0; c < 16; c += 2) ffma2(acc[j][c], acc[j][c + 1], va[c], va[c + 1], sc);
-                            }
-                            if (cb < nck) {
-#pragma unroll
-                                for (int c = 0; c < 16; c += 2) ffma2(acc[j + 1][c], acc[j + 1][c + 1], vb[c], vb[c + 1], sc);
+                                for (int c = 0; c < 16; c += 2) ffma2(acc[j][c], acc[j][c + 1], v[c], v[c + 1], sc);
                             }
                         }
                         tc_fence_before();
@@ -478,8 +480,8 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
             // outputs of this tile: row n, routed rows r0 .. r0+cnt-1
             if (valid) {
 #pragma unroll
-                for (int j = 0; j < kBNMax / 32; ++j) {
-                    const int c0 = half + 2 * j;
+                for (int j = 0; j < 2; ++j) {
+                    const int c0 = cq + 4 * j;
                     if (c0 < nck) {
 #pragma unroll
                         for (int c = 0; c < 16; ++c) {
