@@ -15,18 +15,21 @@
 //               row_token, both into the 128B-swizzled K-major layout
 //   warp 2      packed-weight loader: TMA loads of the tile's 128 rows x 32
 //               bytes per 64 K into a deep ring of its own
-//   warps 3-6   decoders: one weight row per thread; nibbles -> bf16 by byte
-//               permutes, written to shared memory in the 128B-swizzled
-//               K-major layout the MMA reads
+//   warps 3-6   decoders: one weight row per thread (its tensor-memory lane);
+//               nibbles -> bf16 by byte permutes, stored straight into the MMA's
+//               A operand in tensor memory (tcgen05.st), so the decoded tile
+//               never touches shared memory
 //   warps 7-22  rescale epilogue, four warps per tensor-memory lane quadrant, 32
 //               of the tile's columns each: per scale block, read the block's
 //               fp32 sums from tensor memory, multiply by the block scale
 //               (fetched four blocks ahead)
 //               and add into fp32 running sums held in registers; at the end of
 //               a tile, weight, round to bf16 and store (scatter) the outputs
-// The MMA chain of each scale block (64 K for NF4, 32 K for MXFP4) goes to
-// one of four tensor-memory buffers, so the scale is applied in fp32 outside
-// the MMA while the tensor core fills the next buffers.
+// The MMA (A from tensor memory, B from shared memory) chain of each scale block
+// (64 K for NF4, 32 K for MXFP4) goes to one of three tensor-memory accumulators,
+// so the scale is applied in fp32 outside the MMA while the tensor core fills
+// the next ones. Tensor memory: 3 x 128 accumulator columns + 4 x 32 operand
+// columns = 512.
 //
 // Every wait on a barrier is bounded: after ~2^32 cycles without progress the
 // CTA records an error in g_prefill_error, stops its roles and returns.
@@ -51,9 +54,10 @@ constexpr int kBM = 128;             // weight rows per tile
 constexpr int kBNMax = 128;          // routed rows per tile (MMA N)
 constexpr int kStages = 4;           // A (decoded weights) + B (activations) stages
 constexpr int kWStages = 12;         // packed-weight stages (128 rows x 32 bytes)
-constexpr int kAccBufs = 4;          // tensor-memory block accumulators of kBNMax columns
+constexpr int kAccBufs = 3;          // tensor-memory block accumulators of kBNMax columns
+constexpr int kACol0 = kAccBufs * kBNMax;   // first tensor-memory column of the A operand slots
 constexpr int kKStage = 64;          // K per pipeline stage (one 128-byte swizzle row of bf16)
-constexpr int kAStageBytes = kBM * 128;
+constexpr int kAColsPerStage = kKStage / 2;  // 64 K of bf16 pairs = 32 tensor-memory columns per stage
 constexpr int kBStageBytes = kBNMax * 128;
 constexpr int kWStageBytes = kBM * 32;
 constexpr int kMaxExperts = 2048;
@@ -64,8 +68,7 @@ constexpr int kEpiWarps = 16;
 constexpr int kScaleAhead = 4;       // block scales held ahead in epilogue registers
 
 // shared memory map (offsets from a 1024-aligned base)
-constexpr int kOffA = 0;
-constexpr int kOffB = kOffA + kStages * kAStageBytes;
+constexpr int kOffB = 0;
 constexpr int kOffW = kOffB + kStages * kBStageBytes;
 constexpr int kOffBar = kOffW + kWStages * kWStageBytes;
 constexpr int kNumBars = 3 * kStages + 2 * kWStages + 2 * kAccBufs;
@@ -117,6 +120,24 @@ __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64
         " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n"
         ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
 }
+// D (tensor memory) (+)= A (tensor memory: row i in lane i, K pairs along columns) x B (shared memory)
+__device__ __forceinline__ void mma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n"
+        ::"r"(tmem_d), "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+// 16 consecutive 32-bit columns written for this warp's 32 lanes
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+          "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                  ::"r"(bar) : "memory");
@@ -128,8 +149,6 @@ __device__ __forceinline__ void tma_tile_2d(uint32_t dst, const CUtensorMap* map
         " [%0], [%1, {%2, %3}], [%4];"
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
 }
-// four rows (y0..y3) x one box of columns starting at x, written as four consecutive
-// 128-byte rows at dst (the tensor map's box is one row high)
 // 16-byte asynchronous copy global -> shared; bytes past src_bytes (0 or 16) are zero-filled
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
@@ -305,7 +324,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
                     // gathered rows were written by cp.async (generic proxy): order them before the MMA reads
                     if (gather) fence_proxy_async();
                     tc_fence_after();
-                    const uint32_t a_addr = sbase + kOffA + slot * kAStageBytes;
+                    const uint32_t a_col = tmem + kACol0 + slot * kAColsPerStage;
                     const uint32_t b_addr = sbase + kOffB + slot * kBStageBytes;
                     const int nsb = min(SBPS, (p.K - s * kKStage) / SB);
                     for (int sb = 0; sb < nsb; ++sb, ++acc_ctr) {
@@ -315,7 +334,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
 #pragma unroll
                         for (int q = 0; q < K16PSB; ++q) {
                             const uint32_t koff = (uint32_t)(sb * K16PSB + q) * 32u;
-                            mma_bf16(tmem + buf * kBNMax, desc_sw128(a_addr + koff), desc_sw128(b_addr + koff),
+                            mma_bf16_ts(tmem + buf * kBNMax, a_col + (uint32_t)(sb * K16PSB + q) * 8u, desc_sw128(b_addr + koff),
                                      idesc, q > 0 ? 1u : 0u);
                         }
                         mma_commit(bar_accfull + 8 * buf);
@@ -390,37 +409,44 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
     wload_done:
         __syncwarp();
     } else if (warp >= kDecWarp0 && warp < kDecWarp0 + kDecWarps) {
-        // ================= decoders: one weight row per thread =================
-        const int i = (warp - kDecWarp0) * 32 + lane;      // tile row
+        // ================= decoders: one weight row per thread (its tensor-memory lane) =================
+        const int i = (warp & 3) * 32 + lane;              // tile row = tensor-memory lane (quadrant warp % 4)
+        const uint32_t tlane = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const LutPlanes L = p.lut;                         // decode tables in registers
         uint32_t stage_ctr = 0;
         for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
             for (int s = 0; s < nst; ++s, ++stage_ctr) {
                 // packed bytes of this row for this stage (64 K = 32 bytes), from the weight ring
                 const uint32_t wslot = stage_ctr % kWStages, wph = (stage_ctr / kWStages) & 1u;
-                if (!mbar_wait_bounded(bar_wfull + 8 * wslot, wph, abort_flag, err, 32u)) goto dec_done;
+                // (waits are made warp-uniform: the tensor-memory stores below need the whole warp)
+                if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_wfull + 8 * wslot, wph, abort_flag, err, 32u)))
+                    goto dec_done;
                 const uint8_t* wrow = smem + kOffW + wslot * kWStageBytes + i * 32;
                 const uint4 c0 = *reinterpret_cast<const uint4*>(wrow);
                 const uint4 c1 = *reinterpret_cast<const uint4*>(wrow + 16);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_wempty + 8 * wslot);
                 const uint32_t slot = stage_ctr % kStages, ph = ((stage_ctr / kStages) & 1u) ^ 1u;
-                uint8_t* arow = smem + kOffA + slot * kAStageBytes + i * 128;
+                const uint32_t acol = tlane + kACol0 + slot * kAColsPerStage;
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {       // the row in two halves of 32 K (fewer live registers)
+                for (int hh = 0; hh < 2; ++hh) {       // the row in two halves of 32 K = 16 columns each
                     const uint4 cw = hh == 0 ? c0 : c1;
                     const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
                     uint32_t o[4][4];
 #pragma unroll
                     for (int c = 0; c < 4; ++c) decode_word<FMT>(words[c], L, o[c]);
-                    if (hh == 0 && !mbar_wait_bounded(bar_empty + 8 * slot, ph, abort_flag, err, 64u)) goto dec_done;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {       // 16-byte chunk cc: K elements 8cc .. 8cc+7
-                        const int cc = 4 * hh + c;
-                        *reinterpret_cast<uint4*>(arow + ((cc ^ (i & 7)) << 4)) = make_uint4(o[c][0], o[c][1], o[c][2], o[c][3]);
+                    if (hh == 0) {
+                        // the operand slot is free once the MMAs that read it have completed
+                        if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_empty + 8 * slot, ph, abort_flag, err, 64u)))
+                            goto dec_done;
+                        tc_fence_after();
                     }
+                    const uint32_t v[16] = {o[0][0], o[0][1], o[0][2], o[0][3], o[1][0], o[1][1], o[1][2], o[1][3],
+                                            o[2][0], o[2][1], o[2][2], o[2][3], o[3][0], o[3][1], o[3][2], o[3][3]};
+                    tmem_st16(acol + 16 * hh, v);      // columns: K pairs of this half, in order
                 }
-                fence_proxy_async();
+                tmem_wait_st();
+                tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_afull + 8 * slot);
             }
