@@ -52,7 +52,7 @@ namespace pf {
 constexpr int kThreads = 23 * 32;  // see the role list above
 constexpr int kBM = 128;             // weight rows per tile
 constexpr int kBNMax = 128;          // routed rows per tile (MMA N)
-constexpr int kStages = 4;           // A (decoded weights) + B (activations) stages
+constexpr int kStages = 4;           // pipeline stages: B (activations) in shared memory, A slots in tensor memory
 constexpr int kWStages = 12;         // packed-weight stages (128 rows x 32 bytes)
 constexpr int kAccBufs = 3;          // tensor-memory block accumulators of kBNMax columns
 constexpr int kACol0 = kAccBufs * kBNMax;   // first tensor-memory column of the A operand slots

@@ -156,6 +156,24 @@ def test_qwen3_prefill_sampled():
         torch.cuda.empty_cache()
 
 
+def test_prefill_acat_matches_fused_gather():
+    """The pages' interface passes a_cat (token rows already in routed order); the
+    fused gather reads x[row_token[r]] itself. Same activation bytes, same decode and
+    MMAs: the two must give identical bits, and both match the oracle."""
+    E, T, k, K, N = 16, 512, 8, 2048, 512
+    b = synth.make_routed_batch(2, T, E, k)
+    assert np.diff(b.offsets).max() > 64            # the prefill band takes these groups
+    rows, experts = sample_rows(b.offsets, max_rows=48, max_experts=3, seed=5)
+    Wd, Sd, Wh, Sh = build_stack("nf4", E, N, K, seed=2, oracle_experts=experts, tag="w_acat")
+    x = synth.activations_bf16(2, T, K)
+    x_cat = np.ascontiguousarray(x[b.row_token])
+    fused = run_gemm("nf4", x, Wd, Sd, b.offsets, row_token=b.row_token, T_out=b.R)
+    acat = run_gemm("nf4", x_cat, Wd, Sd, b.offsets, T_out=b.R)
+    assert np.array_equal(fused, acat)               # run_gemm returns the bf16 bits on the host
+    ref = O.grouped_rows_f64("nf4", x, Wh, Sh, b.offsets, b.row_token, None, K, rows)
+    check_rows(acat[rows], ref, "a_cat prefill")
+
+
 @pytest.mark.parametrize("T", [1, 8, 64])
 def test_gptoss_mxfp4(T):
     wl = WORKLOADS["gptoss_mxfp4"]
