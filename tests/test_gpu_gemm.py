@@ -164,7 +164,7 @@ def test_prefill_acat_matches_fused_gather():
     b = synth.make_routed_batch(2, T, E, k)
     assert np.diff(b.offsets).max() > 64            # the prefill band takes these groups
     rows, experts = sample_rows(b.offsets, max_rows=48, max_experts=3, seed=5)
-    Wd, Sd, Wh, Sh = build_stack("nf4", E, N, K, seed=2, oracle_experts=experts, tag="w_acat")
+    Wd, Sd, Wh, Sh = build_stack("nf4", E, N, K, seed=2, oracle_experts=experts)
     x = synth.activations_bf16(2, T, K)
     x_cat = np.ascontiguousarray(x[b.row_token])
     fused = run_gemm("nf4", x, Wd, Sd, b.offsets, row_token=b.row_token, T_out=b.R)
