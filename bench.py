@@ -126,6 +126,28 @@ class ClockSampler:
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
 
 
+# --------------------------------------------------------------------------
+# replicas across ranks (one process per GPU; no collective on the data path)
+# --------------------------------------------------------------------------
+def max_over_ranks(values, device):
+    """The per-rank timings, each replaced by its maximum over all ranks (the job
+    takes as long as its slowest replica). Every rank calls this once, in the same
+    order; with one rank it returns the values unchanged."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def replica_rate(world, work_per_rank, seconds):
+    """Whole-job rate of `world` replicas that each did `work_per_rank` units in
+    `seconds` (the max over ranks): weak scaling, work grows with the ranks."""
+    return world * work_per_rank / seconds
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -389,21 +411,17 @@ def run_ours(args, wl):
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
     # max over ranks
-    ms_step = total_ms / args.steps
-    if world > 1:
-        t = torch.tensor([ms_step, e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, e2e_ms = float(t[0]), float(t[1])
+    ms_step, e2e_ms = max_over_ranks([total_ms / args.steps, e2e_ms], dev)
 
     work_bytes = sum(c["bytes"] for c in prepared)
     work_flop = sum(c["flop"] for c in prepared)
     if prefill:
-        value = world * work_flop / (ms_step * 1e-3) / 1e12
-        e2e_v = world * work_flop / (e2e_ms * 1e-3) / 1e12
+        value = replica_rate(world, work_flop, ms_step * 1e-3) / 1e12
+        e2e_v = replica_rate(world, work_flop, e2e_ms * 1e-3) / 1e12
         unit = "TFLOP/s"
     else:
-        value = world * work_bytes / (ms_step * 1e-3) / 1e9
-        e2e_v = world * work_bytes / (e2e_ms * 1e-3) / 1e9
+        value = replica_rate(world, work_bytes, ms_step * 1e-3) / 1e9
+        e2e_v = replica_rate(world, work_bytes, e2e_ms * 1e-3) / 1e9
         unit = "GB/s"
 
     hbm, tc_burst, tc_sust, src = measured_peaks()
