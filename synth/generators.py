@@ -20,7 +20,7 @@ from typing import Optional
 
 import numpy as np
 
-_TAGS = {"w": 1, "x": 2, "route": 3, "w_down": 4, "x_down": 5, "misc": 9}
+_TAGS = {"w": 1, "x": 2, "route": 3, "w_down": 4, "x_down": 5, "h": 6, "y": 7, "misc": 9}
 
 
 def _rng(*key: int) -> np.random.Generator:
