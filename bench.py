@@ -2,6 +2,7 @@
 """Benchmark of the grouped 4-bit MoE GEMM (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--op gemm|swiglu|combine]
 
 A step is one pass of the hot path over one routed batch: for every token count
 of the workload, the gate_up projection (reads token rows, writes sorted rows)
@@ -15,6 +16,11 @@ for the prefill workload. L2: the timed steps rotate over enough copies of the
 weight stacks that the bytes between two uses of one copy exceed twice the L2
 size. Multi-GPU: one independent replica per rank (the path has no exchange
 step), value = all ranks' work / the slowest rank's time.
+
+``--op swiglu`` / ``--op combine`` time instead the memory-bound kernel on one
+side of the GEMM, at the workload's largest token count: bf16 bytes read and
+written per call over device time (HBM roofline), inputs rotated past L2 or L2
+flushed before each call.
 """
 from __future__ import annotations
 
@@ -36,6 +42,8 @@ import synth  # noqa: E402
 from synth.workloads import WORKLOADS, expert_bytes  # noqa: E402
 
 METRIC = "grouped 4-bit MoE GEMM: packed-weight GB/s (decode), TFLOP/s (prefill)"
+GLUE_OPS = {"swiglu": "MoE SwiGLU over gate_up rows: HBM GB/s (bf16 read + written)",
+            "combine": "MoE top-k combine (fp32 slot-order sum): HBM GB/s (bf16 read + written)"}
 DEFAULT_WORKLOAD = "olmoe_decode_nf4"
 PREFILL_WORKLOADS = {"qwen3_prefill_nf4"}
 
@@ -51,6 +59,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--top-k", type=int, default=None, help="sweep workload: top_k (default first)")
     ap.add_argument("--tokens", type=str, default=None, help="comma list overriding the token counts")
+    ap.add_argument("--op", default="gemm", choices=["gemm"] + list(GLUE_OPS),
+                    help="gemm: the grouped GEMM step (default); swiglu / combine: the glue kernel "
+                         "either side of it, on the workload's largest token count")
     return ap.parse_args()
 
 
@@ -468,9 +479,189 @@ def run_ours(args, wl):
         dist.destroy_process_group()
 
 
+# --------------------------------------------------------------------------
+# the glue kernels either side of the GEMM (SwiGLU, top-k combine)
+# --------------------------------------------------------------------------
+def glue_problem(op, wl, k, T):
+    """(input rows, input width, output rows, output width, algorithmic bytes) of one call."""
+    gu, dn = wl.projections
+    if op == "swiglu":
+        R, I = T * k, gu.N // 2
+        return R, 2 * I, R, I, R * 2 * I * 2 + R * I * 2
+    H = dn.N
+    return T * k, H, T, H, T * k * H * 2 + T * H * 2
+
+
+def glue_oracle(op, x_bits, T, k):
+    from oracle import glue as GL
+    return GL.swiglu_rows(x_bits) if op == "swiglu" else GL.combine_topk(x_bits, T, k)
+
+
+def glue_oracle_rate(op, wl, k, T, seed, budget_s):
+    """Oracle bytes/s on whole tokens of the call, repeated until ~budget_s."""
+    rin, win, rout, wout, nbytes = glue_problem(op, wl, k, T)
+    x = synth.activations_bf16(seed, rin, win, tag="h" if op == "swiglu" else "y")
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    done, t0 = 0, time.perf_counter()
+    while True:
+        glue_oracle(op, x, T, k)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return done * nbytes / dt / 1e9, cores, done, dt
+
+
+def run_glue(args, wl):
+    import torch
+    import torch.distributed as dist
+    import bit_grouped_moe_gnf4_b200 as g
+
+    op = args.op
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    k = args.top_k if args.top_k is not None else wl.top_k[-1]
+    T = max(_tokens(args) or wl.T)
+    rin, win, rout, wout, nbytes = glue_problem(op, wl, k, T)
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        vals = []
+        for i in range(args.warmup + args.steps):
+            v, cores, done, dt = glue_oracle_rate(op, wl, k, T, args.seed, 1.0)
+            if i >= args.warmup:
+                vals.append(v)
+        v = float(np.median(vals))
+        print(json.dumps({
+            "metric": GLUE_OPS[op], "value": v, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": nbytes / (v * 1e9) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64" if op == "swiglu" else "f32",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"{op} of {wl.name}: T={T}, top_k={k}, in [{rin}, {win}] -> out [{rout}, {wout}]"},
+            "cpu_baseline": {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": "per step: whole calls repeated for ~1 s"},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
+        return
+
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
+
+    xb = synth.activations_bf16(args.seed + rank, rin, win, tag="h" if op == "swiglu" else "y")
+    xh = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).pin_memory()
+    outh = torch.empty((rout, wout), dtype=torch.bfloat16).pin_memory()
+    # inputs larger than L2 between two uses of one copy, else an L2 flush between calls
+    ncopies = max(1, min(8, int(np.ceil(2.0 * l2 / nbytes)) + 1))
+    flush = ncopies * nbytes < 2 * l2
+    if flush:
+        ncopies = 1
+    xs = [xh.to(dev) for _ in range(ncopies)]
+    outs = [torch.empty((rout, wout), dtype=torch.bfloat16, device=dev) for _ in range(ncopies)]
+    scratch = torch.empty(int(2 * l2) // 4, dtype=torch.float32, device=dev) if flush else None
+
+    def call(j):
+        # the current stream: inside graph capture that is the capturing stream
+        if op == "swiglu":
+            g.swiglu(xs[j], out=outs[j], stream=torch.cuda.current_stream())
+        else:
+            g.combine_topk(xs[j], T, k, out=outs[j], stream=torch.cuda.current_stream())
+
+    for i in range(args.warmup):
+        call(i % ncopies)
+    torch.cuda.synchronize()
+    g.device_status()
+    graphs = []
+    cap = torch.cuda.Stream()
+    for j in range(ncopies):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=cap, capture_error_mode="thread_local"):
+            call(j)
+        graphs.append(gr)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(2e6))
+    for i in range(args.steps):
+        if flush:
+            scratch.fill_(float(i))
+        evs[i][0].record(stream)
+        graphs[i % ncopies].replay()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    g.device_status()
+    call_ms = np.array([a.elapsed_time(b) for a, b in evs])
+    del graphs
+
+    # end to end: pinned host input in, result back, through the public call
+    e2e_steps = max(3, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(e2e_steps):
+        xs[0].copy_(xh, non_blocking=True)
+        call(0)
+        outh.copy_(outs[0], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    ms, e2e_ms = max_over_ranks([float(call_ms.mean()), e2e_ms], dev)
+    value = replica_rate(world, nbytes, ms * 1e-3) / 1e9
+    hbm, _, _, src = measured_peaks()
+    kernel = "swiglu_kernel" if op == "swiglu" else "combine_kernel"
+    line = {
+        "metric": GLUE_OPS[op], "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32" if op == "combine" else "f32 (bf16 in/out)",
+        "data": "synthetic",
+        "config": {"workload": f"{op} of {wl.name}: T={T}, top_k={k}, in [{rin}, {win}] bf16 -> "
+                               f"out [{rout}, {wout}] bf16",
+                   "algorithmic_bytes_per_step": nbytes,
+                   "l2": (f"L2 flushed ({scratch.numel() * 4 / 1e6:.0f} MB write) before each call" if flush
+                          else f"rotating {ncopies} input copies ({ncopies * nbytes / 1e6:.0f} MB of traffic "
+                               f"per rotation; L2 {l2 / 1e6:.0f} MB)"),
+                   "parallelism": f"replicas x{world}"},
+        "gpu_launches": args.steps,
+        "e2e": {"value": replica_rate(world, nbytes, e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": xh.numel() * 2, "d2h_bytes_per_step": outh.numel() * 2},
+        "roofline": {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                     "frac": nbytes / (ms * 1e-3) / 1e9 / hbm, "peak_source": f"{src} HBM copy",
+                     "traffic": recorded_traffic(kernel, wl.name), "kernel": kernel},
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, done, dt = glue_oracle_rate(op, wl, k, T, args.seed, 10.0)
+        line["cpu_baseline"] = {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                "sample": f"{done} whole calls of the oracle ({dt:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     wl = WORKLOADS[args.workload]
+    if args.op in GLUE_OPS:
+        run_glue(args, wl)
+        return
     if args.impl == "reference":
         run_reference(args, wl)
     else:

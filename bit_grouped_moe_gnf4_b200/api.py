@@ -114,6 +114,47 @@ def grouped_gemm_mxfp4(x, W, scales, expert_offsets, **kw):
     return grouped_gemm("mxfp4", x, W, scales, expert_offsets, **kw)
 
 
+def swiglu(gate_up: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """bf16 ``[R, 2I]`` gate_up rows -> bf16 ``[R, I]``: ``silu(gate) * up`` (include/gnf4.h)."""
+    _need(gate_up, torch.bfloat16, "gate_up")
+    if gate_up.dim() != 2 or gate_up.shape[1] % 2:
+        raise ValueError(f"gate_up must be [R, 2I], got {tuple(gate_up.shape)}")
+    R, I = gate_up.shape[0], gate_up.shape[1] // 2
+    if out is None:
+        out = torch.empty((R, I), dtype=torch.bfloat16, device=gate_up.device)
+    else:
+        _need(out, torch.bfloat16, "out")
+        if tuple(out.shape) != (R, I):
+            raise ValueError(f"out must be [{R}, {I}], got {tuple(out.shape)}")
+    check(lib.gnf4_swiglu(_ptr(gate_up), R, I, _ptr(out), _stream(stream)), "gnf4_swiglu")
+    return out
+
+
+def combine_topk(y: torch.Tensor, T: int, k: int, row_of_slot: Optional[torch.Tensor] = None,
+                 slot_weight: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """bf16 ``[R, N]`` down rows -> bf16 ``[T, N]``: the fp32 slot-order sum over each
+    token's k slots (include/gnf4.h)."""
+    _need(y, torch.bfloat16, "y")
+    if y.dim() != 2:
+        raise ValueError("y must be [R, N]")
+    for name, t, dt in (("row_of_slot", row_of_slot, torch.int32), ("slot_weight", slot_weight, torch.float32)):
+        if t is not None:
+            _need(t, dt, name)
+            if t.numel() != T * k:
+                raise ValueError(f"{name} must hold T*k = {T * k} entries, got {t.numel()}")
+    R, N = y.shape
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.bfloat16, device=y.device)
+    else:
+        _need(out, torch.bfloat16, "out")
+        if tuple(out.shape) != (T, N):
+            raise ValueError(f"out must be [{T}, {N}], got {tuple(out.shape)}")
+    check(lib.gnf4_combine_topk(_ptr(y), R, N, _ptr(row_of_slot), _ptr(slot_weight), T, k, _ptr(out),
+                                _stream(stream)), "gnf4_combine_topk")
+    return out
+
+
 def device_status(stream=None) -> None:
     """Synchronise the stream; raise if a kernel gave up waiting on a barrier."""
     check(lib.gnf4_device_status(_stream(stream)), "gnf4_device_status")

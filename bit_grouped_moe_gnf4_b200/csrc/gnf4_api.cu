@@ -1,5 +1,6 @@
 // The C ABI of include/gnf4.h: argument validation, band selection, launches.
 #include <climits>
+#include <cstdint>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -271,6 +272,39 @@ gnf4_status gnf4_device_status(void* stream) {
         return fail(GNF4_ERR_DEVICE_STATUS, "a kernel gave up waiting on a barrier (decode 0x%x, prefill 0x%x)",
                     d, pr);
     return GNF4_OK;
+}
+
+gnf4_status gnf4_swiglu(const void* gate_up, int64_t R, int64_t I, void* out, void* stream) {
+    if (R < 0 || I < 1) return fail(GNF4_ERR_INVALID_ARG, "sizes must be R >= 0 and I >= 1");
+    if (I % 8) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "I must be a multiple of 8");
+    if (R == 0) return GNF4_OK;               // no work: empty buffers may be NULL
+    if (!gate_up || !out) return fail(GNF4_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned16(gate_up) || !aligned16(out))
+        return fail(GNF4_ERR_MISALIGNED, "gate_up and out must be 16-byte aligned");
+    if (!is_device_ptr(gate_up) || !is_device_ptr(out))
+        return fail(GNF4_ERR_INVALID_ARG, "gate_up and out must be device memory");
+    cudaError_t e = launch_swiglu(gate_up, R, I, out, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GNF4_OK : cuda_fail(e, "swiglu launch");
+}
+
+gnf4_status gnf4_combine_topk(const void* y, int64_t R, int64_t N, const int32_t* row_of_slot,
+                              const float* slot_weight, int64_t T, int64_t k, void* out,
+                              void* stream) {
+    if (R < 0 || N < 1 || T < 0 || k < 1)
+        return fail(GNF4_ERR_INVALID_ARG, "sizes must be R, T >= 0 and N, k >= 1");
+    if (N % 8) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "N must be a multiple of 8");
+    if (k > INT_MAX || T > INT64_MAX / k)
+        return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "k must fit in int32 and T*k in int64");
+    if (T == 0) return GNF4_OK;               // no work: empty buffers may be NULL
+    if (!out || (R > 0 && !y)) return fail(GNF4_ERR_INVALID_ARG, "null pointer argument");
+    if ((y && !aligned16(y)) || !aligned16(out))
+        return fail(GNF4_ERR_MISALIGNED, "y and out must be 16-byte aligned");
+    if ((y && !is_device_ptr(y)) || !is_device_ptr(out) || (row_of_slot && !is_device_ptr(row_of_slot)) ||
+        (slot_weight && !is_device_ptr(slot_weight)))
+        return fail(GNF4_ERR_INVALID_ARG, "every buffer must be device memory of the current device");
+    cudaError_t e = launch_combine_topk(y, R, N, row_of_slot, slot_weight, T, k, out,
+                                        reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GNF4_OK : cuda_fail(e, "combine_topk launch");
 }
 
 int gnf4_grouped_gemm_launches(int64_t R, int flags) {

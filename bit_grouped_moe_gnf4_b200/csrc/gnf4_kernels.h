@@ -25,6 +25,13 @@ cudaError_t launch_prefill_band(int fmt, const GroupedArgs& a, int64_t T_in, cud
 cudaError_t launch_check_routing(const GroupedArgs& a, int64_t T_in, int64_t T_out,
                                  unsigned* status_out, cudaStream_t s);
 
+// SwiGLU over [R, 2I] gate_up rows and the fp32 slot-order top-k combine
+// (argument checks are the caller's; sizes already validated).
+cudaError_t launch_swiglu(const void* h, int64_t R, int64_t I, void* out, cudaStream_t s);
+cudaError_t launch_combine_topk(const void* y, int64_t R, int64_t N, const int32_t* row_of_slot,
+                                const float* slot_weight, int64_t T, int64_t k, void* out,
+                                cudaStream_t s);
+
 int device_sm_count();
 
 // Read and clear the error word a band's kernels set when they give up waiting

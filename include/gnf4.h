@@ -148,6 +148,53 @@ gnf4_status gnf4_grouped_gemm_mxfp4(const void* x, const uint8_t* W, const uint8
 gnf4_status gnf4_device_status(void* stream);
 
 /*
+ * SwiGLU over gate_up rows: the step between the gate_up and down grouped GEMMs
+ * of a SwiGLU MoE layer (the decode glue "swiglu_rows" of the status page "MoE
+ * Software Status & Known Limits", section "grouped-nf4-gemm", "Correctness
+ * contracts"; the SwiGLU architectures of the experts4bit-qlora README, "Scope").
+ *   gate = gate_up[r, j], up = gate_up[r, I + j]          (j < I)
+ *   out[r, j] = bf16_rne( silu(gate) * up ),  silu(g) = g / (1 + exp(-g))
+ * computed in fp32 as (g >= 0 ? g : g e) / (1 + e) * up with e = exp(-|g|) = 2^(-|g| log2 e)
+ * from the hardware base-2 exponential and a fast division by 1 + e in [1, 2] (no overflow
+ * for any finite g; about 2^-17 relative error before rounding).
+ * |out - exact| <= (2^-8 + 2^-16) |exact| + 2^-118: one bf16 rounding plus the fp32 error;
+ * the absolute term covers results that fall below the fp32 normal range.
+ * gate_up device bf16 [R, 2I] (row-major, contiguous), 16-byte aligned
+ * out     device bf16 [R, I], 16-byte aligned; may not overlap gate_up
+ * R >= 0, I % 8 == 0. One kernel launch; R == 0 launches nothing and accepts NULL buffers.
+ * Errors: INVALID_ARG (null/host pointer, R < 0, I < 1), UNSUPPORTED_SHAPE (I % 8),
+ * MISALIGNED.
+ */
+gnf4_status gnf4_swiglu(const void* gate_up, int64_t R, int64_t I, void* out, void* stream);
+
+/*
+ * Top-k combine: the step after the down grouped GEMM, one output row per token
+ * ("combine_rows" / "reduce_partials" of the status page, "Correctness contracts":
+ * the partial reduction is bitwise the slot-order sum, and a token's row has the
+ * same bits whether it is combined alone or inside a larger call).
+ *   src(t, s) = row_of_slot ? row_of_slot[t*k + s] : t*k + s
+ *   w(t, s)   = slot_weight ? slot_weight[t*k + s] : 1
+ *   acc = +0; for s = 0 .. k-1 in order, if 0 <= src(t,s) < R:
+ *       acc = fl32( acc + fl32( w(t,s) * y[src(t,s), n] ) )     (no fused multiply-add)
+ *   out[t, n] = bf16_rne(acc)
+ * With the down GEMM's epilogue applying the routing weight and scattering slot s of
+ * token t to row t*k + s, both optional arrays are NULL (the slot-order sum of
+ * already weighted rows); with expert-sorted down rows, row_of_slot is the row of
+ * each (token, slot) and slot_weight its routing weight. The result is a function
+ * of the token's own k slots only: bitwise reproducible and independent of T.
+ * y           device bf16 [R, N], 16-byte aligned (may be NULL when R == 0: every slot dropped)
+ * row_of_slot device int32 [T*k], or NULL; entries outside [0, R) are dropped slots
+ * slot_weight device fp32 [T*k], or NULL
+ * out         device bf16 [T, N], 16-byte aligned; may not overlap y
+ * R, T >= 0, N % 8 == 0, 1 <= k < 2^31. One kernel launch; T == 0 launches nothing and
+ * accepts NULL buffers.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (N % 8), MISALIGNED.
+ */
+gnf4_status gnf4_combine_topk(const void* y, int64_t R, int64_t N, const int32_t* row_of_slot,
+                              const float* slot_weight, int64_t T, int64_t k, void* out,
+                              void* stream);
+
+/*
  * How many kernels one grouped GEMM call with R routed rows and these flags
  * launches (0 when R == 0; GNF4_CHECK adds one). Host-only, no CUDA call.
  */

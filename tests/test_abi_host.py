@@ -21,10 +21,10 @@ def declared_functions():
     return sorted(set(re.findall(r"\b(gnf4_[a-z0-9_]+)\s*\(", src)))
 
 
-def test_header_declares_the_four_ops():
+def test_header_declares_the_ops():
     names = declared_functions()
     for op in ("gnf4_quantize_nf4", "gnf4_quantize_mxfp4", "gnf4_grouped_gemm_nf4",
-               "gnf4_grouped_gemm_mxfp4"):
+               "gnf4_grouped_gemm_mxfp4", "gnf4_swiglu", "gnf4_combine_topk"):
         assert op in names
 
 
@@ -92,3 +92,27 @@ def test_quantize_argument_errors():
     assert lib.gnf4_quantize_mxfp4(FAKE, 4, 48, FAKE, FAKE, None) == _lib.GNF4_ERR_UNSUPPORTED_SHAPE
     assert lib.gnf4_quantize_mxfp4(FAKE, -1, 64, FAKE, FAKE, None) == _lib.GNF4_ERR_INVALID_ARG
     assert lib.gnf4_quantize_nf4(FAKE + 4, 4, 64, FAKE, FAKE, None) == _lib.GNF4_ERR_MISALIGNED
+
+
+def test_glue_argument_errors():
+    sw = lib.gnf4_swiglu
+    assert sw(None, 4, 64, FAKE, None) == _lib.GNF4_ERR_INVALID_ARG
+    assert sw(FAKE, -1, 64, FAKE, None) == _lib.GNF4_ERR_INVALID_ARG
+    assert sw(FAKE, 4, 0, FAKE, None) == _lib.GNF4_ERR_INVALID_ARG
+    assert sw(FAKE, 4, 60, FAKE, None) == _lib.GNF4_ERR_UNSUPPORTED_SHAPE
+    assert sw(FAKE + 2, 4, 64, FAKE, None) == _lib.GNF4_ERR_MISALIGNED
+    assert sw(FAKE, 4, 64, FAKE + 8, None) == _lib.GNF4_ERR_MISALIGNED
+    cb = lib.gnf4_combine_topk
+    assert cb(None, 8, 64, None, None, 2, 4, FAKE, None) == _lib.GNF4_ERR_INVALID_ARG
+    assert cb(None, 8, 64, None, None, 0, 4, None, None) == _lib.GNF4_OK        # no work
+    assert sw(None, 0, 64, None, None) == _lib.GNF4_OK
+    assert cb(FAKE, 8, 64, None, None, 2, 0, FAKE, None) == _lib.GNF4_ERR_INVALID_ARG
+    assert cb(FAKE, 8, 64, None, None, -1, 4, FAKE, None) == _lib.GNF4_ERR_INVALID_ARG
+    assert cb(FAKE, 8, 60, None, None, 2, 4, FAKE, None) == _lib.GNF4_ERR_UNSUPPORTED_SHAPE
+    assert cb(FAKE, 8, 64, None, None, 2, 1 << 31, FAKE, None) == _lib.GNF4_ERR_UNSUPPORTED_SHAPE
+    assert cb(FAKE + 4, 8, 64, None, None, 2, 4, FAKE, None) == _lib.GNF4_ERR_MISALIGNED
+    # host memory is refused (checked before any launch)
+    buf = (ctypes.c_uint16 * 1024)()
+    addr = (ctypes.addressof(buf) + 15) & ~15
+    assert sw(addr, 1, 8, addr + 64, None) == _lib.GNF4_ERR_INVALID_ARG
+    assert b"device memory" in lib.gnf4_last_error()
