@@ -59,9 +59,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--top-k", type=int, default=None, help="sweep workload: top_k (default first)")
     ap.add_argument("--tokens", type=str, default=None, help="comma list overriding the token counts")
-    ap.add_argument("--op", default="gemm", choices=["gemm"] + list(GLUE_OPS),
-                    help="gemm: the grouped GEMM step (default); swiglu / combine: the glue kernel "
-                         "either side of it, on the workload's largest token count")
+    ap.add_argument("--op", default="gemm", choices=["gemm", "dgrad"] + list(GLUE_OPS),
+                    help="gemm: the grouped GEMM step (default); dgrad: its input gradient, every "
+                         "call of the step; swiglu / combine: the glue kernel either side of it, on "
+                         "the workload's largest token count")
     return ap.parse_args()
 
 
@@ -656,9 +657,231 @@ def run_glue(args, wl):
         dist.destroy_process_group()
 
 
+# --------------------------------------------------------------------------
+# the input gradient of the step's grouped GEMM calls
+# --------------------------------------------------------------------------
+def dgrad_oracle_rate(wl, calls, budget_s, seed):
+    """Oracle rate (bytes/s or flop/s) of the input gradient on whole calls, smallest first."""
+    from oracle import dgrad as D
+    from oracle import gnf4_oracle as O
+    from synth import generators as G
+    q = O.quantize_nf4 if wl.fmt == "nf4" else O.quantize_mxfp4
+    sdiv = 64 if wl.fmt == "nf4" else 32
+    done_b = done_f = secs = 0.0
+    n = 0
+    t_begin = time.perf_counter()
+    for T, proj, b in sorted(calls, key=lambda c: c[0]):
+        Wh = np.zeros((wl.E, proj.N, proj.K // 2), np.uint8)
+        Sh = np.zeros((wl.E, proj.N, proj.K // sdiv), np.float32 if wl.fmt == "nf4" else np.uint8)
+        for e in b.active_experts():
+            Wh[e], Sh[e] = q(G.expert_weights(seed, int(e), proj.N, proj.K))
+        src, wt, gb = dgrad_call_inputs(proj, b, seed)
+        t1 = time.perf_counter()
+        D.dgrad(wl.fmt, gb, Wh, Sh, b.offsets, src, wt)
+        secs += time.perf_counter() - t1
+        done_b += call_bytes(wl.fmt, proj, b)[0]
+        done_f += 2.0 * b.R * proj.N * proj.K
+        n += 1
+        if time.perf_counter() - t_begin > budget_s:
+            break
+    return done_b, done_f, n, secs
+
+
+def dgrad_call_inputs(proj, b, seed):
+    """(row_src, row_weight, gradient bits) of the input gradient of one forward call:
+    down scattered row r to t*k + slot with weight w(r), gate_up wrote row r."""
+    if proj.name == "down":
+        return b.row_dest, b.row_weight, synth.activations_bf16(seed, b.T * b.k, proj.N, tag="y")
+    return None, None, synth.activations_bf16(seed, b.R, proj.N, tag="y")
+
+
+def run_dgrad_bench(args, wl):
+    import torch
+    import torch.distributed as dist
+    import bit_grouped_moe_gnf4_b200 as g
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    prefill = wl.name in PREFILL_WORKLOADS
+    calls, k = workload_calls(wl, args.seed, args.top_k, _tokens(args))
+    unit = "TFLOP/s" if prefill else "GB/s"
+    metric = ("grouped 4-bit MoE GEMM input gradient (grad_out @ dequant(W)): packed-weight GB/s "
+              "(decode), TFLOP/s (prefill)")
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        vals = []
+        for i in range(args.warmup + args.steps):
+            nb, nf, n, dt = dgrad_oracle_rate(wl, calls, 4.0, args.seed)
+            if i >= args.warmup:
+                vals.append(nf / dt / 1e12 if prefill else nb / dt / 1e9)
+        v = float(np.median(vals))
+        print(json.dumps({"metric": metric, "value": v, "unit": unit, "n_gpus": args.gpus,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                          "dtype": "f64", "data": "synthetic", "impl": "reference",
+                          "config": {"workload": "dgrad of " + describe(wl, k)},
+                          "cpu_baseline": {"value": v, "unit": unit, "cores": None, "kind": "oracle",
+                                           "sample": "per step: whole calls, smallest first, ~4 s"},
+                          "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}), flush=True)
+        return
+
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(args.seed + 1000 * rank)
+    stacks, stack_bytes = {}, 0
+    for proj in wl.projections:
+        Wl, Sl = [], []
+        for e in range(wl.E):
+            w = torch.randn((proj.N, proj.K), generator=gen, device=dev, dtype=torch.float32) * 0.02
+            p_, s_ = g.quantize_nf4(w) if wl.fmt == "nf4" else g.quantize_mxfp4(w)
+            Wl.append(p_)
+            Sl.append(s_)
+        stacks[proj.name] = [(torch.stack(Wl), torch.stack(Sl))]
+        stack_bytes += stacks[proj.name][0][0].numel() + stacks[proj.name][0][1].numel() * \
+            stacks[proj.name][0][1].element_size()
+        del Wl, Sl
+    step_bytes = sum(call_bytes(wl.fmt, p_, b)[0] for _, p_, b in calls)
+    ncopies = max(1, min(8, int(np.ceil(2.0 * l2 / max(1, step_bytes))) + 1))
+    free = torch.cuda.mem_get_info(dev)[0]
+    while ncopies > 1 and (ncopies - 1) * stack_bytes > 0.5 * free:
+        ncopies -= 1
+    for proj in wl.projections:
+        W0, S0 = stacks[proj.name][0]
+        for _ in range(ncopies - 1):
+            stacks[proj.name].append((W0.clone(), S0.clone()))
+
+    prepared = []
+    for T, proj, b in calls:
+        src, wt, gb = dgrad_call_inputs(proj, b, args.seed)
+        h = {"g": torch.from_numpy(gb.view(np.int16)).view(torch.bfloat16).pin_memory(),
+             "off": torch.from_numpy(b.offsets).pin_memory(),
+             "src": None if src is None else torch.from_numpy(np.ascontiguousarray(src)).pin_memory(),
+             "wt": None if wt is None else torch.from_numpy(np.ascontiguousarray(wt)).pin_memory()}
+        d = {nm: (None if t is None else t.to(dev)) for nm, t in h.items()}
+        out = torch.empty((b.R, proj.K), dtype=torch.bfloat16, device=dev)
+        outh = torch.empty((b.R, proj.K), dtype=torch.bfloat16).pin_memory()
+        prepared.append(dict(T=T, proj=proj, b=b, h=h, d=d, out=out, outh=outh,
+                             bytes=call_bytes(wl.fmt, proj, b)[0], flop=2.0 * b.R * proj.N * proj.K))
+
+    def one_call(c, copy):
+        W_, S_ = stacks[c["proj"].name][copy]
+        d = c["d"]
+        g.dgrad(wl.fmt, d["g"], W_, S_, d["off"], row_src=d["src"], row_weight=d["wt"], R=c["b"].R,
+                out=c["out"], stream=torch.cuda.current_stream())
+
+    for i in range(args.warmup):
+        for c in prepared:
+            one_call(c, i % ncopies)
+    torch.cuda.synchronize()
+    g.device_status()
+    graphs = {}
+    cap = torch.cuda.Stream()
+    for j, c in enumerate(prepared):
+        for copy in range(ncopies):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=cap, capture_error_mode="thread_local"):
+                one_call(c, copy)
+            graphs[(j, copy)] = gr
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in prepared] for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(2e6))
+    for i in range(args.steps):
+        copy = (args.warmup + i) % ncopies
+        for j in range(len(prepared)):
+            ev[i][j][0].record(stream)
+            graphs[(j, copy)].replay()
+            ev[i][j][1].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    g.device_status()
+    call_ms = np.array([[a.elapsed_time(b_) for (a, b_) in row] for row in ev])
+    del graphs
+
+    e2e_steps = max(3, min(args.steps, 10))
+    h2d = sum(sum(t.numel() * t.element_size() for t in c["h"].values() if t is not None) for c in prepared)
+    d2h = sum(c["outh"].numel() * 2 for c in prepared)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(e2e_steps):
+        for c in prepared:
+            for nm, t in c["h"].items():
+                if t is not None:
+                    c["d"][nm].copy_(t, non_blocking=True)
+            one_call(c, i % ncopies)
+            c["outh"].copy_(c["out"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    ms_step, e2e_ms = max_over_ranks([float(call_ms.sum(axis=1).mean()), e2e_ms], dev)
+    work_b = sum(c["bytes"] for c in prepared)
+    work_f = sum(c["flop"] for c in prepared)
+    work = work_f / 1e12 if prefill else work_b / 1e9
+    hbm, tc_burst, tc_sust, src_ = measured_peaks()
+    achieved = work / (ms_step * 1e-3)
+    if prefill:
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_sust, "unit": unit,
+                "frac": achieved / tc_sust, "peak_source": f"{src_} bf16 sustained (kernel inside a step)"}
+    else:
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": unit, "frac": achieved / hbm,
+                "peak_source": f"{src_} HBM copy"}
+    roof["traffic"] = recorded_traffic("dgrad_kernel", wl.name)
+    roof["kernel"] = "dgrad_kernel"
+    roof["per_call_ms"] = [round(float(x), 5) for x in call_ms.mean(axis=0)]
+    roof["per_call"] = [f"T={c['T']} {c['proj'].name}" for c in prepared]
+    line = {"metric": metric, "value": replica_rate(world, work, ms_step * 1e-3), "unit": unit,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": "dgrad of " + describe(wl, k), "format": wl.fmt,
+                       "algorithmic_bytes_per_step": work_b, "flop_per_step": work_f,
+                       "l2": f"rotating {ncopies} weight-stack copies", "parallelism": f"replicas x{world}"},
+            "gpu_launches": len(prepared) * args.steps,
+            "e2e": {"value": replica_rate(world, work, e2e_ms * 1e-3), "unit": unit,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "roofline": roof, "clocks": clk}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nb, nf, n, dt = dgrad_oracle_rate(wl, calls, 10.0, args.seed)
+        try:
+            from threadpoolctl import threadpool_info
+            cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        except Exception:
+            cores = 1
+        line["cpu_baseline"] = {"value": (nf / dt / 1e12) if prefill else (nb / dt / 1e9), "unit": unit,
+                                "cores": cores, "kind": "oracle",
+                                "sample": f"{n} whole calls of the step, smallest first ({dt:.1f} s of oracle "
+                                          f"dgrad; its input quantization untimed)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     args = parse()
     wl = WORKLOADS[args.workload]
+    if args.op == "dgrad":
+        run_dgrad_bench(args, wl)
+        return
     if args.op in GLUE_OPS:
         run_glue(args, wl)
         return

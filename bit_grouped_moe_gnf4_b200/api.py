@@ -114,6 +114,45 @@ def grouped_gemm_mxfp4(x, W, scales, expert_offsets, **kw):
     return grouped_gemm("mxfp4", x, W, scales, expert_offsets, **kw)
 
 
+def dgrad(fmt: str, grad_out: torch.Tensor, W: torch.Tensor, scales: torch.Tensor,
+          expert_offsets: torch.Tensor, row_src: Optional[torch.Tensor] = None,
+          row_weight: Optional[torch.Tensor] = None, R: Optional[int] = None,
+          out: Optional[torch.Tensor] = None, flags: int = 0, stream=None) -> torch.Tensor:
+    """Input gradient of a grouped GEMM call (include/gnf4.h): bf16 ``[R, K]`` with
+    ``out[r] = w(r) * grad_out[src(r)] @ dequant(W[e(r)])``. ``R`` is taken from
+    ``row_src`` / ``row_weight`` when given, else from ``grad_out`` (rows in routed order)."""
+    if fmt not in ("nf4", "mxfp4"):
+        raise ValueError("fmt must be 'nf4' or 'mxfp4'")
+    _need(grad_out, torch.bfloat16, "grad_out")
+    _need(W, torch.uint8, "W")
+    _need(scales, torch.float32 if fmt == "nf4" else torch.uint8, "scales")
+    _need(expert_offsets, torch.int64, "expert_offsets")
+    for name, t, dt in (("row_src", row_src, torch.int32), ("row_weight", row_weight, torch.float32)):
+        if t is not None:
+            _need(t, dt, name)
+    E, N, K2 = W.shape
+    if grad_out.dim() != 2 or grad_out.shape[1] != N:
+        raise ValueError(f"grad_out must be [T_in, N = {N}], got {tuple(grad_out.shape)}")
+    if R is None:
+        for t in (row_src, row_weight):
+            if t is not None:
+                R = t.numel()
+                break
+    if R is None:
+        R = grad_out.shape[0]
+    K = 2 * K2
+    if out is None:
+        out = torch.empty((R, K), dtype=torch.bfloat16, device=grad_out.device)
+    else:
+        _need(out, torch.bfloat16, "out")
+        if tuple(out.shape) != (R, K):
+            raise ValueError(f"out must be [{R}, {K}], got {tuple(out.shape)}")
+    fn = lib.gnf4_dgrad_nf4 if fmt == "nf4" else lib.gnf4_dgrad_mxfp4
+    check(fn(_ptr(grad_out), _ptr(W), _ptr(scales), _ptr(expert_offsets), _ptr(row_src), _ptr(row_weight),
+             E, N, K, R, grad_out.shape[0], _ptr(out), flags, _stream(stream)), f"gnf4_dgrad_{fmt}")
+    return out
+
+
 def swiglu(gate_up: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """bf16 ``[R, 2I]`` gate_up rows -> bf16 ``[R, I]``: ``silu(gate) * up`` (include/gnf4.h)."""
     _need(gate_up, torch.bfloat16, "gate_up")

@@ -216,6 +216,62 @@ static gnf4_status grouped(int fmt, const void* x, const uint8_t* W, const void*
     return GNF4_OK;
 }
 
+static gnf4_status dgrad(int fmt, const void* grad_out, const uint8_t* W, const void* scales,
+                         const int64_t* offsets, const int32_t* row_src, const float* row_weight,
+                         int64_t E, int64_t N, int64_t K, int64_t R, int64_t T_in, void* out,
+                         int flags, void* stream) {
+    if (E < 1 || N < 1 || K < 1 || R < 0 || T_in < 0)
+        return fail(GNF4_ERR_INVALID_ARG, "sizes must be E,N,K >= 1 and R,T_in >= 0");
+    if (flags & ~GNF4_CHECK) return fail(GNF4_ERR_INVALID_ARG, "only GNF4_CHECK is accepted (flags 0x%x)", flags);
+    if (K % 64) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K must be a multiple of 64");
+    if (N % 16) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "N must be a multiple of 16");
+    if (E > 2048) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "at most 2048 experts");
+    if (K > (int64_t)INT_MAX / 2 || E * N > (int64_t)INT_MAX || T_in > INT_MAX || R > INT_MAX)
+        return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K, E*N, T_in and R must fit in int32");
+    if (!row_src && T_in < R) return fail(GNF4_ERR_INVALID_ARG, "row_src is NULL but T_in < R");
+    if (R == 0) return GNF4_OK;                // no work: empty buffers may be NULL
+    if (!grad_out || !W || !scales || !offsets || !out) return fail(GNF4_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned16(grad_out) || !aligned16(W) || !aligned16(out))
+        return fail(GNF4_ERR_MISALIGNED, "grad_out, W and out must be 16-byte aligned");
+    if (!is_device_ptr(grad_out) || !is_device_ptr(W) || !is_device_ptr(scales) || !is_device_ptr(offsets) ||
+        !is_device_ptr(out) || (row_src && !is_device_ptr(row_src)) || (row_weight && !is_device_ptr(row_weight)))
+        return fail(GNF4_ERR_INVALID_ARG, "every buffer must be device memory of the current device");
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    static const LutPlanes lut_nf4 = make_lut(FMT_NF4);
+    static const LutPlanes lut_mx = make_lut(FMT_MXFP4);
+    if (flags & GNF4_CHECK) {
+        GroupedArgs c;
+        std::memset(&c, 0, sizeof(c));
+        c.offsets = offsets;
+        c.row_token = row_src;
+        c.row_weight = row_weight;
+        c.R = R;
+        c.E = (int)E;
+        unsigned st = 0;
+        cudaError_t e = launch_check_routing(c, T_in, R, &st, s);
+        if (e != cudaSuccess) return cuda_fail(e, "routing check");
+        if (st) return fail(GNF4_ERR_DEVICE_STATUS,
+                            "bad routing metadata (status 0x%x: 1 offsets decrease, 2 offsets[0] != 0 "
+                            "or offsets[E] != R, 4 row_src out of range, 16 non-finite row_weight)", st);
+    }
+    DgradArgs a;
+    a.g = reinterpret_cast<const uint16_t*>(grad_out);
+    a.W = W;
+    a.scales = scales;
+    a.offsets = offsets;
+    a.row_src = row_src;
+    a.row_weight = row_weight;
+    a.out = reinterpret_cast<uint16_t*>(out);
+    a.R = R;
+    a.E = (int)E;
+    a.N = (int)N;
+    a.K = (int)K;
+    a.lut = (fmt == FMT_NF4) ? lut_nf4 : lut_mx;
+    cudaError_t e = launch_dgrad(fmt, a, s);
+    return e == cudaSuccess ? GNF4_OK : cuda_fail(e, "dgrad launch");
+}
+
 }  // namespace gnf4
 
 using namespace gnf4;
@@ -305,6 +361,22 @@ gnf4_status gnf4_combine_topk(const void* y, int64_t R, int64_t N, const int32_t
     cudaError_t e = launch_combine_topk(y, R, N, row_of_slot, slot_weight, T, k, out,
                                         reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GNF4_OK : cuda_fail(e, "combine_topk launch");
+}
+
+gnf4_status gnf4_dgrad_nf4(const void* grad_out, const uint8_t* W, const float* absmax,
+                           const int64_t* expert_offsets, const int32_t* row_src,
+                           const float* row_weight, int64_t E, int64_t N, int64_t K, int64_t R,
+                           int64_t T_in, void* out, int flags, void* stream) {
+    return dgrad(FMT_NF4, grad_out, W, absmax, expert_offsets, row_src, row_weight, E, N, K, R, T_in,
+                 out, flags, stream);
+}
+
+gnf4_status gnf4_dgrad_mxfp4(const void* grad_out, const uint8_t* W, const uint8_t* scales,
+                             const int64_t* expert_offsets, const int32_t* row_src,
+                             const float* row_weight, int64_t E, int64_t N, int64_t K, int64_t R,
+                             int64_t T_in, void* out, int flags, void* stream) {
+    return dgrad(FMT_MXFP4, grad_out, W, scales, expert_offsets, row_src, row_weight, E, N, K, R, T_in,
+                 out, flags, stream);
 }
 
 int gnf4_grouped_gemm_launches(int64_t R, int flags) {

@@ -32,6 +32,25 @@ cudaError_t launch_combine_topk(const void* y, int64_t R, int64_t N, const int32
                                 const float* slot_weight, int64_t T, int64_t k, void* out,
                                 cudaStream_t s);
 
+// Input gradient of the grouped GEMM (one launch): out[r, k] = w(r) * sum_n
+// g[src(r), n] * What[e(r), n, k]; sizes already validated (N % 16, K % 64, E <= 2048).
+struct DgradArgs {
+    const uint16_t* g;          // bf16 [T_in, N]
+    const uint8_t* W;           // [E, N, K/2]
+    const void* scales;         // NF4: f32 [E, N, K/64]; MXFP4: u8 [E, N, K/32]
+    const int64_t* offsets;     // [E+1]
+    const int32_t* row_src;     // [R] or null
+    const float* row_weight;    // [R] or null
+    uint16_t* out;              // bf16 [R, K]
+    int64_t R;
+    int E, N, K;
+    LutPlanes lut;
+};
+cudaError_t launch_dgrad(int fmt, const DgradArgs& a, cudaStream_t s);
+// the launch shape the host picks (exported for the tests of the host logic)
+int dgrad_row_tiles(int64_t R, int E);
+int dgrad_splits(int64_t R, int E, int N, int K, int rt);
+
 int device_sm_count();
 
 // Read and clear the error word a band's kernels set when they give up waiting

@@ -148,6 +148,46 @@ gnf4_status gnf4_grouped_gemm_mxfp4(const void* x, const uint8_t* W, const uint8
 gnf4_status gnf4_device_status(void* stream);
 
 /*
+ * Input gradient of the grouped GEMM on NF4-packed weights, every group in one launch:
+ * the grouped-nf4-gemm README (0.11.0), "Training: the backward is a kernel too (0.7.0)"
+ * (grad_out @ dequant(B), decoded on chip, nothing materialised), and the solution page,
+ * "Supported scope" (dgrad_4bit_grouped). For routed rows r sorted by expert as in the
+ * forward call,
+ *
+ *   out[r, k] = bf16_rne( w(r) * sum_n grad_out[src(r), n] * What[e(r), n, k] )
+ *   src(r) = row_src ? row_src[r] : r      (the forward's row_dest, when it scattered)
+ *   w(r)   = row_weight ? row_weight[r] : 1 (the forward's routing weight)
+ *
+ * so out is the gradient of the forward's routed input rows (a_cat order); summing the
+ * rows of one token is gnf4_combine_topk with row_of_slot. The contraction runs over N,
+ * across rows with different block scales, so the scale multiplies each decoded bf16
+ * pair before the MMA: exact for MXFP4 (a power of two), one extra bf16 rounding of the
+ * scaled weight for NF4. fp32 accumulation in a fixed order (deterministic).
+ * grad_out   device bf16 [T_in, N], 16-byte aligned
+ * W, absmax  the forward's packed stack: u8 [E, N, K/2] (16-byte aligned), f32 [E, N, K/64]
+ * expert_offsets device int64 [E+1] as in the forward
+ * row_src    device int32 [R] in [0, T_in), or NULL (then T_in >= R)
+ * row_weight device fp32 [R], or NULL
+ * out        device bf16 [R, K], 16-byte aligned
+ * E in [1, 2048], N % 16 == 0, K % 64 == 0 (both formats), R >= 0 (R == 0 launches nothing
+ * and accepts NULL buffers). flags: 0 or GNF4_CHECK (validates offsets, row_src, row_weight
+ * first, as in the forward). One kernel launch (two with GNF4_CHECK).
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, DEVICE_STATUS (GNF4_CHECK), CUDA.
+ */
+gnf4_status gnf4_dgrad_nf4(const void* grad_out, const uint8_t* W, const float* absmax,
+                           const int64_t* expert_offsets, const int32_t* row_src,
+                           const float* row_weight, int64_t E, int64_t N, int64_t K, int64_t R,
+                           int64_t T_in, void* out, int flags, void* stream);
+
+/*
+ * The same input gradient on MXFP4-packed weights (scales u8 e8m0 [E, N, K/32]).
+ */
+gnf4_status gnf4_dgrad_mxfp4(const void* grad_out, const uint8_t* W, const uint8_t* scales,
+                             const int64_t* expert_offsets, const int32_t* row_src,
+                             const float* row_weight, int64_t E, int64_t N, int64_t K, int64_t R,
+                             int64_t T_in, void* out, int flags, void* stream);
+
+/*
  * SwiGLU over gate_up rows: the step between the gate_up and down grouped GEMMs
  * of a SwiGLU MoE layer (the decode glue "swiglu_rows" of the status page "MoE
  * Software Status & Known Limits", section "grouped-nf4-gemm", "Correctness

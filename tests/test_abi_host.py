@@ -116,3 +116,26 @@ def test_glue_argument_errors():
     addr = (ctypes.addressof(buf) + 15) & ~15
     assert sw(addr, 1, 8, addr + 64, None) == _lib.GNF4_ERR_INVALID_ARG
     assert b"device memory" in lib.gnf4_last_error()
+
+
+def test_dgrad_argument_errors():
+    dg = lib.gnf4_dgrad_nf4
+
+    def call(**kw):
+        a = dict(g=FAKE, W=FAKE, s=FAKE, off=FAKE, src=None, wt=None, E=4, N=128, K=256, R=8, T_in=8,
+                 out=FAKE, flags=0)
+        a.update(kw)
+        return dg(a["g"], a["W"], a["s"], a["off"], a["src"], a["wt"], a["E"], a["N"], a["K"], a["R"],
+                  a["T_in"], a["out"], a["flags"], None)
+
+    assert call(g=None) == _lib.GNF4_ERR_INVALID_ARG
+    assert call(E=0) == _lib.GNF4_ERR_INVALID_ARG
+    assert call(flags=_lib.GNF4_FORCE_DECODE) == _lib.GNF4_ERR_INVALID_ARG
+    assert call(K=96) == _lib.GNF4_ERR_UNSUPPORTED_SHAPE          # K % 64, both formats
+    assert lib.gnf4_dgrad_mxfp4(FAKE, FAKE, FAKE, FAKE, None, None, 4, 128, 96, 8, 8, FAKE, 0,
+                                None) == _lib.GNF4_ERR_UNSUPPORTED_SHAPE
+    assert call(N=120) == _lib.GNF4_ERR_UNSUPPORTED_SHAPE
+    assert call(E=4096) == _lib.GNF4_ERR_UNSUPPORTED_SHAPE
+    assert call(T_in=4) == _lib.GNF4_ERR_INVALID_ARG               # row_src NULL needs T_in >= R
+    assert call(g=FAKE + 4) == _lib.GNF4_ERR_MISALIGNED
+    assert call(R=0, g=None, W=None, s=None, off=None, out=None) == _lib.GNF4_OK   # no work
