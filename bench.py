@@ -59,10 +59,11 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--top-k", type=int, default=None, help="sweep workload: top_k (default first)")
     ap.add_argument("--tokens", type=str, default=None, help="comma list overriding the token counts")
-    ap.add_argument("--op", default="gemm", choices=["gemm", "dgrad"] + list(GLUE_OPS),
+    ap.add_argument("--op", default="gemm", choices=["gemm", "dgrad", "layer"] + list(GLUE_OPS),
                     help="gemm: the grouped GEMM step (default); dgrad: its input gradient, every "
-                         "call of the step; swiglu / combine: the glue kernel either side of it, on "
-                         "the workload's largest token count")
+                         "call of the step; layer: the whole MoE layer (device routing, gate_up, "
+                         "SwiGLU, down, combine) as one CUDA graph per token count; swiglu / combine: "
+                         "the glue kernel either side of the GEMM, on the workload's largest token count")
     return ap.parse_args()
 
 
@@ -876,9 +877,120 @@ def run_dgrad_bench(args, wl):
         dist.destroy_process_group()
 
 
+# --------------------------------------------------------------------------
+# one whole MoE layer per token count, captured as one CUDA graph
+# --------------------------------------------------------------------------
+def run_layer_bench(args, wl):
+    import torch
+    import bit_grouped_moe_gnf4_b200 as g
+
+    if args.impl == "reference" or int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        if int(os.environ.get("RANK", "0")) == 0:
+            print(json.dumps({"impl": args.impl, "unavailable": "--op layer is a 1-GPU measurement of "
+                              "this library's layer; the oracle's layer is timed by --op gemm/swiglu/combine"}))
+        return
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    k = args.top_k if args.top_k is not None else wl.top_k[-1]
+    Ts = _tokens(args) or list(wl.T)
+    gu, dn = wl.projections
+    H, I2 = gu.K, gu.N
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(args.seed)
+
+    def stack(proj):
+        Wl, Sl = [], []
+        for e in range(wl.E):
+            w = torch.randn((proj.N, proj.K), generator=gen, device=dev, dtype=torch.float32) * 0.02
+            p_, s_ = g.quantize_nf4(w) if wl.fmt == "nf4" else g.quantize_mxfp4(w)
+            Wl.append(p_)
+            Sl.append(s_)
+        return torch.stack(Wl), torch.stack(Sl)
+
+    Wg, Sg = stack(gu)
+    Wd, Sd = stack(dn)
+    scratch = torch.empty(64 * 2 ** 20, dtype=torch.float32, device=dev)     # 256 MB: flushes L2
+    layers = []
+    for T in Ts:
+        ids, w = (G_route(wl))(args.seed, T, wl.E, k)
+        b = synth.make_routed_batch(args.seed, T, wl.E, k, routing=wl.routing)
+        R = T * k
+        d = {"ids": torch.from_numpy(ids.astype(np.int32)).to(dev), "w": torch.from_numpy(w).to(dev),
+             "x": torch.from_numpy(synth.activations_bf16(args.seed, T, H).view(np.int16)).to(dev).view(torch.bfloat16),
+             "h": torch.empty((R, I2), dtype=torch.bfloat16, device=dev),
+             "a": torch.empty((R, I2 // 2), dtype=torch.bfloat16, device=dev),
+             "y": torch.empty((R, dn.N), dtype=torch.bfloat16, device=dev),
+             "out": torch.empty((T, dn.N), dtype=torch.bfloat16, device=dev)}
+        nbytes = call_bytes(wl.fmt, gu, b)[0] + call_bytes(wl.fmt, dn, b)[0]
+        layers.append((T, d, nbytes, b))
+
+    def layer(d, T):
+        st = torch.cuda.current_stream()
+        off, tok, wt, dst = g.routing_metadata(d["ids"], d["w"], wl.E, stream=st)
+        g.grouped_gemm(wl.fmt, d["x"], Wg, Sg, off, row_token=tok, out=d["h"], R=T * k, stream=st)
+        g.swiglu(d["h"], out=d["a"], stream=st)
+        g.grouped_gemm(wl.fmt, d["a"], Wd, Sd, off, row_weight=wt, row_dest=dst, out=d["y"], R=T * k, stream=st)
+        g.combine_topk(d["y"], T, k, out=d["out"], stream=st)
+
+    for _ in range(args.warmup):
+        for T, d, _, _ in layers:
+            layer(d, T)
+    torch.cuda.synchronize()
+    g.device_status()
+    graphs = []
+    cap = torch.cuda.Stream()
+    for T, d, _, _ in layers:
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=cap, capture_error_mode="thread_local"):
+            layer(d, T)
+        graphs.append(gr)
+    torch.cuda.synchronize()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in layers]
+          for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        for j in range(len(layers)):
+            scratch.fill_(float(i))                      # L2 flushed before each layer
+            ev[i][j][0].record(stream)
+            graphs[j].replay()
+            ev[i][j][1].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    g.device_status()
+    ms = np.array([[a.elapsed_time(b_) for a, b_ in row] for row in ev]).mean(axis=0)
+    tokens = sum(T for T, _, _, _ in layers)
+    wbytes = sum(nb for _, _, nb, _ in layers)
+    hbm, _, _, src = measured_peaks()
+    achieved = wbytes / (ms.sum() * 1e-3) / 1e9
+    line = {"metric": "MoE layer (device routing, gate_up, SwiGLU, down, combine): tokens/s",
+            "value": tokens / (ms.sum() * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": float(ms.sum()), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "layer of " + describe(wl, k), "l2": "flushed (256 MB write) before each layer",
+                       "layers": [f"T={T}" for T, _, _, _ in layers]},
+            "gpu_launches": 5 * len(layers) * args.steps,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                         "peak_source": f"{src} HBM copy", "traffic": None,
+                         "note": "packed-weight bytes of both projections over the whole layer's time",
+                         "per_layer_ms": [round(float(x), 5) for x in ms]},
+            "clocks": clk}
+    print(json.dumps(line), flush=True)
+
+
+def G_route(wl):
+    from synth import generators as G
+    return G.route_softmax_topk if wl.routing == "softmax" else G.route_zipf_topk
+
+
 def main():
     args = parse()
     wl = WORKLOADS[args.workload]
+    if args.op == "layer":
+        run_layer_bench(args, wl)
+        return
     if args.op == "dgrad":
         run_dgrad_bench(args, wl)
         return

@@ -29,7 +29,7 @@ STATUS_NAMES = {0: "GNF4_OK", 1: "GNF4_ERR_INVALID_ARG", 2: "GNF4_ERR_UNSUPPORTE
 EXPORTED = ("gnf4_last_error", "gnf4_version", "gnf4_quantize_nf4", "gnf4_quantize_mxfp4",
             "gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4", "gnf4_grouped_gemm_launches",
             "gnf4_device_status", "gnf4_swiglu", "gnf4_combine_topk", "gnf4_dgrad_nf4",
-            "gnf4_dgrad_mxfp4")
+            "gnf4_dgrad_mxfp4", "gnf4_routing_metadata")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
@@ -53,6 +53,8 @@ for _name in ("gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4"):
 for _name in ("gnf4_dgrad_nf4", "gnf4_dgrad_mxfp4"):
     getattr(lib, _name).restype = _i32
     getattr(lib, _name).argtypes = [_p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _i64, _p, _i32, _p]
+lib.gnf4_routing_metadata.restype = _i32
+lib.gnf4_routing_metadata.argtypes = [_p, _p, _i64, _i64, _i64, _p, _p, _p, _p, _p]
 lib.gnf4_swiglu.restype = _i32
 lib.gnf4_swiglu.argtypes = [_p, _i64, _i64, _p, _p]
 lib.gnf4_combine_topk.restype = _i32

@@ -153,6 +153,29 @@ def dgrad(fmt: str, grad_out: torch.Tensor, W: torch.Tensor, scales: torch.Tenso
     return out
 
 
+def routing_metadata(topk_ids: torch.Tensor, topk_weights: Optional[torch.Tensor], E: int,
+                     stream=None):
+    """Router top-k ``[T, k]`` (int32 ids, fp32 weights or None) -> (expert_offsets int64 [E+1],
+    row_token int32 [T*k], row_weight fp32 [T*k] or None, row_dest int32 [T*k]) on the device,
+    rows sorted by (expert, token, slot) (include/gnf4.h)."""
+    _need(topk_ids, torch.int32, "topk_ids")
+    if topk_ids.dim() != 2:
+        raise ValueError("topk_ids must be [T, k]")
+    T, k = topk_ids.shape
+    if topk_weights is not None:
+        _need(topk_weights, torch.float32, "topk_weights")
+        if tuple(topk_weights.shape) != (T, k):
+            raise ValueError("topk_weights must match topk_ids")
+    dev = topk_ids.device
+    offsets = torch.empty(E + 1, dtype=torch.int64, device=dev)
+    row_token = torch.empty(T * k, dtype=torch.int32, device=dev)
+    row_weight = None if topk_weights is None else torch.empty(T * k, dtype=torch.float32, device=dev)
+    row_dest = torch.empty(T * k, dtype=torch.int32, device=dev)
+    check(lib.gnf4_routing_metadata(_ptr(topk_ids), _ptr(topk_weights), T, k, E, _ptr(offsets), _ptr(row_token),
+                                    _ptr(row_weight), _ptr(row_dest), _stream(stream)), "gnf4_routing_metadata")
+    return offsets, row_token, row_weight, row_dest
+
+
 def swiglu(gate_up: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """bf16 ``[R, 2I]`` gate_up rows -> bf16 ``[R, I]``: ``silu(gate) * up`` (include/gnf4.h)."""
     _need(gate_up, torch.bfloat16, "gate_up")

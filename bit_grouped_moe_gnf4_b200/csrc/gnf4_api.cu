@@ -379,6 +379,29 @@ gnf4_status gnf4_dgrad_mxfp4(const void* grad_out, const uint8_t* W, const uint8
                  out, flags, stream);
 }
 
+gnf4_status gnf4_routing_metadata(const int32_t* topk_ids, const float* topk_weights, int64_t T,
+                                  int64_t k, int64_t E, int64_t* expert_offsets, int32_t* row_token,
+                                  float* row_weight, int32_t* row_dest, void* stream) {
+    if (T < 0 || k < 1 || E < 1) return fail(GNF4_ERR_INVALID_ARG, "sizes must be T >= 0, k >= 1, E >= 1");
+    if (E > 2048) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "at most 2048 experts");
+    if (k > INT_MAX || T > (int64_t)INT_MAX / k) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "T*k must fit in int32");
+    if (!expert_offsets || (T > 0 && (!row_token || !topk_ids)))   // T == 0: empty row arrays may be NULL
+        return fail(GNF4_ERR_INVALID_ARG, "null pointer argument");
+    if (T > 0 && (topk_weights == nullptr) != (row_weight == nullptr))
+        return fail(GNF4_ERR_INVALID_ARG, "topk_weights and row_weight are given together or not at all");
+    const void* ptrs[] = {topk_ids, topk_weights, expert_offsets, row_token, row_weight, row_dest};
+    for (const void* q : ptrs) {
+        if (!q) continue;
+        if (reinterpret_cast<uintptr_t>(q) & 3u) return fail(GNF4_ERR_MISALIGNED, "buffers must be 4-byte aligned");
+        if (!is_device_ptr(q)) return fail(GNF4_ERR_INVALID_ARG, "every buffer must be device memory of the current device");
+    }
+    if (reinterpret_cast<uintptr_t>(expert_offsets) & 7u)
+        return fail(GNF4_ERR_MISALIGNED, "expert_offsets must be 8-byte aligned");
+    cudaError_t e = launch_routing(topk_ids, topk_weights, T, k, (int)E, expert_offsets, row_token, row_weight,
+                                   row_dest, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GNF4_OK : cuda_fail(e, "routing launch");
+}
+
 int gnf4_grouped_gemm_launches(int64_t R, int flags) {
     if (R <= 0) return 0;
     int n = (flags & GNF4_CHECK) ? 1 : 0;

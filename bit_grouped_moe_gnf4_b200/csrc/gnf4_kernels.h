@@ -51,6 +51,11 @@ cudaError_t launch_dgrad(int fmt, const DgradArgs& a, cudaStream_t s);
 int dgrad_row_tiles(int64_t R, int E);
 int dgrad_splits(int64_t R, int E, int N, int K, int rt);
 
+// Routing metadata from the router's top-k choices (one CTA; sizes validated).
+cudaError_t launch_routing(const int32_t* ids, const float* weights, int64_t T, int64_t k, int E,
+                           int64_t* offsets, int32_t* row_token, float* row_weight, int32_t* row_dest,
+                           cudaStream_t s);
+
 int device_sm_count();
 
 // Read and clear the error word a band's kernels set when they give up waiting

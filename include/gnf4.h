@@ -188,6 +188,31 @@ gnf4_status gnf4_dgrad_mxfp4(const void* grad_out, const uint8_t* W, const uint8
                              int64_t T_in, void* out, int flags, void* stream);
 
 /*
+ * Routing metadata on the device: the router's top-k choices become the arguments of a
+ * grouped call, so that a whole MoE layer runs without the host. The grouped call takes
+ * its rows "group-sorted", with sort and scatter outside the kernel (solution page,
+ * "Supported scope"; "Smallest correct example": sizes per expert, rows of one expert
+ * contiguous). Routed rows are the pairs (t, s), t < T, s < k, ordered by expert
+ * topk_ids[t*k + s], then t, then s (a stable counting sort):
+ *   expert_offsets[e] = number of pairs with expert < e           (int64 [E+1])
+ *   row r = pair (t, s):  row_token[r] = t, row_dest[r] = t*k + s, row_weight[r] = topk_weights[t*k + s]
+ * An id outside [0, E) is a dropped slot and gets no row; then R = expert_offsets[E] < T*k
+ * and only the first R entries of the row arrays are written. With every id valid R = T*k,
+ * known on the host, and the grouped calls can be captured in one CUDA graph with this one.
+ * topk_ids     device int32 [T, k] (with T == 0 the row arrays and topk_ids may be NULL;
+ *              expert_offsets is still written, all zero)
+ * topk_weights device fp32 [T, k], or NULL (then row_weight must be NULL)
+ * expert_offsets device int64 [E+1] (8-byte aligned); row_token device int32 [T*k];
+ * row_weight device fp32 [T*k] or NULL; row_dest device int32 [T*k] or NULL
+ * E in [1, 2048], T*k < 2^31. One kernel launch of one CTA; deterministic (the same bits
+ * on every call), no atomics on the outputs.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, CUDA.
+ */
+gnf4_status gnf4_routing_metadata(const int32_t* topk_ids, const float* topk_weights, int64_t T,
+                                  int64_t k, int64_t E, int64_t* expert_offsets, int32_t* row_token,
+                                  float* row_weight, int32_t* row_dest, void* stream);
+
+/*
  * SwiGLU over gate_up rows: the step between the gate_up and down grouped GEMMs
  * of a SwiGLU MoE layer (the decode glue "swiglu_rows" of the status page "MoE
  * Software Status & Known Limits", section "grouped-nf4-gemm", "Correctness

@@ -139,3 +139,14 @@ def test_dgrad_argument_errors():
     assert call(T_in=4) == _lib.GNF4_ERR_INVALID_ARG               # row_src NULL needs T_in >= R
     assert call(g=FAKE + 4) == _lib.GNF4_ERR_MISALIGNED
     assert call(R=0, g=None, W=None, s=None, off=None, out=None) == _lib.GNF4_OK   # no work
+
+
+def test_routing_argument_errors():
+    rm = lib.gnf4_routing_metadata
+    assert rm(FAKE, FAKE, 8, 0, 16, FAKE, FAKE, FAKE, FAKE, None) == _lib.GNF4_ERR_INVALID_ARG     # k = 0
+    assert rm(FAKE, FAKE, 8, 2, 0, FAKE, FAKE, FAKE, FAKE, None) == _lib.GNF4_ERR_INVALID_ARG     # E = 0
+    assert rm(FAKE, FAKE, 8, 2, 4096, FAKE, FAKE, FAKE, FAKE, None) == _lib.GNF4_ERR_UNSUPPORTED_SHAPE
+    assert rm(FAKE, FAKE, 1 << 30, 4, 16, FAKE, FAKE, FAKE, FAKE, None) == _lib.GNF4_ERR_UNSUPPORTED_SHAPE
+    assert rm(None, FAKE, 8, 2, 16, FAKE, FAKE, FAKE, FAKE, None) == _lib.GNF4_ERR_INVALID_ARG
+    assert rm(FAKE, FAKE, 8, 2, 16, FAKE, FAKE, None, FAKE, None) == _lib.GNF4_ERR_INVALID_ARG    # weights without row_weight
+    assert rm(FAKE + 2, None, 8, 2, 16, FAKE, FAKE, None, FAKE, None) == _lib.GNF4_ERR_MISALIGNED
