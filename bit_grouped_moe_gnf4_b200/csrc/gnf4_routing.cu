@@ -6,8 +6,8 @@
 // packed MoE expert weights, without dequantizing to bf16 first?", "Supported
 // scope"); this is that sort.
 //
-// One CTA of NW warps. The n = T*k pairs are cut into NW contiguous segments,
-// one per warp, in pair order.
+// One CTA of NW warps (about one per 512 pairs, at most 32). The n = T*k pairs are
+// cut into NW contiguous segments, one per warp, in pair order.
 //   1. Each warp counts its segment per expert: lanes with the same expert find
 //      each other with __match_any_sync and the lowest of them adds the group's
 //      size to the warp's row of a [NW][E] count table in shared memory.
@@ -59,6 +59,7 @@ __global__ void routing_kernel(const int32_t* __restrict__ ids, const float* __r
         }
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
+            if (base + 32 * u >= i1) break;           // warp-uniform: no pair left in this round
             const int e = ev[u];
             const bool valid = e >= 0 && e < E;
             const unsigned peers = __match_any_sync(0xffffffffu, valid ? e : -1 - lane);
@@ -110,6 +111,7 @@ __global__ void routing_kernel(const int32_t* __restrict__ ids, const float* __r
         }
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
+            if (base + 32 * u >= i1) break;           // warp-uniform: no pair left in this round
             const int64_t i = base + 32 * u + lane;
             const int e = ev[u];
             const bool valid = e >= 0 && e < E;
@@ -134,16 +136,20 @@ __global__ void routing_kernel(const int32_t* __restrict__ ids, const float* __r
 
 }  // namespace
 
-int routing_warps(int E) {
-    // the count table is NW x E words; keep it within 200 KB of shared memory
+int routing_warps(int E, int64_t n) {
+    // about 512 pairs per warp (a small call takes one warp: every warp pays for the
+    // count table and the scans); the table is NW x E words, within 200 KB of shared memory
     const int fit = (int)((200 * 1024) / (4 * (int64_t)(E > 0 ? E : 1))) - 1;
-    return fit < 1 ? 1 : (fit < kRouteMaxWarps ? fit : kRouteMaxWarps);
+    const int64_t by_n = (n + 511) / 512;
+    int nw = fit < kRouteMaxWarps ? fit : kRouteMaxWarps;
+    if (by_n < nw) nw = (int)by_n;
+    return nw < 1 ? 1 : nw;
 }
 
 cudaError_t launch_routing(const int32_t* ids, const float* weights, int64_t T, int64_t k, int E,
                            int64_t* offsets, int32_t* row_token, float* row_weight, int32_t* row_dest,
                            cudaStream_t s) {
-    const int nw = routing_warps(E);
+    const int nw = routing_warps(E, T * k);
     const size_t smem = ((size_t)nw * E + E + 1) * sizeof(uint32_t);
     static size_t attr = 0;
     if (smem > 48 * 1024 && attr < smem) {
