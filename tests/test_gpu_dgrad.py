@@ -48,6 +48,19 @@ def test_small_ragged_all_elements(fmt, counts):
     check_rows(got2, ref2, f"dgrad {fmt} {counts} plain")
 
 
+@pytest.mark.parametrize("fmt", ["nf4", "mxfp4"])
+def test_two_row_tiles_with_split_contraction(fmt):
+    """Groups averaging 66 rows over a narrow K: the host picks two 16-row tiles per item
+    and an 8-way split of the contraction (partial sums added through shared memory)."""
+    counts, N, K = [100, 0, 60, 40], 512, 128
+    Wd, Sd, Wh, Sh = build_stack(fmt, len(counts), N, K, seed=34)
+    b = G.explicit_batch(counts, seed=35)
+    g = synth.activations_bf16(36, b.R, N, tag="y")
+    got = run_dgrad(fmt, g, Wd, Sd, b.offsets, None, b.row_weight)
+    ref = D.dgrad_rows_f64(fmt, g, Wh, Sh, b.offsets, None, b.row_weight, np.arange(b.R))
+    check_rows(got, ref, f"dgrad {fmt} RT=2 split")
+
+
 def test_one_hot_mxfp4_reads_the_weight_row_exactly():
     E, N, K = 2, 64, 256
     Wd, Sd, Wh, Sh = build_stack("mxfp4", E, N, K, seed=25)
