@@ -18,8 +18,12 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
 
 
 def _stream(stream) -> int:
+    """A torch.cuda.Stream, a raw cudaStream_t handle as an int (0 = the legacy default
+    stream), or None for torch's current stream."""
     if stream is None:
         stream = torch.cuda.current_stream()
+    if isinstance(stream, int):
+        return stream
     return stream.cuda_stream
 
 
