@@ -451,13 +451,17 @@ def run_ours(args, wl):
     roof["kernel"] = "prefill_band_kernel" if prefill else "decode_band_kernel"
     roof["per_call_ms"] = [round(float(x), 5) for x in mean_call_ms]
     roof["per_call"] = [f"T={c['T']} {c['proj'].name}" for c in prepared]
+    # the same step counted on the 4-bit codes alone (no scale bytes)
+    work_nib = sum(c["nib"] for c in prepared)
+    roof["nibble_only_gbs"] = work_nib / (call_ms.sum(axis=1).mean() * 1e-3) / 1e9
 
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": describe(wl, k), "format": wl.fmt,
-                   "algorithmic_bytes_per_step": work_bytes, "flop_per_step": work_flop,
+                   "algorithmic_bytes_per_step": work_bytes, "nibble_bytes_per_step": work_nib,
+                   "flop_per_step": work_flop,
                    "l2": f"rotating {ncopies} weight-stack copies ({ncopies * stack_bytes / 1e6:.0f} MB; "
                          f"step reads {step_bytes / 1e6:.0f} MB; L2 {l2 / 1e6:.0f} MB)",
                    "parallelism": f"replicas x{world}"},
