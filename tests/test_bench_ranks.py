@@ -85,3 +85,26 @@ def test_reference_arm_rank0_prints_one_line():
     assert d["unit"] == "GB/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_glue_and_dgrad_accounting():
+    """Byte counts of the glue legs and the inputs of the gradient leg, on the workload
+    shapes (host arithmetic only)."""
+    import bench
+    import synth
+    from synth.workloads import WORKLOADS
+    wl = WORKLOADS["qwen3_prefill_nf4"]
+    # SwiGLU: [32768, 1536] bf16 read, [32768, 768] written
+    assert bench.glue_problem("swiglu", wl, 8, 4096) == (32768, 1536, 32768, 768,
+                                                         32768 * 1536 * 2 + 32768 * 768 * 2)
+    # combine: [32768, 2048] read, [4096, 2048] written
+    assert bench.glue_problem("combine", wl, 8, 4096) == (32768, 2048, 4096, 2048,
+                                                          32768 * 2048 * 2 + 4096 * 2048 * 2)
+    # gradient of down: gathered from the forward's scatter rows with its weights;
+    # gradient of gate_up: rows already in routed order, unweighted
+    b = synth.make_routed_batch(0, 16, 64, 8)
+    gu, dn = WORKLOADS["olmoe_decode_nf4"].projections
+    src, wt, gb = bench.dgrad_call_inputs(dn, b, 0)
+    assert src is b.row_dest and wt is b.row_weight and gb.shape == (16 * 8, dn.N)
+    src, wt, gb = bench.dgrad_call_inputs(gu, b, 0)
+    assert src is None and wt is None and gb.shape == (b.R, gu.N)
