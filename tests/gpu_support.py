@@ -83,6 +83,27 @@ def check_rows(out_bits, ref_f64, what=""):
     return worst
 
 
+GROUP_FROB_TOL = 1e-2
+
+
+def check_group_frobenius(out_bits, ref_f64, offsets, what=""):
+    """The pages' own bound beside the per-row one: per expert group, relative Frobenius
+    error ||out - ref||_F / ||ref||_F <= 1e-2 (rows aligned with the routed order)."""
+    got = O.bf16_to_f64(out_bits)
+    worst = 0.0
+    offsets = np.asarray(offsets)
+    for e in range(len(offsets) - 1):
+        r0, r1 = int(offsets[e]), int(offsets[e + 1])
+        if r1 <= r0:
+            continue
+        den = np.linalg.norm(ref_f64[r0:r1])
+        if den == 0:
+            continue
+        worst = max(worst, float(np.linalg.norm(got[r0:r1] - ref_f64[r0:r1]) / den))
+    assert worst <= GROUP_FROB_TOL, f"{what}: group relative Frobenius error {worst:.3e} > {GROUP_FROB_TOL}"
+    return worst
+
+
 def run_gemm(fmt, x_bits, Wd, Sd, offsets, row_token=None, row_weight=None, row_dest=None,
              T_out=None, flags=0, out_init_bits=None):
     import bit_grouped_moe_gnf4_b200 as g

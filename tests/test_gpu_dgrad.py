@@ -16,7 +16,8 @@ from oracle import gnf4_oracle as O
 from synth import generators as G
 from synth.workloads import WORKLOADS
 
-from gpu_support import bf16_dev, bf16_host_bits, build_stack, check_rows, sample_rows, to_dev
+from gpu_support import (bf16_dev, bf16_host_bits, build_stack, check_group_frobenius, check_rows,
+                         sample_rows, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -42,6 +43,7 @@ def test_small_ragged_all_elements(fmt, counts):
     got = run_dgrad(fmt, g, Wd, Sd, b.offsets, src, b.row_weight)
     ref = D.dgrad_rows_f64(fmt, g, Wh, Sh, b.offsets, src, b.row_weight, np.arange(b.R))
     check_rows(got, ref, f"dgrad {fmt} {counts}")
+    check_group_frobenius(got, ref, b.offsets, f"dgrad {fmt} {counts}")
     # rows already in routed order, no weight
     got2 = run_dgrad(fmt, g[:b.R], Wd, Sd, b.offsets)
     ref2 = D.dgrad_rows_f64(fmt, g[:b.R], Wh, Sh, b.offsets, None, None, np.arange(b.R))

@@ -13,8 +13,8 @@ from oracle import gnf4_oracle as O
 from synth import generators as G
 from synth.workloads import WORKLOADS
 
-from gpu_support import (bf16_dev, bf16_host_bits, build_stack, check_rows, run_gemm,
-                         sample_rows, to_dev)
+from gpu_support import (bf16_dev, bf16_host_bits, build_stack, check_group_frobenius, check_rows,
+                         run_gemm, sample_rows, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -40,6 +40,7 @@ def test_tiny_all_elements(fmt, band):
                    T_out=T * k, flags=BANDS[band])
     ref = O.grouped_rows_f64(fmt, x, Wh, Sh, b.offsets, b.row_token, b.row_weight, K, np.arange(b.R))
     check_rows(out[b.row_dest], ref, f"tiny {fmt} {band}")
+    check_group_frobenius(out[b.row_dest], ref, b.offsets, f"tiny {fmt} {band}")
 
 
 @pytest.mark.parametrize("fmt", ["nf4", "mxfp4"])
@@ -56,6 +57,7 @@ def test_ragged_groups_several_tiles(fmt, band):
                    T_out=b.R, flags=BANDS[band])
     ref = O.grouped_rows_f64(fmt, x, Wh, Sh, b.offsets, b.row_token, b.row_weight, K, np.arange(b.R))
     check_rows(out[b.row_dest], ref, f"ragged {fmt} {band}")
+    check_group_frobenius(out[b.row_dest], ref, b.offsets, f"ragged {fmt} {band}")
 
 
 @pytest.mark.parametrize("fmt", ["nf4", "mxfp4"])
