@@ -236,6 +236,18 @@ def oracle_sample(wl, calls, budget_s=15.0, seed=0):
     return done_bytes, done_flop, ncalls, gemm_s, cores
 
 
+def oracle_one_core(wl, calls, seed, prefill, budget_s=4.0):
+    """The same oracle sample with its BLAS limited to one thread (None if that limit
+    cannot be set): the single-core figure beside the all-cores one."""
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            nb, nf, nc, dt, _ = oracle_sample(wl, calls, budget_s=budget_s, seed=seed)
+        return (nf / dt / 1e12) if prefill else (nb / dt / 1e9)
+    except Exception:
+        return None
+
+
 def run_reference(args, wl):
     """The reference arm: the oracle as it stands, timed on the host cores."""
     rank = int(os.environ.get("RANK", "0"))
@@ -478,6 +490,9 @@ def run_ours(args, wl):
                                 "sample": f"{nc} whole grouped GEMM calls of the step (smallest token "
                                           f"counts first); {dt:.1f} s in the oracle's grouped GEMM, "
                                           f"its quantization of the inputs untimed"}
+        one = oracle_one_core(wl, [(c["T"], c["proj"], c["b"]) for c in prepared], args.seed, prefill)
+        if one is not None:
+            line["cpu_baseline"]["value_one_core"] = one
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
