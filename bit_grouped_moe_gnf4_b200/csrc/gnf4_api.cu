@@ -157,6 +157,12 @@ static gnf4_status grouped(int fmt, const void* x, const uint8_t* W, const void*
     if (R > 0 && (T_in == 0 || T_out == 0)) return fail(GNF4_ERR_INVALID_ARG, "R > 0 needs T_in, T_out >= 1");
     if (!aligned16(x) || !aligned16(W) || !aligned16(out))
         return fail(GNF4_ERR_MISALIGNED, "x, W and out must be 16-byte aligned");
+    if (fmt == FMT_NF4 && (reinterpret_cast<uintptr_t>(scales) & 3u))
+        return fail(GNF4_ERR_MISALIGNED, "absmax must be 4-byte aligned (fp32)");
+    if ((reinterpret_cast<uintptr_t>(offsets) & 7u) || (row_token && (reinterpret_cast<uintptr_t>(row_token) & 3u)) ||
+        (row_weight && (reinterpret_cast<uintptr_t>(row_weight) & 3u)) ||
+        (row_dest && (reinterpret_cast<uintptr_t>(row_dest) & 3u)))
+        return fail(GNF4_ERR_MISALIGNED, "expert_offsets must be 8-byte and row arrays 4-byte aligned");
     if (!is_device_ptr(x) || !is_device_ptr(W) || !is_device_ptr(scales) || !is_device_ptr(offsets) ||
         !is_device_ptr(out) || (row_token && !is_device_ptr(row_token)) ||
         (row_weight && !is_device_ptr(row_weight)) || (row_dest && !is_device_ptr(row_dest)))

@@ -1,52 +1,58 @@
-// Decode band of the grouped 4-bit GEMM: groups with few routed rows, where
-// the packed weight bytes are the whole cost (the GEMV path of the solution page
-// "How do I run a grouped GEMM directly on NF4 packed MoE expert weights,
-// without dequantizing to bf16 first?", "Supported scope": one-token groups
-// take the GEMV path).
+// Decode band of the grouped 4-bit GEMM: groups with few routed rows, where the
+// packed weight bytes are the whole cost (the GEMV path of the solution page "How
+// do I run a grouped GEMM directly on NF4 packed MoE expert weights, without
+// dequantizing to bf16 first?", "Supported scope": one-token groups take the
+// GEMV path; the status page "MoE Software Status & Known Limits", "Decode and
+// serving": a bandwidth-targeted expert GEMV).
 //
-// One persistent CTA per SM takes a contiguous run of work items; an item is
-// (active expert, ROWS = 48 weight rows; fewer when K is very large). A producer
-// thread streams each item's packed rows, one K chunk of 256 at a time, into a
-// ring of 8 KB shared-memory stages with one 2-D TMA load per chunk (a box of
-// 128 bytes x ROWS rows, 128B-swizzled); the stage holds nothing else, so the
-// producer issues one copy per stage and the copy engine keeps HBM busy. The
-// item's block scales (ROWS rows x all blocks, one contiguous range) land in a
-// scale slot with a barrier of their own, issued one item ahead.
+// Work. A unit is (active expert, tile of 64 weight rows, pass), where a pass
+// covers up to 8*NG routed rows of the expert (larger groups take several
+// passes). Units are numbered expert by expert, tile-major, and every CTA of the
+// persistent grid (one per SM, 16 warps) takes an equal contiguous range. The 16
+// warps form 4 quads; warp w of a quad owns rows 16w .. 16w + 15 of a tile. The K
+// axis of a tile is cut into np parts (np depends on K alone); the quads form
+// 4/np groups of np quads, group gi takes the CTA's units gi, gi + 4/np, ..., and
+// quad p of the group computes part p of each of them.
 //
-// 12 consumer warps: warp (rt, ks) owns row tile rt (16 rows of the item) and
-// the K chunks kc with kc % nks == ks (nks = 4 for 48-row items, so K chunks
-// of any multiple of 1024 split evenly), so each stage is read by ROWS/16 warps
-// and stages are consumed in parallel. Ownership goes
-// by K position only, so the fp32 grouping of a row's sum never depends on the
-// other rows of the call. Because owners skip the stages of other warps, a ring
-// slot carries a tag naming the chunk that was last issued into it; an owner
-// reads the slot's barrier only once the tag shows its chunk, which keeps
-// every parity wait within one phase.
+// Loads. The packed weights stream through the tensor memory accelerator: one
+// lane of each quad issues, per 256-K chunk, one 2-D box of 64 rows x 128 bytes
+// (8 KB, 128B-swizzled) into a 3-stage ring of the quad, so two chunks (64 KB a
+// CTA) are in flight while the quad reads the third. A full barrier per stage
+// carries the copy's byte count; an empty barrier per stage collects the four
+// warps' release before the stage is refilled. Block scales and activations are
+// small: each warp reads its rows' scales one chunk ahead into registers, and the
+// activations (shared by every tile of an expert) through L1.
 //
-// The activations of the routed rows are small and shared by every item of an
-// expert, so the consumers read them straight from global memory through L1
-// (prefetched into L1 before the wait for the chunk's weights). Nibbles are
-// decoded by a table in shared memory that maps each packed byte to its two
-// bf16 values (replicated per lane, so 32 lookups never conflict; a byte
-// permute forms the address); for MXFP4, whose register decode is short, one
-// of the lane's two rows goes through byte permutes on register tables instead,
-// to spread the work over the shared-memory and ALU pipes. The products run on warp-level bf16 MMAs with 16
-// weight rows as the M side and up to 8 routed rows per MMA as the N side.
-// Every MMA chain covers exactly one scale block (64 K for NF4, 32 K for
-// MXFP4), so the block sum leaves the tensor core in fp32 and is scaled and
-// accumulated in fp32 outside it.
+// Decode. A lane-replicated table in shared memory maps each packed byte to its
+// two 16-bit values (entry b of lane l at b*256 + l*4: 32 lookups hit 32 banks).
+// The table sits on a 64 KB boundary of the shared window, so one byte permute
+// forms a lookup's whole address. It holds the codebook rounded to the
+// activations' 16-bit type: the NF4 values, or the OCP e2m1 values with bit 3 as
+// the sign.
 //
-// At the end of each pass over an item the consumer warps hand their fp32
-// partial sums to an epilogue warp through double-buffered slots (kept in the
-// unused half of every 256-byte row of the lookup table) and go on; the
-// epilogue warp adds the K splits in a fixed order (deterministic), applies the
-// routing weight, rounds to bf16 and stores at the destination rows.
+// Math. Warp-level MMAs (m16n8k16, 16 weight rows x 8 routed rows) run one
+// chain per scale block (64 K for NF4, 32 K for MXFP4), so every block sum
+// leaves the tensor core in fp32 and is multiplied by its fp32 block scale and
+// accumulated outside it. Lane (g, t) supplies the k-slots 2t, 2t+1, 2t+8, 2t+9
+// of rows g and g+8; they are mapped to the four consecutive K positions
+// 16t + 4s + {0,1,2,3} (NF4) or 8t + 4s + {..} (MXFP4) of step s inside the
+// block, the same for both operands, so each lane reads contiguous bytes.
 //
-// MMA k-slot mapping: in m16n8k16, lane (g, t) supplies k-slots 2t, 2t+1,
-// 2t+8, 2t+9 of both operands. They are mapped to the four consecutive K
-// positions base + (SB/4)*t + 4*s + {0,1,2,3} of step s, the same for A and
-// B, so each lane reads contiguous bytes of the packed rows and of x.
+// Order of the fp32 sums. Each part's sum runs over its blocks in K order; the
+// parts' sums are added in part order. np and the parts depend on K only, so a
+// row's bits never depend on the other rows of the call (row-count invariance)
+// nor on which warp or CTA computed it. With np > 1 the quads of a group hand
+// their part sums over shared memory (double-buffered, one named barrier per
+// unit) and each warp reduces a share of its rows, applies the routing weight,
+// rounds and scatters. Nothing but the output is written to global memory.
+//
+// Waits. Every barrier wait is bounded: a wait that gives up records an error
+// for gnf4_device_status, raises the CTA's abort flag (every other wait then
+// returns at once, the math is skipped, the named-barrier schedule is kept), and
+// before the CTA exits each quad's issuing lane waits, bounded again, for the
+// copies it issued.
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
@@ -62,25 +68,78 @@ __device__ unsigned g_decode_error;
 
 namespace db {
 
-constexpr int kConsumers = 12;                     // consumer warps: 4 row tiles x 3 K-split owners
-constexpr int kProducerWarp = kConsumers;          // one thread issues all copies
-constexpr int kEpilogueWarp = kConsumers + 1;      // reduces and stores the partial sums
-constexpr int kThreads = (kConsumers + 2) * 32;    // 14 warps: at most 4 per SM sub-partition,
-constexpr int kRegBound = 512;                     // so 128 registers a thread (bounds for 16 warps)
-constexpr int kChunkK = 256;                       // K per stage: 128 packed bytes per row = one TMA box
+constexpr int kWarps = 16;
+constexpr int kThreads = kWarps * 32;
+constexpr int kQuads = kWarps / 4;
+constexpr int kTileRows = 64;                  // weight rows of a unit: 16 per warp of a quad
+constexpr int kChunkK = 256;                   // K per chunk: 128 packed bytes of every row
 constexpr int kBoxBytes = 128;
-constexpr int kLutBytes = 256 * 256;               // byte value b, lane l -> offset b*256 + l*4
-constexpr int kMaxTableRows = 1024;                // routed rows whose metadata fits the CTA's table
-constexpr int kMaxRowTiles = 4;                    // ROWS / 16 is at most 3
+constexpr int kStageBytes = kTileRows * kBoxBytes;   // 8 KB: one TMA box
+constexpr int kStages = 3;
+constexpr int kLutBytes = 256 * 256;           // byte b, lane l -> b*256 + l*4 (bytes 128..255 of each row hold the part slots)
+constexpr int kMaxTableRows = 1024;            // routed rows whose metadata the CTA stages in shared memory
+constexpr int kMaxSmem = 227 * 1024;
+
+// calls whose groups can exceed this many routed rows take 16 rows per pass
+#ifndef GNF4_DB_NG1_MAX
+#define GNF4_DB_NG1_MAX 8
+#endif
+// most K parts of a tile (a power of two, at most kQuads)
+#ifndef GNF4_DB_MAXPARTS
+#define GNF4_DB_MAXPARTS 2
+#endif
 
 struct Plan {
-    int rows;         // weight rows per item (48, 32 or 16)
-    int nch;          // stages per item pass
-    int stage_bytes;  // rows x 128 bytes (a multiple of 1024)
-    int scale_bytes;  // slot for one item's scales (rows x all blocks), rounded to 128
-    int nstages;      // ring stages
-    int nslots;       // item scale slots
+    int np;          // K parts
+    int nc;          // chunks of kChunkK (the last may be short)
+    int nblk;        // scale blocks per weight row
+    int vec_scales;  // a chunk's scales of one row can be read with one vector load
+    int smem_bytes;  // dynamic shared memory of the launch
 };
+
+// Scale storage of the band: f32 (NF4 absmax), bf16 (NF4 absmax stored as bf16),
+// e8m0 (MXFP4).
+enum ScaleKind : int { SC_F32 = 0, SC_BF16 = 1, SC_E8M0 = 2 };
+
+template <int FMT>
+struct ChunkGeom {
+    static constexpr int SB = (FMT == FMT_NF4) ? 64 : 32;        // K per scale block
+    static constexpr int NB = kChunkK / SB;                       // blocks per chunk (4 or 8)
+    static constexpr int LB = SB / 8;                             // packed bytes per lane per row per block (8 or 4)
+    static constexpr int LW = LB / 4;                             // 32-bit words of them (2 or 1)
+};
+
+// raw scale bits of one chunk for the lane's rows g and g + 8
+template <int SCL>
+struct Scales {
+    uint32_t s[2][(SCL == SC_F32) ? 4 : 2];
+};
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint2 ld_nc_v2(const void* p) {
+    uint2 v;
+    asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_nc_u32(const void* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_nc_u16(const void* p) {
+    uint16_t v;
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_nc_u8(const void* p) {
+    uint16_t v;
+    asm volatile("ld.global.nc.u8 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
 
 __device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
     asm volatile(
@@ -88,525 +147,628 @@ __device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int
         " [%0], [%1, {%2, %3}], [%4];"
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
 }
-__device__ __forceinline__ void bulk_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
-}
 
-// Wait until the ring slot's tag names chunk `want` (the producer has issued it,
-// so the slot's previous fill was consumed). Bounded like mbar_wait_bounded.
-__device__ __forceinline__ bool wait_tag(const int* tag, uint32_t want, volatile int* abort_flag, unsigned* err,
-                                         unsigned code) {
-    const uint32_t a = smem_addr(tag);
-    uint32_t v;
-    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
-    if (v == want) return true;
-    const long long t0 = clock64();
-    for (uint32_t it = 1;; ++it) {
-        __nanosleep(64);
-        asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
-        if (v == want) return true;
-        if ((it & 7u) == 0u) {
-            if (*abort_flag) return false;
-            if (clock64() - t0 > kWaitTimeoutCycles) {
-                *abort_flag = 1;
-                atomicOr(err, code);
-                return false;
-            }
-        }
-    }
-}
-
-__device__ __forceinline__ void prefetch_l1(const void* p) {
-    asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
-}
-
-// Partial-sum slot of unit u (= ((buffer * row tiles + rt) * nks + ks) * GMAX + j)
-// for one lane: 512 bytes per unit, spread over four 128-byte holes of the lookup
-// table (bytes 128..255 of each 256-byte row, which the table leaves unused).
-__device__ __forceinline__ float4* red_slot(uint8_t* lut, int u, int lane) {
-    return reinterpret_cast<float4*>(lut + (u * 4 + (lane >> 3)) * 256 + 128 + (lane & 7) * 16);
-}
-
-// The MMAs of one chunk for one consumer warp: 16 weight rows (ra = row g, rb =
-// row g + 8 of the row tile) x NG groups of 8 routed rows x NBC scale blocks
-// (only the first nbc when the chunk is the ragged end of K).
-template <int FMT, int GMAX, int NG, bool FULL>
-__device__ __forceinline__ void chunk_mma(const uint8_t* __restrict__ st, const uint8_t* __restrict__ ss,
-                                          const uint8_t* __restrict__ lut, uint32_t lane_sel, const LutPlanes& L,
-                                          const uint16_t* xr0, const uint16_t* xr1, int ra, int rb, int t, int nbk,
-                                          int kc, int nbc, bool vec_scales, float (&acc)[GMAX][4]) {
-    constexpr int SB = (FMT == FMT_NF4) ? 64 : 32;   // K elements per scale block
-    constexpr int STEPS = SB / 16;                   // k16 MMA steps per block
-    constexpr int BPL = SB / 8;                      // packed bytes per lane per row per block (8 or 4)
-    constexpr int XW = SB / 8;                       // bf16x2 words of x per lane per block
-    constexpr int NBC = kChunkK / SB;                // scale blocks in a full chunk (4 or 8)
-    const int bg0 = kc * NBC;                        // first scale block of the chunk
-    // block scales of rows ra and rb for this chunk: one vector load per row when the
-    // rows' blocks are aligned for it, picked per block by selects (no local arrays)
-    float4 va4 = make_float4(0.f, 0.f, 0.f, 0.f), vb4 = va4;
-    uint2 va2 = make_uint2(0u, 0u), vb2 = va2;
-    const bool vec = FULL && vec_scales;
-    if (vec) {
-        if constexpr (FMT == FMT_NF4) {
-            va4 = *reinterpret_cast<const float4*>(ss + (ra * nbk + bg0) * 4);
-            vb4 = *reinterpret_cast<const float4*>(ss + (rb * nbk + bg0) * 4);
+// the chunk's block scales of rows g and g + 8 (sp at row g's first; s8 = 8 rows)
+template <int SCL>
+__device__ __forceinline__ void load_scales(Scales<SCL>& ck, const uint8_t* sp, int64_t s8, int nb, bool vec) {
+    const uint8_t* sq = sp + s8;
+    if constexpr (SCL == SC_F32) {
+        if (vec) {
+            const uint4 a = ld_nc_v4(sp);
+            const uint4 b = ld_nc_v4(sq);
+            ck.s[0][0] = a.x; ck.s[0][1] = a.y; ck.s[0][2] = a.z; ck.s[0][3] = a.w;
+            ck.s[1][0] = b.x; ck.s[1][1] = b.y; ck.s[1][2] = b.z; ck.s[1][3] = b.w;
         } else {
-            va2 = *reinterpret_cast<const uint2*>(ss + ra * nbk + bg0);
-            vb2 = *reinterpret_cast<const uint2*>(ss + rb * nbk + bg0);
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                ck.s[0][b] = b < nb ? ld_nc_u32(sp + 4 * b) : 0u;
+                ck.s[1][b] = b < nb ? ld_nc_u32(sq + 4 * b) : 0u;
+            }
+        }
+    } else if constexpr (SCL == SC_BF16) {
+        if (vec) {
+            const uint2 a = ld_nc_v2(sp);
+            const uint2 b = ld_nc_v2(sq);
+            ck.s[0][0] = a.x; ck.s[0][1] = a.y;
+            ck.s[1][0] = b.x; ck.s[1][1] = b.y;
+        } else {
+            uint32_t v0[4], v1[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                v0[b] = b < nb ? ld_nc_u16(sp + 2 * b) : 0u;
+                v1[b] = b < nb ? ld_nc_u16(sq + 2 * b) : 0u;
+            }
+            ck.s[0][0] = v0[0] | (v0[1] << 16); ck.s[0][1] = v0[2] | (v0[3] << 16);
+            ck.s[1][0] = v1[0] | (v1[1] << 16); ck.s[1][1] = v1[2] | (v1[3] << 16);
+        }
+    } else {
+        if (vec) {
+            const uint2 a = ld_nc_v2(sp);
+            const uint2 b = ld_nc_v2(sq);
+            ck.s[0][0] = a.x; ck.s[0][1] = a.y;
+            ck.s[1][0] = b.x; ck.s[1][1] = b.y;
+        } else {
+            uint32_t v0[8], v1[8];
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                v0[b] = b < nb ? ld_nc_u8(sp + b) : 0u;
+                v1[b] = b < nb ? ld_nc_u8(sq + b) : 0u;
+            }
+            ck.s[0][0] = v0[0] | (v0[1] << 8) | (v0[2] << 16) | (v0[3] << 24);
+            ck.s[0][1] = v0[4] | (v0[5] << 8) | (v0[6] << 16) | (v0[7] << 24);
+            ck.s[1][0] = v1[0] | (v1[1] << 8) | (v1[2] << 16) | (v1[3] << 24);
+            ck.s[1][1] = v1[4] | (v1[5] << 8) | (v1[6] << 16) | (v1[7] << 24);
         }
     }
-#pragma unroll 2
-    for (int b = 0; b < NBC; ++b) {
-        if (FULL || b < nbc) {
-            float sa, sb;
-            if (vec) {
-                if constexpr (FMT == FMT_NF4) {
-                    const int i = b & 3;
-                    sa = i == 0 ? va4.x : i == 1 ? va4.y : i == 2 ? va4.z : va4.w;
-                    sb = i == 0 ? vb4.x : i == 1 ? vb4.y : i == 2 ? vb4.z : vb4.w;
-                } else {
-                    const uint32_t sh = 8u * (uint32_t)(b & 3);
-                    sa = e8m0_to_f32(((b < 4 ? va2.x : va2.y) >> sh) & 0xFFu);
-                    sb = e8m0_to_f32(((b < 4 ? vb2.x : vb2.y) >> sh) & 0xFFu);
-                }
-            } else {
-                if constexpr (FMT == FMT_NF4) {
-                    sa = reinterpret_cast<const float*>(ss)[ra * nbk + bg0 + b];
-                    sb = reinterpret_cast<const float*>(ss)[rb * nbk + bg0 + b];
-                } else {
-                    sa = e8m0_to_f32(ss[ra * nbk + bg0 + b]);
-                    sb = e8m0_to_f32(ss[rb * nbk + bg0 + b]);
-                }
-            }
-            // this lane's packed bytes of rows ra and rb: byte o of the row's 128-byte
-            // chunk sits in 16-byte piece (o/16) ^ (row%8) of the swizzled box row
-            const int o = b * (SB / 2) + t * BPL;
-            const int pc = o >> 4, po = o & 15;
-            const uint8_t* rp0 = st + ra * kBoxBytes + ((pc ^ (ra & 7)) << 4) + po;
-            const uint8_t* rp1 = st + rb * kBoxBytes + ((pc ^ (rb & 7)) << 4) + po;
-            uint32_t w0[BPL / 4], w1[BPL / 4];
-            if constexpr (BPL == 8) {
-                const uint2 u0 = *reinterpret_cast<const uint2*>(rp0);
-                const uint2 u1 = *reinterpret_cast<const uint2*>(rp1);
-                w0[0] = u0.x; w0[BPL / 4 - 1] = u0.y;
-                w1[0] = u1.x; w1[BPL / 4 - 1] = u1.y;
-            } else {
-                w0[0] = *reinterpret_cast<const uint32_t*>(rp0);
-                w1[0] = *reinterpret_cast<const uint32_t*>(rp1);
-            }
-            // row ra by the shared-memory table; row rb by the table too (NF4) or by
-            // byte permutes on register tables (MXFP4)
-            uint32_t d0[BPL], d1[BPL];
+}
+
+// fp32 value of block b's scale of one row from the chunk's raw scale words
+template <int SCL>
+__device__ __forceinline__ float scale_of(const uint32_t* s, int b) {
+    if constexpr (SCL == SC_F32) {
+        return __uint_as_float(s[b]);
+    } else if constexpr (SCL == SC_BF16) {
+        return __uint_as_float(((s[b >> 1] >> (16 * (b & 1))) & 0xFFFFu) << 16);
+    } else {
+        return e8m0_to_f32((s[b >> 2] >> (8 * (b & 3))) & 0xFFu);
+    }
+}
+
+// m16n8k16 with 16-bit operands of the activations' type, fp32 accumulate (no side
+// effects: the compiler may interleave the chains of different blocks)
+template <int XH>
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    if constexpr (XH == 0) {
+        asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+            "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    } else {
+        asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+            "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    }
+}
+
+// one table lookup: a byte permute assembles the address from the lane's selector
+// word (lane * 4 in byte 0, the table's 64 KB-aligned base in bytes 2..3) and packed
+// byte i of w (byte 1). Not volatile, so the compiler may schedule it freely; it
+// cannot rise above the table fill because lane_sel is produced after the barrier
+// that follows the fill.
+__device__ __forceinline__ uint32_t lut_lookup(uint32_t w, uint32_t lane_sel, int i) {
+    const uint32_t a = prmt(w, lane_sel, 0x7604u | ((uint32_t)i << 4));
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds_v2(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+
+// The MMAs of one chunk for one warp: rows g / g+8 of the warp's 16 rows against NGC
+// groups of 8 routed rows; acc[j] += blocksum * scale per block. The packed bytes
+// come from the stage: rowa is row ra = 16w + g of the 128B-swizzled box, woff[b] the
+// lane's byte offset of block b inside a row. xp[j] points at this lane's first
+// activation of the chunk (or is null: zeros). FULL: every block of the chunk exists.
+template <int FMT, int SCL, int XH, int NGC, int NG, bool FULL>
+__device__ __forceinline__ void chunk_math(uint32_t rowa, const uint32_t (&woff)[ChunkGeom<FMT>::NB],
+                                           const Scales<SCL>& sc, uint32_t lane_sel,
+                                           const uint16_t* const (&xp)[NG], int nb, float (&acc)[NG][4]) {
+    using G = ChunkGeom<FMT>;
+    constexpr int XW = G::SB / 8;               // x words of one lane per block (8 or 4)
+    constexpr int STEPS = G::SB / 16;           // k16 steps per block (4 or 2)
+    // every packed word of the lane for the chunk, rows ra and ra + 8
+    uint32_t w[2][G::NB * G::LW];
+    const uint32_t rowb = rowa + 8 * kBoxBytes;
 #pragma unroll
-            for (int j = 0; j < BPL; ++j) {
-                const uint32_t sel = 0x5504u | ((uint32_t)(j & 3) << 4);
-                d0[j] = *reinterpret_cast<const uint32_t*>(lut + prmt(w0[j >> 2], lane_sel, sel));
-                if constexpr (FMT == FMT_NF4)
-                    d1[j] = *reinterpret_cast<const uint32_t*>(lut + prmt(w1[j >> 2], lane_sel, sel));
-            }
-            if constexpr (FMT == FMT_MXFP4) {
+    for (int b = 0; b < G::NB; ++b) {
+        if constexpr (G::LW == 2) {
+            const uint2 va = lds_v2(rowa + woff[b]), vb = lds_v2(rowb + woff[b]);
+            w[0][2 * b] = va.x; w[0][2 * b + 1] = va.y;
+            w[1][2 * b] = vb.x; w[1][2 * b + 1] = vb.y;
+        } else {
+            w[0][b] = lds_u32(rowa + woff[b]);
+            w[1][b] = lds_u32(rowb + woff[b]);
+        }
+    }
 #pragma unroll
-                for (int q = 0; q < BPL / 4; ++q) {
-                    uint32_t o4[4];
-                    decode_word<FMT>(w1[q], L, o4);
-                    d1[4 * q] = o4[0]; d1[4 * q + 1] = o4[1]; d1[4 * q + 2] = o4[2]; d1[4 * q + 3] = o4[3];
-                }
-            }
+    for (int b = 0; b < G::NB; ++b) {
+        if (FULL || b < nb) {
+            uint32_t xw[NGC][XW];
 #pragma unroll
-            for (int j = 0; j < NG; ++j) {
-                // activations of routed row 8j + g of the pass, from global memory (L1);
-                // lanes past the pass's rows feed zeros to output columns never stored
-                uint32_t xw[XW];
+            for (int j = 0; j < NGC; ++j) {
+                if (xp[j] != nullptr) {
+                    const uint4* src = reinterpret_cast<const uint4*>(xp[j] + b * G::SB);
 #pragma unroll
-                for (int w = 0; w < XW; ++w) xw[w] = 0u;
-                const uint16_t* xr = (j == 0) ? xr0 : xr1;
-                if (xr != nullptr) {
-                    const uint4* xs = reinterpret_cast<const uint4*>(xr + kc * kChunkK + b * SB + t * (SB / 4));
-#pragma unroll
-                    for (int w = 0; w < XW / 4; ++w) {
-                        const uint4 v = __ldg(xs + w);
-                        xw[4 * w] = v.x; xw[4 * w + 1] = v.y; xw[4 * w + 2] = v.z; xw[4 * w + 3] = v.w;
+                    for (int q = 0; q < XW / 4; ++q) {
+                        const uint4 v = __ldg(src + q);
+                        xw[j][4 * q] = v.x; xw[j][4 * q + 1] = v.y; xw[j][4 * q + 2] = v.z; xw[j][4 * q + 3] = v.w;
                     }
-                }
-                // two independent MMA chains per block (first and second half of its steps)
-                float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+                } else {
 #pragma unroll
-                for (int s = 0; s < STEPS; ++s) {
-                    if (s < STEPS / 2)
-                        mma_bf16_16816(c0, d0[2 * s], d1[2 * s], d0[2 * s + 1], d1[2 * s + 1], xw[2 * s], xw[2 * s + 1]);
-                    else
-                        mma_bf16_16816(c1, d0[2 * s], d1[2 * s], d0[2 * s + 1], d1[2 * s + 1], xw[2 * s], xw[2 * s + 1]);
+                    for (int q = 0; q < XW; ++q) xw[j][q] = 0u;
                 }
-                acc[j][0] = fmaf(c0[0] + c1[0], sa, acc[j][0]);
-                acc[j][1] = fmaf(c0[1] + c1[1], sa, acc[j][1]);
-                acc[j][2] = fmaf(c0[2] + c1[2], sb, acc[j][2]);
-                acc[j][3] = fmaf(c0[3] + c1[3], sb, acc[j][3]);
+            }
+            // decode: byte i of the lane's bytes -> one 16-bit pair (lower K first)
+            uint32_t da[G::LB], dbv[G::LB];
+#pragma unroll
+            for (int i = 0; i < G::LB; ++i) {
+                da[i] = lut_lookup(w[0][G::LW * b + (i >> 2)], lane_sel, i & 3);
+                dbv[i] = lut_lookup(w[1][G::LW * b + (i >> 2)], lane_sel, i & 3);
+            }
+            const float sa = scale_of<SCL>(sc.s[0], b);
+            const float sb = scale_of<SCL>(sc.s[1], b);
+#pragma unroll
+            for (int j = 0; j < NGC; ++j) {
+                // one MMA chain per block and group, the same for every group count, so a
+                // row's sum never depends on how many groups share its pass
+                float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int s = 0; s < STEPS; ++s)
+                    mma16816<XH>(c, da[2 * s], dbv[2 * s], da[2 * s + 1], dbv[2 * s + 1], xw[j][2 * s], xw[j][2 * s + 1]);
+                acc[j][0] = fmaf(c[0], sa, acc[j][0]);
+                acc[j][1] = fmaf(c[1], sa, acc[j][1]);
+                acc[j][2] = fmaf(c[2], sb, acc[j][2]);
+                acc[j][3] = fmaf(c[3], sb, acc[j][3]);
             }
         }
     }
+}
+
+template <int XH>
+__device__ __forceinline__ uint16_t to_out16(float v) {
+    if constexpr (XH == 0) return f32_to_bf16_rne(v);
+    else return __half_as_ushort(__float2half_rn(v));
+}
+
+// bytes of the shared memory other than the table and the rings: barriers and abort
+// flag, expert tables, scan scratch, row table (16-byte multiple)
+__host__ __device__ constexpr uint32_t other_bytes(int E) {
+    return (uint32_t)(((2 * kQuads * kStages * 8 + 16 + 8ull * (E + 1) + 8ull * E + 8ull * kWarps + 4ull * E +
+                        4ull * E + 4ull * kWarps + 12ull * kMaxTableRows) + 15) & ~15ull);
+}
+
+// Where the rings and the rest go, given the window address of the dynamic shared
+// memory: the table on the first 64 KB boundary; the rings (1024-aligned) after the
+// table if they fit, else before it; the rest in whichever gap is left. Returns false
+// if nothing fits (the host sizes the launch so that it does).
+struct Layout {
+    uint32_t lut, ring, other;
+};
+__host__ __device__ inline bool make_layout(uint32_t base, uint32_t bytes, int E, Layout& L) {
+    const uint32_t end = base + bytes;
+    const uint32_t lut = (base + 0xFFFFu) & ~0xFFFFu;
+    const uint32_t rb = kQuads * kStages * kStageBytes, ob = other_bytes(E);
+    if (lut + kLutBytes > end) return false;
+    uint32_t lo = base, hi = lut + kLutBytes;         // free space: [lo, lut) and [hi, end)
+    uint32_t ring;
+    if (hi + rb <= end) {
+        ring = hi;
+        hi += rb;
+    } else {
+        ring = (lo + 1023u) & ~1023u;
+        if (ring + rb > lut) return false;
+        lo = ring + rb;
+    }
+    uint32_t other;
+    if (lo + ob <= lut) other = lo;
+    else if (hi + ob <= end) other = hi;
+    else return false;
+    L.lut = lut;
+    L.ring = ring;
+    L.other = other;
+    return true;
+}
+
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    return mbar_wait_bounded(bar, parity, abort_flag, &g_decode_error, 1u);
 }
 
 }  // namespace db
 
-template <int FMT, int GMAX>
-__global__ void __launch_bounds__(db::kRegBound, 1)
-decode_band_kernel(const GroupedArgs p, const db::Plan plan, const __grid_constant__ CUtensorMap wmap) {
+template <int FMT, int SCL, int XH, int NG>
+__global__ void __launch_bounds__(db::kThreads, 1)
+decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant__ CUtensorMap wmap) {
     using namespace db;
-    constexpr int SB = (FMT == FMT_NF4) ? 64 : 32;   // K elements per scale block
+    using G = ChunkGeom<FMT>;
+    constexpr int SSZ = (SCL == SC_F32) ? 4 : (SCL == SC_BF16) ? 2 : 1;   // bytes per scale
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // [lut (+ partial-sum slots in its holes)][ring: stages x stage_bytes][scale slots][barriers]
-    // [abort, count, warp counts, tags][experts][row table]
-    uint8_t* lut = smem;                                            // [256][64] words
-    uint8_t* ring = smem + kLutBytes;                               // 1024-aligned stages
-    uint8_t* sslots = ring + plan.nstages * plan.stage_bytes;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sslots + plan.nslots * plan.scale_bytes);
-    // full[ns], empty[ns], scale slot free[nslots], scale slot full[nslots],
-    // partials ready[2][kMaxRowTiles], partial slots free[2][kMaxRowTiles]
-    int* tailw = reinterpret_cast<int*>(bars + 2 * plan.nstages + 2 * plan.nslots + 4 * kMaxRowTiles);
-    volatile int* abort_flag = tailw;
-    int* s_wcnt = tailw + 8;                                       // [16] active experts per warp (scan)
-    int* tags = tailw + 24;                                        // [ns] chunk counter last issued per slot
-    int64_t* s_r0 = reinterpret_cast<int64_t*>(tailw + 24 + ((plan.nstages + 1) & ~1)); // [E] first routed row
-    int* s_active = reinterpret_cast<int*>(s_r0 + p.E);            // [E] expert id
-    int* s_cnt = s_active + p.E;                                   // [E] routed rows
-    int* t_tok = s_cnt + p.E;                                      // [kMaxTableRows] per routed row
+    const uint32_t smem_s = smem_addr(smem_raw);
+    Layout lay;
+    if (!make_layout(smem_s, (uint32_t)pl.smem_bytes, p.E, lay)) {
+        if (threadIdx.x == 0) atomicOr(&g_decode_error, 0x100u);
+        return;
+    }
+    uint8_t* lut = smem_raw + (lay.lut - smem_s);
+    const uint32_t ring_s = lay.ring;
+    uint8_t* other = smem_raw + (lay.other - smem_s);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(other);            // full[kQuads][kStages], empty[..]
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * kQuads * kStages);
+    int64_t* s_up = reinterpret_cast<int64_t*>(other + 2 * kQuads * kStages * 8 + 16);
+    int64_t* s_r0 = s_up + (p.E + 1);
+    int64_t* s_wu = s_r0 + p.E;                     // [kWarps] scan scratch
+    int* s_e = reinterpret_cast<int*>(s_wu + kWarps);
+    int* s_m = s_e + p.E;
+    int* s_wc = s_m + p.E;                          // [kWarps]
+    int* t_tok = s_wc + kWarps;
     float* t_wt = reinterpret_cast<float*>(t_tok + kMaxTableRows);
     int* t_dst = reinterpret_cast<int*>(t_wt + kMaxTableRows);
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ns = plan.nstages, nsl = plan.nslots;
-    const int ROWS = plan.rows;
-    const int nrt = ROWS / 16, nks = kConsumers / nrt;
-    uint64_t* full = bars;
-    uint64_t* empty = bars + ns;
-    uint64_t* sfree = bars + 2 * ns;
-    uint64_t* sfull = bars + 2 * ns + nsl;
-    uint64_t* rready = bars + 2 * ns + 2 * nsl;                   // [buffer * kMaxRowTiles + rt]
-    uint64_t* rfree = rready + 2 * kMaxRowTiles;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int quad = warp >> 2, wq = warp & 3;       // quad, warp within the quad (its 16 rows)
+    const int ntile = (p.N + kTileRows - 1) / kTileRows;
 
-    if (warp == kProducerWarp && lane == 0) {
-        for (int i = 0; i < ns; ++i) {
-            mbar_init(smem_addr(full + i), 1);       // producer + tx bytes
-            mbar_init(smem_addr(empty + i), nrt);    // the warps that own the chunk
+    if (tid == 0) {
+        for (int i = 0; i < kQuads * kStages; ++i) {
+            mbar_init(smem_addr(bars + i), 1);                               // full: issuing lane + bytes
+            mbar_init(smem_addr(bars + kQuads * kStages + i), 4);            // empty: the quad's warps
         }
-        for (int i = 0; i < nsl; ++i) {
-            mbar_init(smem_addr(sfree + i), kConsumers);
-            mbar_init(smem_addr(sfull + i), 1);
-        }
-        for (int i = 0; i < 2 * kMaxRowTiles; ++i) {
-            mbar_init(smem_addr(rready + i), nks);   // the K-split warps of the row tile
-            mbar_init(smem_addr(rfree + i), 1);      // the epilogue warp
-        }
-        for (int i = 0; i < ns; ++i) tags[i] = -1;
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap)) : "memory");
     }
-    // experts of this band, in id order (every CTA derives the same list): one
-    // expert per thread, a ballot per warp, a prefix over the warps
+
+    // ---- active experts of this band and their unit counts (every CTA derives the same list) ----
     int nact = 0;
+    int64_t utot = 0;
     for (int e0 = 0; e0 < p.E; e0 += kThreads) {
-        const int e = e0 + (int)threadIdx.x;
-        bool act = false;
-        int64_t o0 = 0, o1 = 0;
+        const int e = e0 + tid;
+        int act = 0, m = 0;
+        int64_t o0 = 0, u = 0;
         if (e < p.E) {
             o0 = p.offsets[e];
-            o1 = p.offsets[e + 1];
-            act = (o1 - o0 >= p.m_lo) && (o1 - o0 <= p.m_hi);
+            m = (int)(p.offsets[e + 1] - o0);
+            act = (m >= p.m_lo && m <= p.m_hi) ? 1 : 0;
+            if (act) u = (int64_t)ntile * ((m + 8 * NG - 1) / (8 * NG));
         }
-        const unsigned bal = __ballot_sync(0xffffffffu, act);
-        if (lane == 0) s_wcnt[warp] = __popc(bal);
-        __syncthreads();
-        int before = nact, total = 0;
-        for (int w = 0; w < kThreads / 32; ++w) {
-            const int c = s_wcnt[w];
-            if (w < warp) before += c;
-            total += c;
-        }
-        if (act) {
-            const int idx = before + __popc(bal & ((1u << lane) - 1u));
-            s_active[idx] = e;
-            s_r0[idx] = o0;
-            s_cnt[idx] = (int)(o1 - o0);
-        }
-        nact += total;
-        __syncthreads();
-    }
-
-    const int nit = (p.N + ROWS - 1) / ROWS;           // items per expert
-    const int total = nact * nit;
-    const int i0 = (int)((int64_t)blockIdx.x * total / gridDim.x);
-    const int i1 = (int)((int64_t)(blockIdx.x + 1) * total / gridDim.x);
-    const int nbk = p.K / SB;                          // scale blocks per weight row
-    const int ssz = FMT == FMT_NF4 ? 4 : 1;
-
-    // routed rows of this CTA's experts: one contiguous range [rlo, rhi)
-    int64_t rlo = 0, rhi = 0;
-    if (i0 < i1) {
-        const int a0 = i0 / nit, a1 = (i1 - 1) / nit;
-        rlo = s_r0[a0];
-        rhi = s_r0[a1] + s_cnt[a1];
-    }
-    const bool table = (rhi - rlo) <= kMaxTableRows;
-
-    const int nch = plan.nch;
-    if (warp == kProducerWarp) {
-        // ================= producer (one thread): starts right away =================
-        if (lane == 0) {
-            uint32_t ctr = 0, slot = 0, ph = 1;       // ring position; empty-barrier parity to wait on
-            uint32_t sslot = 0, sph = 1;              // next scale slot to fill; its free-barrier parity
-            int sa_ = (i1 > i0) ? i0 / nit : 0, sit = (i1 > i0) ? i0 % nit : 0;   // next item whose scales go out
-            int s_next = i0;
-            int a = sa_, it = sit;
-            bool ok = true;
-            for (int item = i0; item < i1 && ok; ++item) {
-                // scales go out one item ahead: those of this item and of the next
-                while (s_next < i1 && s_next <= item + 1) {
-                    // an item's scales: its rows x all blocks, one contiguous range (a multiple of 16 bytes)
-                    if (!mbar_wait_bounded(smem_addr(sfree + sslot), sph, abort_flag, &g_decode_error, 4u)) {
-                        ok = false;
-                        break;
-                    }
-                    const int se = s_active[sa_];
-                    const int sn0 = sit * ROWS;
-                    const uint32_t sbytes = (uint32_t)(min(ROWS, p.N - sn0) * nbk * ssz);
-                    const uint8_t* ssrc = reinterpret_cast<const uint8_t*>(p.scales) + ((int64_t)se * p.N + sn0) * nbk * ssz;
-                    const uint32_t sb = smem_addr(sfull + sslot);
-                    mbar_arrive_tx(sb, sbytes);
-                    bulk_1d(smem_addr(sslots + sslot * plan.scale_bytes), ssrc, sbytes, sb);
-                    if (++sslot == (uint32_t)nsl) {
-                        sslot = 0;
-                        sph ^= 1u;
-                    }
-                    if (++sit == nit) {
-                        sit = 0;
-                        ++sa_;
-                    }
-                    ++s_next;
-                }
-                const int e = s_active[a];
-                const int n0 = it * ROWS;
-                const int npass = (s_cnt[a] + 8 * GMAX - 1) / (8 * GMAX);
-                for (int pass = 0; pass < npass && ok; ++pass) {
-                    for (int kc = 0; kc < nch; ++kc) {
-                        if (!mbar_wait_bounded(smem_addr(empty + slot), ph, abort_flag, &g_decode_error, 1u)) {
-                            ok = false;
-                            break;
-                        }
-                        // the slot's previous chunk is consumed: name the chunk it now receives
-                        asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_addr(tags + slot)), "r"(ctr)
-                                     : "memory");
-                        const uint32_t fb = smem_addr(full + slot);
-                        mbar_arrive_tx(fb, (uint32_t)(kBoxBytes * ROWS));
-                        tma_2d(smem_addr(ring + slot * plan.stage_bytes), &wmap, kc * (kChunkK / 2), e * p.N + n0, fb);
-                        ++ctr;
-                        if (++slot == (uint32_t)ns) {
-                            slot = 0;
-                            ph ^= 1u;
-                        }
-                    }
-                }
-                if (++it == nit) {
-                    it = 0;
-                    ++a;
-                }
+        int ca = act;
+        int64_t cu = u;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int ya = __shfl_up_sync(0xffffffffu, ca, d);
+            const int64_t yu = __shfl_up_sync(0xffffffffu, cu, d);
+            if (lane >= d) {
+                ca += ya;
+                cu += yu;
             }
         }
-        __syncwarp();
-        return;
+        if (lane == 31) {
+            s_wc[warp] = ca;
+            s_wu[warp] = cu;
+        }
+        __syncthreads();
+        int pa = nact, ta = 0;
+        int64_t pu = utot, tu = 0;
+        for (int w = 0; w < kWarps; ++w) {
+            const int c = s_wc[w];
+            const int64_t cw = s_wu[w];
+            if (w < warp) {
+                pa += c;
+                pu += cw;
+            }
+            ta += c;
+            tu += cw;
+        }
+        if (act) {
+            const int idx = pa + ca - 1;
+            s_e[idx] = e;
+            s_m[idx] = m;
+            s_r0[idx] = o0;
+            s_up[idx] = pu + cu - u;
+        }
+        nact += ta;
+        utot += tu;
+        __syncthreads();
+    }
+    const int64_t U0 = (int64_t)blockIdx.x * utot / gridDim.x;
+    const int64_t U1 = (int64_t)(blockIdx.x + 1) * utot / gridDim.x;
+    if (U0 >= U1) return;                            // whole CTA: no unit (no copy was issued)
+    if (tid == 0) s_up[nact] = utot;
+    __syncthreads();
+
+    // ---- this quad's units and K part ----
+    const int np = pl.np, ngroups = kQuads / np;
+    const int gi = quad / np, part = quad - gi * np;
+    const int c_lo = part * pl.nc / np, c_hi = (part + 1) * pl.nc / np;
+    const int nck = c_hi - c_lo;
+    const int nunit = (U1 - U0 > gi) ? (int)((U1 - U0 - gi + ngroups - 1) / ngroups) : 0;
+    const int nsteps = nunit * nck;
+    const int64_t s8 = 8 * (int64_t)pl.nblk * SSZ;
+    const bool vec = pl.vec_scales != 0;
+    const uint8_t* Sb = reinterpret_cast<const uint8_t*>(p.scales);
+    const bool issuer = (wq == 0 && lane == 0);     // issues the quad's copies
+    uint64_t* full = bars + quad * kStages;
+    uint64_t* empty = bars + kQuads * kStages + quad * kStages;
+    const uint32_t qring = ring_s + (uint32_t)(quad * kStages * kStageBytes);
+
+    // unit u -> (active expert a, first weight row n0, first routed row of the pass mc);
+    // a only moves forward along a quad's units, so it is found by walking
+    auto locate = [&](int64_t u, int& a, int& n0, int& mc) {
+        while (s_up[a + 1] <= u) ++a;
+        const int m = s_m[a];
+        const int npass = (m + 8 * NG - 1) / (8 * NG);
+        const int local = (int)(u - s_up[a]);
+        int tile = local, pass = 0;
+        if (npass > 1) {
+            tile = local / npass;
+            pass = local - tile * npass;
+        }
+        n0 = tile * kTileRows;
+        mc = pass * 8 * NG;
+    };
+
+    // copy cursor (issuing lane only): chunk j of the quad's sequence into stage j % kStages
+    int cp_left = nsteps, cp_c = c_lo, cp_a = 0, cp_y = 0, cp_j = 0, cp_s = 0;
+    int64_t cp_u = U0 + gi;
+    auto cp_unit = [&]() {
+        int n0, mc;
+        locate(cp_u, cp_a, n0, mc);
+        cp_y = s_e[cp_a] * p.N + n0;
+        cp_c = c_lo;
+    };
+    auto issue_next = [&]() {
+        const uint32_t fb = smem_addr(full + cp_s);
+        mbar_arrive_tx(fb, (uint32_t)kStageBytes);
+        tma_2d(qring + (uint32_t)cp_s * kStageBytes, &wmap, cp_c * kBoxBytes, cp_y, fb);
+        if (++cp_s == kStages) cp_s = 0;
+        ++cp_j;
+        --cp_left;
+        if (++cp_c == c_hi && cp_left > 0) {
+            cp_u += ngroups;
+            cp_unit();
+        }
+    };
+    if (issuer && nsteps > 0) {
+        cp_unit();
+        for (int j = 0; j < kStages && cp_left > 0; ++j) issue_next();
     }
 
-    // consumers and the epilogue warp, while the producer's first copies are in flight:
-    // the byte -> bf16x2 table (one copy per lane: 8 sixteen-byte pieces per byte value)
-    // and the routing metadata of the CTA's rows
-    if (threadIdx.x < kConsumers * 32) {
-        const LutPlanes Lt = p.lut;
-        for (int i = threadIdx.x; i < 256 * 8; i += kConsumers * 32) {
+    // scale cursor (every warp, its own rows): one chunk ahead of the math
+    int sc_left = nsteps, sc_c = c_lo, sc_a = 0;
+    int64_t sc_u = U0 + gi;
+    const uint8_t* sc_p = nullptr;
+    auto sc_unit = [&]() {
+        int n0, mc;
+        locate(sc_u, sc_a, n0, mc);
+        // rows past N (a short last tile) read row 0 of the expert instead: in bounds, unused
+        const int rr = (n0 + 16 * wq < p.N) ? n0 + 16 * wq + g : g;
+        const int64_t row = (int64_t)s_e[sc_a] * p.N + rr;
+        sc_p = Sb + (row * pl.nblk + (int64_t)c_lo * G::NB) * SSZ;
+        sc_c = c_lo;
+    };
+    auto scales_next = [&](Scales<SCL>& sc) {
+        if (sc_left <= 0) return;
+        load_scales<SCL>(sc, sc_p, s8, min(G::NB, pl.nblk - sc_c * G::NB), vec);
+        --sc_left;
+        sc_p += G::NB * SSZ;
+        if (++sc_c == c_hi && sc_left > 0) {
+            sc_u += ngroups;
+            sc_unit();
+        }
+    };
+    Scales<SCL> scN;                                 // the next chunk's scales
+    if (nsteps > 0) {
+        sc_unit();
+        scales_next(scN);
+    }
+
+    // ---- lookup table and the CTA's routing metadata, while the first copies fly ----
+    {
+        const LutPlanes L = p.lut;
+        for (int i = tid; i < 256 * 8; i += kThreads) {
             const int b = i >> 3, q = i & 7;
-            const uint32_t v = byte_bf16x2<FMT>((uint32_t)b, Lt);
+            const uint32_t v = byte_bf16x2<FMT>((uint32_t)b, L);
             *reinterpret_cast<uint4*>(lut + b * 256 + q * 16) = make_uint4(v, v, v, v);
         }
     }
-    if (table) {
-        for (int64_t r = rlo + threadIdx.x; r < rhi; r += kConsumers * 32)
-            if (threadIdx.x < kConsumers * 32) {
+    int64_t rlo = 0;
+    bool table = false;
+    {
+        int a0 = 0, a1 = 0, n0, mc;
+        locate(U0, a0, n0, mc);
+        locate(U1 - 1, a1, n0, mc);
+        rlo = s_r0[a0];
+        const int64_t rhi = s_r0[a1] + s_m[a1];
+        table = (rhi - rlo) <= kMaxTableRows;
+        if (table) {
+            for (int64_t r = rlo + tid; r < rhi; r += kThreads) {
                 const int k = (int)(r - rlo);
                 t_tok[k] = p.row_token ? __ldg(p.row_token + r) : (int)r;
                 t_wt[k] = p.row_weight ? __ldg(p.row_weight + r) : 1.f;
                 t_dst[k] = p.row_dest ? __ldg(p.row_dest + r) : (int)r;
             }
+        }
     }
-    asm volatile("bar.sync 1, %0;" ::"r"((kConsumers + 1) * 32) : "memory");
+    __syncthreads();
 
-    if (warp == kEpilogueWarp) {
-        // ================= epilogue: fixed-order K-split sums, weight, bf16, scatter =================
-        bool dead = false;
-        uint32_t P = 0;                                 // pass counter of the CTA
-        int a = (i1 > i0) ? i0 / nit : 0, it = (i1 > i0) ? i0 % nit : 0;
-        for (int item = i0; item < i1; ++item) {
-            const int m = s_cnt[a];
-            const int n0 = it * ROWS;
-            const int64_t r0 = s_r0[a];
-            const int npass = (m + 8 * GMAX - 1) / (8 * GMAX);
-            const int vrows = min(ROWS, p.N - n0);
-            for (int pass = 0; pass < npass; ++pass, ++P) {
-                const int mc = pass * 8 * GMAX;
-                const int nvalid = min(8 * GMAX, m - mc);
-                const int G = (nvalid + 7) >> 3;
-                const uint32_t buf = P & 1u, ph = (P >> 1) & 1u;
-                for (int rt = 0; rt < nrt; ++rt) {
-                    const int bi = (int)buf * kMaxRowTiles + rt;
-                    if (!dead && !mbar_wait_bounded(smem_addr(rready + bi), ph, abort_flag, &g_decode_error, 32u))
-                        dead = true;
-                    if (!dead) {
-                        for (int q = lane; q < G * 32; q += 32) {
-                            const int j = q >> 5, ln = q & 31;
-                            float4 v = *red_slot(lut, (((int)buf * nrt + rt) * nks + 0) * GMAX + j, ln);
-                            for (int k2 = 1; k2 < nks; ++k2) {
-                                const float4 w = *red_slot(lut, (((int)buf * nrt + rt) * nks + k2) * GMAX + j, ln);
-                                v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
-                            }
-                            const float vv[4] = {v.x, v.y, v.z, v.w};
+    // selector word of this lane's table lookups, made after the barrier (the volatile
+    // move keeps every lookup, which depends on it, below the table fill)
+    uint32_t lane_sel;
+    asm volatile("mov.b32 %0, %1;" : "=r"(lane_sel) : "r"((lay.lut & 0xFFFF0000u) | ((uint32_t)lane << 2)) : "memory");
+    auto tok_of = [&](int64_t r) -> int {
+        return table ? t_tok[r - rlo] : (p.row_token ? __ldg(p.row_token + r) : (int)r);
+    };
+    auto wt_of = [&](int64_t r) -> float {
+        return table ? t_wt[r - rlo] : (p.row_weight ? __ldg(p.row_weight + r) : 1.f);
+    };
+    auto dst_of = [&](int64_t r) -> int64_t {
+        return table ? (int64_t)t_dst[r - rlo] : (p.row_dest ? (int64_t)__ldg(p.row_dest + r) : r);
+    };
+    uint16_t* out = p.out;
+    // part sums of one lane: 16-byte slot s in the unused halves of the table's rows
+    auto slot_ptr = [&](int s) -> float4* {
+        return reinterpret_cast<float4*>(lut + (s >> 3) * 256 + 128 + (s & 7) * 16);
+    };
+
+    // ---- math cursor ----
+    int mt_ck = 0, mt_a = 0, mt_n0 = 0, mt_mc = 0, mt_unit = 0, nvalid = 0, ng = 0;
+    int64_t mt_u = U0 + gi, mt_r0 = 0;
+    bool rows_ok = false;                           // this warp's 16 rows exist (n0 + 16 wq < N)
+    float acc[NG][4];
+    const uint16_t* xp[NG];
+    bool dead = false;
+
+    auto unit_begin = [&]() {
+        locate(mt_u, mt_a, mt_n0, mt_mc);
+        mt_r0 = s_r0[mt_a];
+        nvalid = min(8 * NG, s_m[mt_a] - mt_mc);
+        ng = (nvalid + 7) >> 3;
+        rows_ok = mt_n0 + 16 * wq < p.N;
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const int row = mc + 8 * j + 2 * (ln & 3) + (i & 1);       // C column 2t (+1)
-                                const int nr = rt * 16 + (ln >> 2) + ((i & 2) ? 8 : 0);    // C row g (+8)
-                                if (row < m && nr < vrows) {
-                                    const int64_t r = r0 + row;
-                                    float wgt;
-                                    int64_t dst;
-                                    if (table) {
-                                        wgt = t_wt[r - rlo];
-                                        dst = t_dst[r - rlo];
-                                    } else {
-                                        wgt = p.row_weight ? __ldg(p.row_weight + r) : 1.f;
-                                        dst = p.row_dest ? (int64_t)__ldg(p.row_dest + r) : r;
-                                    }
-                                    p.out[dst * p.N + n0 + nr] = f32_to_bf16_rne(vv[i] * wgt);
-                                }
-                            }
-                        }
-                    }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_addr(rfree + bi));
-                }
-            }
-            if (++it == nit) {
-                it = 0;
-                ++a;
+        for (int j = 0; j < NG; ++j) {
+            xp[j] = nullptr;
+            const int jr = 8 * j + g;
+            if (jr < nvalid)
+                xp[j] = p.x + (int64_t)tok_of(mt_r0 + mt_mc + jr) * p.K + c_lo * kChunkK + t * (G::SB / 4);
+            acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+        }
+    };
+    // store one lane's four sums (rows n0 + 16 wq + lg and + 8; routed columns 2 lt, 2 lt + 1 of group grp)
+    auto store4 = [&](const float4& v, int lg, int lt, int grp) {
+        const int n_a = mt_n0 + 16 * wq + lg, n_b = n_a + 8;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int jc = 8 * grp + 2 * lt + h;
+            if (jc < nvalid) {
+                const int64_t r = mt_r0 + mt_mc + jc;
+                const float w = wt_of(r);
+                const int64_t d = dst_of(r) * p.N;
+                out[d + n_a] = to_out16<XH>((h ? v.y : v.x) * w);
+                out[d + n_b] = to_out16<XH>((h ? v.w : v.z) * w);
             }
         }
-        return;
-    }
-
-    // ================= consumers =================
-    const int rt = warp % nrt, ks = warp / nrt;     // row tile, K split (chunks kc % nks == ks)
-    const int g = lane >> 2, t = lane & 3;
-    const int ra = rt * 16 + g, rb = ra + 8;        // the two item rows of this lane
-    const uint32_t lane_sel = (uint32_t)lane * 4u;  // lut offset of this lane's copy
-    const LutPlanes L = p.lut;                      // register tables for the permute decode
-    const bool vec_scales = (FMT == FMT_NF4) ? (nbk % 4 == 0) : (nbk % 8 == 0);
-    bool dead = false;   // set when a wait gives up: the warp then only keeps the barrier schedule
-    float acc[GMAX][4];
+    };
+    auto unit_end = [&]() {
+        if (np == 1) {
+            if (rows_ok && !dead) {
 #pragma unroll
-    for (int j = 0; j < GMAX; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-    uint32_t base = 0;                              // chunk counter at the start of the pass
-    uint32_t P = 0;                                 // pass counter of the CTA
-    uint32_t sslot = 0, sph = 0;                    // scale slot; its full-barrier parity
-    int a = (i1 > i0) ? i0 / nit : 0, it = (i1 > i0) ? i0 % nit : 0;
-    for (int item = i0; item < i1; ++item) {
-        const int m = s_cnt[a];
-        const int64_t r0 = s_r0[a];
-        const int npass = (m + 8 * GMAX - 1) / (8 * GMAX);
-        // every warp waits for the item's scales (also those that own no chunk of it)
-        if (!dead && !mbar_wait_bounded(smem_addr(sfull + sslot), sph, abort_flag, &g_decode_error, 8u))
-            dead = true;
-        const uint8_t* ss = sslots + sslot * plan.scale_bytes;
-        for (int pass = 0; pass < npass; ++pass, ++P) {
-            const int mc = pass * 8 * GMAX;
-            const int nvalid = min(8 * GMAX, m - mc);   // routed rows of this pass
-            // x rows of this lane's routed rows (8j + g of the pass), or null past the pass's end
-            const uint16_t* xr0 = nullptr;
-            const uint16_t* xr1 = nullptr;
-            if (g < nvalid) {
-                const int64_t r = r0 + mc + g;
-                const int tk = table ? t_tok[r - rlo] : (p.row_token ? __ldg(p.row_token + r) : (int)r);
-                xr0 = p.x + (int64_t)tk * p.K;
+                for (int j = 0; j < NG; ++j)
+                    if (j < ng) store4(make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]), g, t, j);
             }
-            if (GMAX == 2 && 8 + g < nvalid) {
-                const int64_t r = r0 + mc + 8 + g;
-                const int tk = table ? t_tok[r - rlo] : (p.row_token ? __ldg(p.row_token + r) : (int)r);
-                xr1 = p.x + (int64_t)tk * p.K;
-            }
-            int kc = ks;                                // chunks kc = ks, ks + nks, ...
-            uint32_t ctr = base + (uint32_t)kc;
-            uint32_t slot = ctr % (uint32_t)ns, ph = (ctr / (uint32_t)ns) & 1u;
-            for (; kc < nch; kc += nks) {
-                // bring this chunk's activations into L1 while the weights are on their way
-                // (lane t of row g: the t-th 128-byte line of the row's 512-byte chunk)
-                if (kc * kChunkK + t * 64 < p.K) {
-                    if (xr0 != nullptr) prefetch_l1(xr0 + kc * kChunkK + t * 64);
-                    if (xr1 != nullptr) prefetch_l1(xr1 + kc * kChunkK + t * 64);
-                }
-                if (!dead && !wait_tag(tags + slot, ctr, abort_flag, &g_decode_error, 16u)) dead = true;
-                if (!dead && !mbar_wait_bounded(smem_addr(full + slot), ph, abort_flag, &g_decode_error, 2u))
-                    dead = true;
-                if (!dead) {
-                    const uint8_t* st = ring + slot * plan.stage_bytes;
-                    const int kb = kc * kChunkK;
-                    if (p.K - kb >= kChunkK) {
-                        if (GMAX == 2 && nvalid > 8)
-                            chunk_mma<FMT, GMAX, (GMAX == 2 ? 2 : 1), true>(st, ss, lut, lane_sel, L, xr0, xr1, ra, rb, t, nbk, kc,
-                                                                            0, vec_scales, acc);
-                        else
-                            chunk_mma<FMT, GMAX, 1, true>(st, ss, lut, lane_sel, L, xr0, xr1, ra, rb, t, nbk, kc, 0, vec_scales,
-                                                          acc);
-                    } else {
-                        const int nbc = (p.K - kb) / SB;
-                        chunk_mma<FMT, GMAX, GMAX, false>(st, ss, lut, lane_sel, L, xr0, xr1, ra, rb, t, nbk, kc, nbc, vec_scales,
-                                                          acc);
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(empty + slot));
-                ctr += (uint32_t)nks;
-                slot += (uint32_t)nks;                      // nks <= ns: at most one wrap
-                if (slot >= (uint32_t)ns) {
-                    slot -= (uint32_t)ns;
-                    ph ^= 1u;
-                }
-            }
-            base += (uint32_t)nch;
-            // end of a pass: hand the partial sums to the epilogue warp
-            const uint32_t buf = P & 1u, fph = ((P >> 1) & 1u) ^ 1u;
-            const int bi = (int)buf * kMaxRowTiles + rt;
-            if (!dead && !mbar_wait_bounded(smem_addr(rfree + bi), fph, abort_flag, &g_decode_error, 64u))
-                dead = true;
-            if (!dead) {
-#pragma unroll
-                for (int j = 0; j < GMAX; ++j)
-                    *red_slot(lut, (((int)buf * nrt + rt) * nks + ks) * GMAX + j, lane) =
-                        make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(rready + bi));
-#pragma unroll
-            for (int j = 0; j < GMAX; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+            return;
         }
-        // every warp is done with this item's scales
+        // hand the part sums to the group (slot of parity, warp, group, lane), then
+        // reduce a share of this warp's rows in part order
+        const int par = mt_unit & 1;
+#pragma unroll
+        for (int j = 0; j < NG; ++j)
+            if (j < ng) *slot_ptr(((par * kWarps + warp) * NG + j) * 32 + lane) = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + gi), "r"(np * 128) : "memory");
+        const int ipw = (NG * 32) / np;             // items (one lane's float4 of one group) per warp
+        if (lane < ipw && rows_ok && !dead) {
+            const int q = part * ipw + lane;
+            const int src = q & 31, grp = q >> 5;
+            if (grp < ng) {
+                // warp wq of quad (gi * np + pp) holds part pp of these rows
+                float4 v = *slot_ptr(((par * kWarps + (gi * np) * 4 + wq) * NG + grp) * 32 + src);
+                for (int pp = 1; pp < np; ++pp) {
+                    const float4 w = *slot_ptr(((par * kWarps + (gi * np + pp) * 4 + wq) * NG + grp) * 32 + src);
+                    v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+                }
+                store4(v, src >> 2, src & 3, grp);
+            }
+        }
+    };
+
+    // this lane's byte offset of each block inside a 128-byte row of a stage (swizzled by g)
+    uint32_t woff[G::NB];
+#pragma unroll
+    for (int b = 0; b < G::NB; ++b)
+        woff[b] = (G::LW == 2) ? (((uint32_t)((2 * b + (t >> 1)) ^ g) << 4) + (uint32_t)(t & 1) * 8u)
+                               : (((uint32_t)(b ^ g) << 4) + (uint32_t)t * 4u);
+    const uint32_t lane_row = (uint32_t)(16 * wq + g) * kBoxBytes;
+    const int nfull = pl.nblk / G::NB;              // chunks with every block present
+    int cs = 0;                                     // stage of the current chunk
+    uint32_t cph = 0;                               // its full-barrier parity
+    int rs = 0;                                     // stage the issuing lane refills next
+    uint32_t rph = 0;                               // parity of that stage's release
+
+    auto step = [&]() {
+        const Scales<SCL> use = scN;                // this chunk's scales (loaded a step ago)
+        scales_next(scN);
+        if (mt_ck == 0) unit_begin();
+        if (!dead && !wait_bounded(smem_addr(full + cs), cph, abort_flag)) dead = true;
+        if (!dead && rows_ok) {
+            const int c = c_lo + mt_ck;
+            const uint32_t rowa = qring + (uint32_t)cs * kStageBytes + lane_row;
+            if (c < nfull) {
+                if (NG == 1 || ng == 1)
+                    chunk_math<FMT, SCL, XH, 1, NG, true>(rowa, woff, use, lane_sel, xp, G::NB, acc);
+                else
+                    chunk_math<FMT, SCL, XH, (NG > 1 ? 2 : 1), NG, true>(rowa, woff, use, lane_sel, xp, G::NB, acc);
+            } else {
+                const int nb = pl.nblk - c * G::NB;
+                if (NG == 1 || ng == 1)
+                    chunk_math<FMT, SCL, XH, 1, NG, false>(rowa, woff, use, lane_sel, xp, nb, acc);
+                else
+                    chunk_math<FMT, SCL, XH, (NG > 1 ? 2 : 1), NG, false>(rowa, woff, use, lane_sel, xp, nb, acc);
+            }
+        }
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_addr(sfree + sslot));
-        if (++sslot == (uint32_t)nsl) {
-            sslot = 0;
-            sph ^= 1u;
+        if (lane == 0) mbar_arrive(smem_addr(empty + cs));
+        if (++cs == kStages) {
+            cs = 0;
+            cph ^= 1u;
         }
-        if (++it == nit) {
-            it = 0;
-            ++a;
+        // the issuing lane refills the oldest stage once all four warps released it
+        // (the chunk kStages before the one it now receives)
+        if (issuer && cp_left > 0 && cp_j >= kStages) {
+            if (!dead && !wait_bounded(smem_addr(empty + rs), rph, abort_flag)) dead = true;
+            if (!dead) issue_next();
+            if (++rs == kStages) {
+                rs = 0;
+                rph ^= 1u;
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < NG; ++q)
+            if (xp[q] != nullptr) xp[q] += kChunkK;
+        if (++mt_ck == nck) {
+            unit_end();
+            mt_ck = 0;
+            ++mt_unit;
+            mt_u += ngroups;
+        }
+    };
+
+    for (int j = 0; j < nsteps; ++j) step();
+
+    // before the CTA exits: every copy this quad issued has landed. On the normal path
+    // the math already waited for all of them; after an abort this wait (bounded, and
+    // deaf to the abort flag) keeps the CTA's shared memory alive until they land.
+    if (issuer) {
+        for (int j = (cp_j > kStages ? cp_j - kStages : 0); j < cp_j; ++j) {
+            const uint32_t bar = smem_addr(full + j % kStages), par = (uint32_t)((j / kStages) & 1);
+            const long long t0 = clock64();
+            while (!mbar_try_wait(bar, par, 2000u))
+                if (clock64() - t0 > kWaitTimeoutCycles) {
+                    atomicOr(&g_decode_error, 2u);
+                    break;
+                }
         }
     }
+}
+
+static int pick_parts(int nc) {
+    // the largest power of two (at most GNF4_DB_MAXPARTS, at most nc) whose parts are
+    // within 15 % of even
+    for (int np = GNF4_DB_MAXPARTS; np > 1; np >>= 1) {
+        if (np > nc) continue;
+        const int per = (nc + np - 1) / np;
+        if (per * np * 100 <= nc * 115) return np;
+    }
+    return 1;
 }
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn_db() {
@@ -621,70 +783,74 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn_db() {
     return fn;
 }
 
-template <int FMT, int GMAX>
-static cudaError_t launch_db(const GroupedArgs& a, cudaStream_t s) {
-    using namespace db;
-    const int SB = (FMT == FMT_NF4) ? 64 : 32;
-    const int ssz = (FMT == FMT_NF4) ? 4 : 1;
-    Plan plan;
-    plan.nch = (a.K + kChunkK - 1) / kChunkK;
-    const int tables = 96 + 16 * a.E + 12 * kMaxTableRows;
-    int smem = 0;
-    plan.rows = 0;
-    for (int rows = 48; rows >= 16 && plan.rows == 0; rows -= 16) {
-        const int stage_bytes = rows * kBoxBytes;       // 6, 4 or 2 KB: multiples of 1024
-        const int scale_bytes = ((rows * (a.K / SB) * ssz + 127) / 128) * 128;
-        const int nks = kConsumers * 16 / rows;          // K-split warps per row tile: the ring holds at least one chunk each
-        for (int nst = 12; nst >= nks && plan.rows == 0; --nst) {
-            for (int nsl = 3; nsl >= 2; --nsl) {
-                const int need = 1024 + kLutBytes + nst * stage_bytes + nsl * scale_bytes +
-                                 (2 * nst + 2 * nsl + 4 * kMaxRowTiles) * 8 + 4 * ((nst + 1) & ~1) + tables;
-                if (need <= 226 * 1024) {
-                    plan.rows = rows;
-                    plan.stage_bytes = stage_bytes;
-                    plan.scale_bytes = scale_bytes;
-                    plan.nstages = nst;
-                    plan.nslots = nsl;
-                    smem = need;
-                    break;
-                }
-            }
-        }
+template <int FMT, int SCL, int XH, int NG>
+static cudaError_t launch_db(const GroupedArgs& a, db::Plan& pl, cudaStream_t s) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    // the dynamic shared memory starts after the per-block reserved bytes (this kernel
+    // has no static shared memory); size the launch so that the layout fits there
+    static int reserved[64] = {0};
+    static bool have_reserved[64] = {false};
+    if (!have_reserved[dev]) {
+        int r = 0;
+        if (cudaDeviceGetAttribute(&r, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess) r = 1024;
+        reserved[dev] = r;
+        have_reserved[dev] = true;
     }
-    if (plan.rows == 0) return cudaErrorInvalidValue;
-    static int smem_set = 0;                 // largest dynamic shared memory opted in so far
-    if (smem > smem_set) {
-        cudaError_t e = cudaFuncSetAttribute(decode_band_kernel<FMT, GMAX>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    db::Layout lay;
+    uint32_t bytes = 0;
+    for (uint32_t b = 64 * 1024; b <= (uint32_t)db::kMaxSmem; b += 1024)
+        if (db::make_layout((uint32_t)reserved[dev], b, a.E, lay)) {
+            bytes = b;
+            break;
+        }
+    if (bytes == 0) return cudaErrorInvalidConfiguration;
+    pl.smem_bytes = (int)bytes;
+    static bool attr_done[64] = {false};            // per device: dynamic shared memory opted in
+    if (!attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(decode_band_kernel<FMT, SCL, XH, NG>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, db::kMaxSmem);
         if (e != cudaSuccess) return e;
-        smem_set = smem;
+        attr_done[dev] = true;
     }
     auto enc = encode_fn_db();
     if (!enc) return cudaErrorNotSupported;
-    // packed weights as bytes [E*N, K/2]: boxes of 128 bytes x rows, 128B swizzle
+    // packed weights as bytes [E*N, K/2]: boxes of 128 bytes x 64 rows, 128B swizzle
     CUtensorMap wmap;
     cuuint64_t dims[2] = {(cuuint64_t)(a.K / 2), (cuuint64_t)a.E * (cuuint64_t)a.N};
     cuuint64_t strides[1] = {(cuuint64_t)(a.K / 2)};
-    cuuint32_t box[2] = {(cuuint32_t)kBoxBytes, (cuuint32_t)plan.rows};
+    cuuint32_t box[2] = {(cuuint32_t)db::kBoxBytes, (cuuint32_t)db::kTileRows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.W), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    const int64_t groups_max = a.R < (int64_t)a.E ? a.R : (int64_t)a.E;
-    const int64_t items_max = groups_max * ((a.N + plan.rows - 1) / plan.rows);
-    int64_t grid = device_sm_count();
-    if (items_max < grid) grid = items_max;
-    if (grid < 1) return cudaSuccess;
-    decode_band_kernel<FMT, GMAX><<<(unsigned)grid, kThreads, smem, s>>>(a, plan, wmap);
+    const int grid = device_sm_count();
+    decode_band_kernel<FMT, SCL, XH, NG><<<grid, db::kThreads, bytes, s>>>(a, pl, wmap);
     return cudaGetLastError();
 }
 
 cudaError_t launch_decode_band(int fmt, const GroupedArgs& a, cudaStream_t s) {
-    const int64_t mmax = a.R < (int64_t)a.m_hi ? a.R : (int64_t)a.m_hi;   // no group exceeds this
-    // up to 16 routed rows per pass over a weight tile; larger groups take several passes
-    if (fmt == FMT_NF4) return mmax <= 8 ? launch_db<FMT_NF4, 1>(a, s) : launch_db<FMT_NF4, 2>(a, s);
-    return mmax <= 8 ? launch_db<FMT_MXFP4, 1>(a, s) : launch_db<FMT_MXFP4, 2>(a, s);
+    db::Plan pl;
+    const int SB = (fmt == FMT_NF4) ? 64 : 32;
+    pl.nblk = a.K / SB;
+    pl.nc = (a.K + db::kChunkK - 1) / db::kChunkK;
+    pl.np = pick_parts(pl.nc);
+    pl.smem_bytes = 0;
+    const int per_chunk = db::kChunkK / SB;           // blocks of a chunk: one vector of scales per row
+    // one vector load per row for a chunk's scales when every chunk's scales start
+    // on a vector boundary (16 bytes of f32 x 4, 8 bytes of e8m0 x 8); else scalar loads
+    const uintptr_t sbase = reinterpret_cast<uintptr_t>(a.scales);
+    if (fmt == FMT_NF4) pl.vec_scales = (pl.nblk % 4 == 0) && (sbase % 16 == 0);
+    else pl.vec_scales = (pl.nblk % per_chunk == 0) && (sbase % 8 == 0);
+    const int64_t mmax = a.R < (int64_t)a.m_hi ? a.R : (int64_t)a.m_hi;      // no group exceeds this
+    if (fmt == FMT_NF4) {
+        if (mmax <= GNF4_DB_NG1_MAX) return launch_db<FMT_NF4, db::SC_F32, 0, 1>(a, pl, s);
+        return launch_db<FMT_NF4, db::SC_F32, 0, 2>(a, pl, s);
+    }
+    if (mmax <= GNF4_DB_NG1_MAX) return launch_db<FMT_MXFP4, db::SC_E8M0, 0, 1>(a, pl, s);
+    return launch_db<FMT_MXFP4, db::SC_E8M0, 0, 2>(a, pl, s);
 }
 
 unsigned take_decode_error(cudaError_t* err) {
