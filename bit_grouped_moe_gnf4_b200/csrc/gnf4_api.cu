@@ -1,4 +1,5 @@
 // The C ABI of include/gnf4.h: argument validation, band selection, launches.
+#include <atomic>
 #include <climits>
 #include <cstdint>
 #include <cstdarg>
@@ -34,28 +35,45 @@ static gnf4_status cuda_fail(cudaError_t e, const char* what) {
     return fail(GNF4_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
+// device (or managed) memory of the current device; managed memory is accepted on
+// any device, since the GPU reaches it through page migration
 static bool is_device_ptr(const void* p) {
     cudaPointerAttributes attr;
     if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
         cudaGetLastError();
         return false;
     }
-    return attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged;
+    if (attr.type == cudaMemoryTypeManaged) return true;
+    if (attr.type != cudaMemoryTypeDevice) return false;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return attr.device == dev;
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int device_sm_count() {
-    static int cached[64] = {0};
+int current_device() {
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) dev = 0;
-    if (cached[dev] == 0) {
-        int n = 0;
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        cached[dev] = n > 0 ? n : 1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        dev = 0;
     }
-    return cached[dev];
+    return (dev < 0 || dev >= 64) ? 0 : dev;
+}
+
+int device_sm_count() {
+    static std::atomic<int> cached[64];
+    const int dev = current_device();
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 1;
+        cached[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
 }
 
 static uint16_t host_bf16_rne(float f) {
@@ -96,10 +114,14 @@ static gnf4_status check_quantize_args(const float* w, int64_t rows, int64_t K, 
     return GNF4_OK;
 }
 
-// status word of the routing check
-__device__ unsigned g_check_status;
+// Status words of the routing check: each checked call takes the next of these slots
+// (round robin), so calls checked at the same time on different streams (up to the
+// slot count) never share a word.
+constexpr int kCheckSlots = 256;
+__device__ unsigned g_check_status[kCheckSlots];
+static std::atomic<unsigned> g_check_next{0};
 
-__global__ void check_routing_kernel(const GroupedArgs p, int64_t T_in, int64_t T_out) {
+__global__ void check_routing_kernel(const GroupedArgs p, int64_t T_in, int64_t T_out, int slot) {
     unsigned bad = 0;
     const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -117,18 +139,20 @@ __global__ void check_routing_kernel(const GroupedArgs p, int64_t T_in, int64_t 
         }
         if (p.row_weight && !isfinite(p.row_weight[r])) bad |= 16u;
     }
-    if (bad) atomicOr(&g_check_status, bad);
+    if (bad) atomicOr(&g_check_status[slot], bad);
 }
 
 cudaError_t launch_check_routing(const GroupedArgs& a, int64_t T_in, int64_t T_out,
                                  unsigned* status_out, cudaStream_t s) {
+    const int slot = (int)(g_check_next.fetch_add(1u, std::memory_order_relaxed) % kCheckSlots);
+    const size_t off = sizeof(unsigned) * (size_t)slot;
     const unsigned zero = 0;
-    cudaError_t e = cudaMemcpyToSymbolAsync(g_check_status, &zero, sizeof(zero), 0,
+    cudaError_t e = cudaMemcpyToSymbolAsync(g_check_status, &zero, sizeof(zero), off,
                                             cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess) return e;
-    check_routing_kernel<<<64, 256, 0, s>>>(a, T_in, T_out);
+    check_routing_kernel<<<64, 256, 0, s>>>(a, T_in, T_out, slot);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    e = cudaMemcpyFromSymbolAsync(status_out, g_check_status, sizeof(unsigned), 0,
+    e = cudaMemcpyFromSymbolAsync(status_out, g_check_status, sizeof(unsigned), off,
                                   cudaMemcpyDeviceToHost, s);
     if (e != cudaSuccess) return e;
     return cudaStreamSynchronize(s);

@@ -56,6 +56,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <climits>
 #include <cstdint>
 
@@ -785,34 +786,33 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn_db() {
 
 template <int FMT, int SCL, int XH, int NG>
 static cudaError_t launch_db(const GroupedArgs& a, db::Plan& pl, cudaStream_t s) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) dev = 0;
+    const int dev = current_device();
     // the dynamic shared memory starts after the per-block reserved bytes (this kernel
     // has no static shared memory); size the launch so that the layout fits there
-    static int reserved[64] = {0};
-    static bool have_reserved[64] = {false};
-    if (!have_reserved[dev]) {
-        int r = 0;
-        if (cudaDeviceGetAttribute(&r, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess) r = 1024;
-        reserved[dev] = r;
-        have_reserved[dev] = true;
+    static std::atomic<int> reserved[64];            // per device: reserved shared bytes + 1 (0 = unknown)
+    int rsv = reserved[dev].load(std::memory_order_relaxed) - 1;
+    if (rsv < 0) {
+        if (cudaDeviceGetAttribute(&rsv, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess) {
+            cudaGetLastError();
+            rsv = 1024;
+        }
+        reserved[dev].store(rsv + 1, std::memory_order_relaxed);
     }
     db::Layout lay;
     uint32_t bytes = 0;
     for (uint32_t b = 64 * 1024; b <= (uint32_t)db::kMaxSmem; b += 1024)
-        if (db::make_layout((uint32_t)reserved[dev], b, a.E, lay)) {
+        if (db::make_layout((uint32_t)rsv, b, a.E, lay)) {
             bytes = b;
             break;
         }
     if (bytes == 0) return cudaErrorInvalidConfiguration;
     pl.smem_bytes = (int)bytes;
-    static bool attr_done[64] = {false};            // per device: dynamic shared memory opted in
-    if (!attr_done[dev]) {
+    static std::atomic<bool> attr_done[64];          // per device: dynamic shared memory opted in
+    if (!attr_done[dev].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(decode_band_kernel<FMT, SCL, XH, NG>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, db::kMaxSmem);
         if (e != cudaSuccess) return e;
-        attr_done[dev] = true;
+        attr_done[dev].store(true, std::memory_order_release);
     }
     auto enc = encode_fn_db();
     if (!enc) return cudaErrorNotSupported;

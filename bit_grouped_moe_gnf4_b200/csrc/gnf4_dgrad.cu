@@ -1,3 +1,4 @@
+#include <atomic>
 // Input gradient of the grouped 4-bit GEMM: for every routed row r of expert e,
 //   dx[r, k] = w(r) * sum_n g[src(r), n] * What[e, n, k]
 // in one launch over all experts, decoding the packed weights on chip (the
@@ -340,12 +341,13 @@ __global__ void __launch_bounds__(kDgThreads, 2) dgrad_kernel(const DgradArgs p)
 template <int FMT, int RT, int S>
 cudaError_t launch_dg(const DgradArgs& a, cudaStream_t s) {
     const size_t smem = prefix_bytes(a.E) + work_bytes<RT, S>();
-    static bool attr_set = false;
-    if (!attr_set) {
+    static std::atomic<bool> attr_set[64];           // per device: dynamic shared memory opted in
+    const int dev = current_device();
+    if (!attr_set[dev].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(dgrad_kernel<FMT, RT, S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)(prefix_bytes(kDgMaxExperts) + work_bytes<RT, S>()));
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        attr_set[dev].store(true, std::memory_order_release);
     }
     const int grid = device_sm_count() * 2;
     dgrad_kernel<FMT, RT, S><<<grid, kDgThreads, smem, s>>>(a);

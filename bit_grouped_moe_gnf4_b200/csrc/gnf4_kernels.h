@@ -58,6 +58,10 @@ cudaError_t launch_routing(const int32_t* ids, const float* weights, int64_t T, 
 
 int device_sm_count();
 
+// The current CUDA device, clamped to [0, 64) for the per-device caches (kernel
+// attribute opt-ins are per device, so every cache of them is keyed by this).
+int current_device();
+
 // Read and clear the error word a band's kernels set when they give up waiting
 // on a barrier (synchronous; 0 = no event). Returns a CUDA error through *err.
 unsigned take_decode_error(cudaError_t* err);

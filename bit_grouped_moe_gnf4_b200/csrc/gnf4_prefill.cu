@@ -1,3 +1,4 @@
+#include <atomic>
 // Prefill band of the grouped 4-bit GEMM: groups with many routed rows, where
 // the work is a dense contraction and runs on the 5th-generation tensor cores
 // (tcgen05, accumulators in tensor memory). The M-tile path of the solution
@@ -552,12 +553,13 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 template <int FMT>
 static cudaError_t launch_pf(const GroupedArgs& a, int64_t T_in, cudaStream_t s) {
-    static bool configured = false;
-    if (!configured) {
+    static std::atomic<bool> configured[64];         // per device: dynamic shared memory opted in
+    const int dev = current_device();
+    if (!configured[dev].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(prefill_band_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              pf::kSmemBytes);
         if (e != cudaSuccess) return e;
-        configured = true;
+        configured[dev].store(true, std::memory_order_release);
     }
     auto enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;

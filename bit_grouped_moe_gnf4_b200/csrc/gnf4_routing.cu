@@ -1,3 +1,4 @@
+#include <atomic>
 // Routing metadata of a grouped call on the device: the router's top-k choices
 // become expert_offsets, row_token, row_weight and row_dest (rows sorted by
 // expert, then token, then slot), so that a whole MoE layer can run without the
@@ -151,12 +152,13 @@ cudaError_t launch_routing(const int32_t* ids, const float* weights, int64_t T, 
                            cudaStream_t s) {
     const int nw = routing_warps(E, T * k);
     const size_t smem = ((size_t)nw * E + E + 1) * sizeof(uint32_t);
-    static size_t attr = 0;
-    if (smem > 48 * 1024 && attr < smem) {
+    static std::atomic<bool> attr[64];               // per device: the largest table opted in
+    const int dev = current_device();
+    if (smem > 48 * 1024 && !attr[dev].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(routing_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)(201 * 1024 + 4 * 2049));
         if (e != cudaSuccess) return e;
-        attr = 201 * 1024 + 4 * 2049;
+        attr[dev].store(true, std::memory_order_release);
     }
     routing_kernel<<<1, nw * 32, smem, s>>>(ids, weights, T * k, (int)k, E, offsets, row_token, row_weight,
                                             row_dest);

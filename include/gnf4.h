@@ -5,7 +5,8 @@
  * C ABI. Every pointer argument marked "device" must be device (or managed)
  * memory of the current CUDA device; the library checks this and refuses host
  * pointers. The caller owns and allocates every buffer; the library allocates
- * nothing and keeps no per-call state. Every call is asynchronous on `stream`
+ * nothing and keeps no per-call state beyond a few status words of its own in
+ * device memory (see GNF4_CHECK and gnf4_device_status). Every call is asynchronous on `stream`
  * (a cudaStream_t passed as void*, NULL = the legacy default stream) and does
  * no host synchronisation unless GNF4_CHECK is set.
  *
@@ -36,7 +37,11 @@ typedef enum gnf4_status {
 /* flags for the grouped GEMM entry points */
 #define GNF4_CHECK          0x1  /* validate offsets / row_token / row_dest on the device
                                     first (one extra kernel and a stream sync); a bad
-                                    value returns GNF4_ERR_DEVICE_STATUS, nothing else runs */
+                                    value returns GNF4_ERR_DEVICE_STATUS, nothing else runs.
+                                    Each checked call reports through its own status word
+                                    (one of 256 taken round robin), so checked calls on
+                                    different streams at the same time do not mix up their
+                                    results as long as fewer than 256 are in flight */
 #define GNF4_FORCE_DECODE   0x2  /* run every group through the decode band (testing) */
 #define GNF4_FORCE_PREFILL  0x4  /* run every group through the prefill band (testing) */
 
@@ -98,12 +103,14 @@ gnf4_status gnf4_quantize_mxfp4(const float* w, int64_t rows, int64_t K,
  *
  * x              device bf16 [T_in, K], 16-byte aligned
  * W              device uint8 [E, N, K/2] (NF4 codes as gnf4_quantize_nf4 writes them), 16-byte aligned
- * absmax         device fp32  [E, N, K/64]
- * expert_offsets device int64 [E+1]: offsets[0] = 0, non-decreasing, offsets[E] = R;
- *                empty experts (equal neighbours) are legal and cost nothing
- * row_token      device int32 [R] in [0, T_in), or NULL (then T_in >= R)
- * row_weight     device fp32  [R], or NULL
- * row_dest       device int32 [R] in [0, T_out), pairwise distinct, or NULL (then T_out >= R)
+ * absmax         device fp32  [E, N, K/64], 4-byte aligned (any offset into a float
+ *                array); 16-byte alignment lets the kernels use vector loads
+ * expert_offsets device int64 [E+1], 8-byte aligned: offsets[0] = 0, non-decreasing,
+ *                offsets[E] = R; empty experts (equal neighbours) are legal and cost nothing
+ * row_token      device int32 [R] in [0, T_in), or NULL (then T_in >= R); 4-byte aligned
+ * row_weight     device fp32  [R], or NULL; 4-byte aligned
+ * row_dest       device int32 [R] in [0, T_out), pairwise distinct, or NULL (then T_out >= R);
+ *                4-byte aligned
  * out            device bf16 [T_out, N], 16-byte aligned; rows that no routed row
  *                names are not written
  * E >= 1, N % 16 == 0, K % 64 == 0, R >= 0 (R == 0 launches nothing), T_in, T_out < 2^31.
@@ -112,9 +119,10 @@ gnf4_status gnf4_quantize_mxfp4(const float* w, int64_t rows, int64_t K,
  * flags: 0, or GNF4_CHECK / GNF4_FORCE_DECODE / GNF4_FORCE_PREFILL (above).
  * Bands: groups of at most 64 rows run in the decode band, larger groups in the
  * prefill band (tensor cores); a call with R <= 128 runs every group in the
- * decode band (one launch). Results are deterministic for a given call; a row
- * computed in different bands may differ in the last bits (fp32 summation order).
- * Results are deterministic: the same inputs give the same bits on every call.
+ * decode band (one launch). Results are deterministic: the same inputs give the
+ * same bits on every call. Inside the decode band a row's bits do not depend on
+ * the other rows of the call (its fp32 summation order is fixed by K alone); a row
+ * computed in the prefill band may differ from it in the last bits.
  */
 gnf4_status gnf4_grouped_gemm_nf4(const void* x, const uint8_t* W, const float* absmax,
                                   const int64_t* expert_offsets, const int32_t* row_token,

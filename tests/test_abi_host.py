@@ -74,6 +74,13 @@ def _gemm(**kw):
     (dict(T_out=4), _lib.GNF4_ERR_INVALID_ARG),         # row_dest NULL needs T_out >= R
     (dict(x=FAKE + 8), _lib.GNF4_ERR_MISALIGNED),
     (dict(out=FAKE + 2), _lib.GNF4_ERR_MISALIGNED),
+    # fp32 absmax at a non-float boundary, offsets off their 8-byte boundary, row arrays off 4:
+    # all refused before any launch (no kernel ever sees an unaligned vector load)
+    (dict(s=FAKE + 2), _lib.GNF4_ERR_MISALIGNED),
+    (dict(off=FAKE + 4), _lib.GNF4_ERR_MISALIGNED),
+    (dict(tok=FAKE + 2), _lib.GNF4_ERR_MISALIGNED),
+    (dict(wt=FAKE + 1), _lib.GNF4_ERR_MISALIGNED),
+    (dict(dst=FAKE + 2), _lib.GNF4_ERR_MISALIGNED),
 ])
 def test_grouped_gemm_argument_errors(kw, status):
     assert _gemm(**kw) == status
