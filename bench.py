@@ -57,6 +57,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sub-records", action="store_true",
+                    help="default workload only: skip the prefill and MXFP4 sub-records")
     ap.add_argument("--top-k", type=int, default=None, help="sweep workload: top_k (default first)")
     ap.add_argument("--tokens", type=str, default=None, help="comma list overriding the token counts")
     ap.add_argument("--op", default="gemm", choices=["gemm", "dgrad", "layer"] + list(GLUE_OPS),
@@ -286,10 +288,14 @@ def _tokens(args):
 # --------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------
+# the other halves of the metric, measured after the headline step in the same run:
+# the tensor-bound prefill workload and the MXFP4 decode workload
+SUB_RECORDS = (("prefill", "qwen3_prefill_nf4"), ("mxfp4", "gptoss_mxfp4"))
+
+
 def run_ours(args, wl):
     import torch
     import torch.distributed as dist
-    import bit_grouped_moe_gnf4_b200 as g
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -299,10 +305,35 @@ def run_ours(args, wl):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     dev = torch.device("cuda", torch.cuda.current_device())
+    line = measure_step(args, wl, dev, world, rank, headline=True)
+    if wl.name == DEFAULT_WORKLOAD and not args.no_sub_records and not args.tokens and args.top_k is None:
+        for key, name in SUB_RECORDS:
+            sub = measure_step(args, WORKLOADS[name], dev, world, rank, headline=False)
+            line[key] = {k2: sub[k2] for k2 in ("value", "unit", "ms_per_step", "dtype", "config",
+                                                "roofline", "clocks", "gpu_launches")}
+            torch.cuda.empty_cache()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def measure_step(args, wl, dev, world, rank, headline=True):
+    """Time the workload's step (every call, per-call CUDA graphs) and build its
+    JSON record. The headline record also carries the end-to-end figure and the CPU
+    baseline; a sub-record (another half of the metric) carries neither. Every rank
+    calls this the same number of times in the same order (max over ranks inside)."""
+    import torch
+    import torch.distributed as dist
+    import bit_grouped_moe_gnf4_b200 as g
+
     stream = torch.cuda.current_stream()
     prefill = wl.name in PREFILL_WORKLOADS
+    tokens = _tokens(args) if headline else None
+    top_k = args.top_k if headline else None
 
-    calls, k = workload_calls(wl, args.seed, args.top_k, _tokens(args))
+    calls, k = workload_calls(wl, args.seed, top_k, tokens)
     props = torch.cuda.get_device_properties(dev)
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20) or 126 * 2 ** 20
 
@@ -417,7 +448,7 @@ def run_ours(args, wl):
     del graphs
 
     # end-to-end: host buffers in, result back, through the same public call
-    e2e_steps = max(3, min(args.steps, 10))
+    e2e_steps = max(3, min(args.steps, 10)) if headline else 1
     h2d = sum(sum(t.numel() * t.element_size() for t in c["h"].values() if t is not None) for c in prepared)
     d2h = sum(c["outh"].numel() * 2 for c in prepared)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -482,7 +513,7 @@ def run_ours(args, wl):
         "roofline": roof,
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if headline and rank == 0 and world == 1 and not args.no_cpu_baseline:
         nb, nf, nc, dt, cores = oracle_sample(wl, [(c["T"], c["proj"], c["b"]) for c in prepared],
                                               budget_s=12.0, seed=args.seed)
         v = (nf / dt / 1e12) if prefill else (nb / dt / 1e9)
@@ -493,11 +524,10 @@ def run_ours(args, wl):
         one = oracle_one_core(wl, [(c["T"], c["proj"], c["b"]) for c in prepared], args.seed, prefill)
         if one is not None:
             line["cpu_baseline"]["value_one_core"] = one
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    if not headline:
+        line.pop("e2e", None)
+    del stacks, prepared
+    return line
 
 
 # --------------------------------------------------------------------------

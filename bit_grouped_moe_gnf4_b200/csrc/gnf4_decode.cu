@@ -69,22 +69,24 @@ __device__ unsigned g_decode_error;
 
 namespace db {
 
-constexpr int kWarps = 16;
-constexpr int kThreads = kWarps * 32;
-constexpr int kQuads = kWarps / 4;
+// A warp computes TPW tiles of 16 rows per chunk (1 or 2, a kernel template
+// parameter): the 64-row box of a unit is shared by 4 / TPW warps, and a CTA has
+// kQuads boxes in flight side by side (one ring each), so 16 / TPW warps.
+constexpr int kQuads = 4;
+constexpr int kMaxWarps = 16;
 constexpr int kTileRows = 64;                  // weight rows of a unit: 16 per warp of a quad
 constexpr int kChunkK = 256;                   // K per chunk: 128 packed bytes of every row
 constexpr int kBoxBytes = 128;
 constexpr int kStageBytes = kTileRows * kBoxBytes;   // 8 KB: one TMA box
-constexpr int kStages = 3;
+#ifndef GNF4_DB_STAGES
+#define GNF4_DB_STAGES 3
+#endif
+constexpr int kStages = GNF4_DB_STAGES;       // ring stages per quad
+constexpr int kRingBytes = kStages * kStageBytes;
 constexpr int kLutBytes = 256 * 256;           // byte b, lane l -> b*256 + l*4 (bytes 128..255 of each row hold the part slots)
 constexpr int kMaxTableRows = 1024;            // routed rows whose metadata the CTA stages in shared memory
 constexpr int kMaxSmem = 227 * 1024;
 
-// calls whose groups can exceed this many routed rows take 16 rows per pass
-#ifndef GNF4_DB_NG1_MAX
-#define GNF4_DB_NG1_MAX 8
-#endif
 // most K parts of a tile (a power of two, at most kQuads)
 #ifndef GNF4_DB_MAXPARTS
 #define GNF4_DB_MAXPARTS 2
@@ -255,71 +257,94 @@ __device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
     return v;
 }
 
-// The MMAs of one chunk for one warp: rows g / g+8 of the warp's 16 rows against NGC
-// groups of 8 routed rows; acc[j] += blocksum * scale per block. The packed bytes
-// come from the stage: rowa is row ra = 16w + g of the 128B-swizzled box, woff[b] the
-// lane's byte offset of block b inside a row. xp[j] points at this lane's first
-// activation of the chunk (or is null: zeros). FULL: every block of the chunk exists.
-template <int FMT, int SCL, int XH, int NGC, int NG, bool FULL>
-__device__ __forceinline__ void chunk_math(uint32_t rowa, const uint32_t (&woff)[ChunkGeom<FMT>::NB],
-                                           const Scales<SCL>& sc, uint32_t lane_sel,
-                                           const uint16_t* const (&xp)[NG], int nb, float (&acc)[NG][4]) {
+// The MMAs of one chunk for one warp: for each of its TPW tiles of 16 rows, rows
+// g / g+8 against NGC groups of 8 routed rows; acc[tt][j] += blocksum * scale per
+// block. The packed bytes come from the stage: rowa[tt] is the lane's row ra = g of
+// tile tt in the 128B-swizzled box, woff[b] the lane's byte offset of block b inside
+// a row. xp[j] points at this lane's first activation of the chunk (or is null:
+// zeros); the activations are shared by the tiles. FULL: every block is present.
+template <int FMT, int SCL, int XH, int NGC, int NG, int TPW, bool FULL>
+__device__ __forceinline__ void chunk_math(const uint32_t (&rowa)[TPW], const uint32_t (&woff)[ChunkGeom<FMT>::NB],
+                                           const Scales<SCL> (&sc)[TPW], uint32_t lane_sel,
+                                           const uint16_t* const (&xp)[NG], int nb, float (&acc)[TPW][NG][4]) {
     using G = ChunkGeom<FMT>;
     constexpr int XW = G::SB / 8;               // x words of one lane per block (8 or 4)
     constexpr int STEPS = G::SB / 16;           // k16 steps per block (4 or 2)
-    // every packed word of the lane for the chunk, rows ra and ra + 8
-    uint32_t w[2][G::NB * G::LW];
-    const uint32_t rowb = rowa + 8 * kBoxBytes;
+    // every packed word of the lane for the chunk: tiles x rows ra, ra + 8
+    uint32_t w[TPW][2][G::NB * G::LW];
 #pragma unroll
-    for (int b = 0; b < G::NB; ++b) {
-        if constexpr (G::LW == 2) {
-            const uint2 va = lds_v2(rowa + woff[b]), vb = lds_v2(rowb + woff[b]);
-            w[0][2 * b] = va.x; w[0][2 * b + 1] = va.y;
-            w[1][2 * b] = vb.x; w[1][2 * b + 1] = vb.y;
-        } else {
-            w[0][b] = lds_u32(rowa + woff[b]);
-            w[1][b] = lds_u32(rowb + woff[b]);
+    for (int tt = 0; tt < TPW; ++tt) {
+        const uint32_t rowb = rowa[tt] + 8 * kBoxBytes;
+#pragma unroll
+        for (int b = 0; b < G::NB; ++b) {
+            if constexpr (G::LW == 2) {
+                const uint2 va = lds_v2(rowa[tt] + woff[b]), vb = lds_v2(rowb + woff[b]);
+                w[tt][0][2 * b] = va.x; w[tt][0][2 * b + 1] = va.y;
+                w[tt][1][2 * b] = vb.x; w[tt][1][2 * b + 1] = vb.y;
+            } else {
+                w[tt][0][b] = lds_u32(rowa[tt] + woff[b]);
+                w[tt][1][b] = lds_u32(rowb + woff[b]);
+            }
         }
     }
+    // activations of block b for every group (zeros where the lane has no routed row)
+    auto load_x = [&](uint32_t (&xw)[NGC][XW], int b) {
+#pragma unroll
+        for (int j = 0; j < NGC; ++j) {
+            if (xp[j] != nullptr) {
+                const uint4* src = reinterpret_cast<const uint4*>(xp[j] + b * G::SB);
+#pragma unroll
+                for (int q = 0; q < XW / 4; ++q) {
+                    const uint4 v = __ldg(src + q);
+                    xw[j][4 * q] = v.x; xw[j][4 * q + 1] = v.y; xw[j][4 * q + 2] = v.z; xw[j][4 * q + 3] = v.w;
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < XW; ++q) xw[j][q] = 0u;
+            }
+        }
+    };
+    // the next block's activations are loaded while this block computes
+    uint32_t xa[NGC][XW], xb[NGC][XW];
+    load_x(xa, 0);
 #pragma unroll
     for (int b = 0; b < G::NB; ++b) {
         if (FULL || b < nb) {
-            uint32_t xw[NGC][XW];
+            uint32_t (&xw)[NGC][XW] = (b & 1) ? xb : xa;
+            uint32_t (&xn)[NGC][XW] = (b & 1) ? xa : xb;
+            if (b + 1 < G::NB && (FULL || b + 1 < nb)) load_x(xn, b + 1);
+            float c[TPW][NGC][4];
 #pragma unroll
-            for (int j = 0; j < NGC; ++j) {
-                if (xp[j] != nullptr) {
-                    const uint4* src = reinterpret_cast<const uint4*>(xp[j] + b * G::SB);
+            for (int tt = 0; tt < TPW; ++tt)
 #pragma unroll
-                    for (int q = 0; q < XW / 4; ++q) {
-                        const uint4 v = __ldg(src + q);
-                        xw[j][4 * q] = v.x; xw[j][4 * q + 1] = v.y; xw[j][4 * q + 2] = v.z; xw[j][4 * q + 3] = v.w;
-                    }
-                } else {
+                for (int j = 0; j < NGC; ++j) c[tt][j][0] = c[tt][j][1] = c[tt][j][2] = c[tt][j][3] = 0.f;
+            // one MMA chain per block, tile and group, the same for every group count and
+            // tile count, so a row's sum never depends on what shares its pass. The A operand
+            // of step st is bytes 2st and 2st + 1 of rows ra and rb, decoded in operand order.
 #pragma unroll
-                    for (int q = 0; q < XW; ++q) xw[j][q] = 0u;
+            for (int st = 0; st < STEPS; ++st) {
+#pragma unroll
+                for (int tt = 0; tt < TPW; ++tt) {
+                    const uint32_t a0 = lut_lookup(w[tt][0][G::LW * b + ((2 * st) >> 2)], lane_sel, (2 * st) & 3);
+                    const uint32_t a1 = lut_lookup(w[tt][1][G::LW * b + ((2 * st) >> 2)], lane_sel, (2 * st) & 3);
+                    const uint32_t a2 = lut_lookup(w[tt][0][G::LW * b + ((2 * st + 1) >> 2)], lane_sel, (2 * st + 1) & 3);
+                    const uint32_t a3 = lut_lookup(w[tt][1][G::LW * b + ((2 * st + 1) >> 2)], lane_sel, (2 * st + 1) & 3);
+#pragma unroll
+                    for (int j = 0; j < NGC; ++j)
+                        mma16816<XH>(c[tt][j], a0, a1, a2, a3, xw[j][2 * st], xw[j][2 * st + 1]);
                 }
             }
-            // decode: byte i of the lane's bytes -> one 16-bit pair (lower K first)
-            uint32_t da[G::LB], dbv[G::LB];
 #pragma unroll
-            for (int i = 0; i < G::LB; ++i) {
-                da[i] = lut_lookup(w[0][G::LW * b + (i >> 2)], lane_sel, i & 3);
-                dbv[i] = lut_lookup(w[1][G::LW * b + (i >> 2)], lane_sel, i & 3);
-            }
-            const float sa = scale_of<SCL>(sc.s[0], b);
-            const float sb = scale_of<SCL>(sc.s[1], b);
+            for (int tt = 0; tt < TPW; ++tt) {
+                const float sa = scale_of<SCL>(sc[tt].s[0], b);
+                const float sb = scale_of<SCL>(sc[tt].s[1], b);
 #pragma unroll
-            for (int j = 0; j < NGC; ++j) {
-                // one MMA chain per block and group, the same for every group count, so a
-                // row's sum never depends on how many groups share its pass
-                float c[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int s = 0; s < STEPS; ++s)
-                    mma16816<XH>(c, da[2 * s], dbv[2 * s], da[2 * s + 1], dbv[2 * s + 1], xw[j][2 * s], xw[j][2 * s + 1]);
-                acc[j][0] = fmaf(c[0], sa, acc[j][0]);
-                acc[j][1] = fmaf(c[1], sa, acc[j][1]);
-                acc[j][2] = fmaf(c[2], sb, acc[j][2]);
-                acc[j][3] = fmaf(c[3], sb, acc[j][3]);
+                for (int j = 0; j < NGC; ++j) {
+                    acc[tt][j][0] = fmaf(c[tt][j][0], sa, acc[tt][j][0]);
+                    acc[tt][j][1] = fmaf(c[tt][j][1], sa, acc[tt][j][1]);
+                    acc[tt][j][2] = fmaf(c[tt][j][2], sb, acc[tt][j][2]);
+                    acc[tt][j][3] = fmaf(c[tt][j][3], sb, acc[tt][j][3]);
+                }
             }
         }
     }
@@ -334,39 +359,41 @@ __device__ __forceinline__ uint16_t to_out16(float v) {
 // bytes of the shared memory other than the table and the rings: barriers and abort
 // flag, expert tables, scan scratch, row table (16-byte multiple)
 __host__ __device__ constexpr uint32_t other_bytes(int E) {
-    return (uint32_t)(((2 * kQuads * kStages * 8 + 16 + 8ull * (E + 1) + 8ull * E + 8ull * kWarps + 4ull * E +
-                        4ull * E + 4ull * kWarps + 12ull * kMaxTableRows) + 15) & ~15ull);
+    return (uint32_t)(((2 * kQuads * kStages * 8 + 16 + 8ull * (E + 1) + 8ull * E + 8ull * kMaxWarps + 4ull * E +
+                        4ull * E + 4ull * kMaxWarps + 12ull * kMaxTableRows) + 15) & ~15ull);
 }
 
 // Where the rings and the rest go, given the window address of the dynamic shared
-// memory: the table on the first 64 KB boundary; the rings (1024-aligned) after the
-// table if they fit, else before it; the rest in whichever gap is left. Returns false
-// if nothing fits (the host sizes the launch so that it does).
+// memory: the table on the first 64 KB boundary; each quad's ring (1024-aligned) and
+// then the rest go into the first of the two gaps (before and after the table) that
+// still holds them. Returns false if something does not fit (the host sizes the
+// launch so that everything does).
 struct Layout {
-    uint32_t lut, ring, other;
+    uint32_t lut, ring[kQuads], other;
 };
 __host__ __device__ inline bool make_layout(uint32_t base, uint32_t bytes, int E, Layout& L) {
     const uint32_t end = base + bytes;
     const uint32_t lut = (base + 0xFFFFu) & ~0xFFFFu;
-    const uint32_t rb = kQuads * kStages * kStageBytes, ob = other_bytes(E);
     if (lut + kLutBytes > end) return false;
     uint32_t lo = base, hi = lut + kLutBytes;         // free space: [lo, lut) and [hi, end)
-    uint32_t ring;
-    if (hi + rb <= end) {
-        ring = hi;
-        hi += rb;
-    } else {
-        ring = (lo + 1023u) & ~1023u;
-        if (ring + rb > lut) return false;
-        lo = ring + rb;
+    for (int q = 0; q < kQuads; ++q) {
+        const uint32_t a = (lo + 1023u) & ~1023u;
+        if (a + kRingBytes <= lut) {
+            L.ring[q] = a;
+            lo = a + kRingBytes;
+            continue;
+        }
+        const uint32_t b = (hi + 1023u) & ~1023u;
+        if (b + kRingBytes > end) return false;
+        L.ring[q] = b;
+        hi = b + kRingBytes;
     }
-    uint32_t other;
-    if (lo + ob <= lut) other = lo;
-    else if (hi + ob <= end) other = hi;
+    const uint32_t ob = other_bytes(E);
+    const uint32_t a = (lo + 15u) & ~15u, b = (hi + 15u) & ~15u;
+    if (a + ob <= lut) L.other = a;
+    else if (b + ob <= end) L.other = b;
     else return false;
     L.lut = lut;
-    L.ring = ring;
-    L.other = other;
     return true;
 }
 
@@ -376,10 +403,14 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
 
 }  // namespace db
 
-template <int FMT, int SCL, int XH, int NG>
-__global__ void __launch_bounds__(db::kThreads, 1)
+template <int FMT, int SCL, int XH, int NG, int TPW>
+__global__ void __launch_bounds__(512 / TPW, 1)
 decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant__ CUtensorMap wmap) {
     using namespace db;
+    constexpr int kTPW = TPW;
+    constexpr int kBoxWarps = 4 / TPW;              // warps reading one box
+    constexpr int kWarps = kQuads * kBoxWarps;
+    constexpr int kThreads = kWarps * 32;
     using G = ChunkGeom<FMT>;
     constexpr int SSZ = (SCL == SC_F32) ? 4 : (SCL == SC_BF16) ? 2 : 1;   // bytes per scale
 
@@ -391,29 +422,29 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
         return;
     }
     uint8_t* lut = smem_raw + (lay.lut - smem_s);
-    const uint32_t ring_s = lay.ring;
     uint8_t* other = smem_raw + (lay.other - smem_s);
     uint64_t* bars = reinterpret_cast<uint64_t*>(other);            // full[kQuads][kStages], empty[..]
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * kQuads * kStages);
     int64_t* s_up = reinterpret_cast<int64_t*>(other + 2 * kQuads * kStages * 8 + 16);
     int64_t* s_r0 = s_up + (p.E + 1);
-    int64_t* s_wu = s_r0 + p.E;                     // [kWarps] scan scratch
-    int* s_e = reinterpret_cast<int*>(s_wu + kWarps);
+    int64_t* s_wu = s_r0 + p.E;                     // [kMaxWarps] scan scratch
+    int* s_e = reinterpret_cast<int*>(s_wu + kMaxWarps);
     int* s_m = s_e + p.E;
-    int* s_wc = s_m + p.E;                          // [kWarps]
-    int* t_tok = s_wc + kWarps;
+    int* s_wc = s_m + p.E;                          // [kMaxWarps]
+    int* t_tok = s_wc + kMaxWarps;
     float* t_wt = reinterpret_cast<float*>(t_tok + kMaxTableRows);
     int* t_dst = reinterpret_cast<int*>(t_wt + kMaxTableRows);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
-    const int quad = warp >> 2, wq = warp & 3;       // quad, warp within the quad (its 16 rows)
+    const int quad = warp / kBoxWarps, wq = warp % kBoxWarps;   // box ring, warp within it
+    const int row0 = 16 * kTPW * wq;                 // the warp's first row inside a unit's 64
     const int ntile = (p.N + kTileRows - 1) / kTileRows;
 
     if (tid == 0) {
         for (int i = 0; i < kQuads * kStages; ++i) {
             mbar_init(smem_addr(bars + i), 1);                               // full: issuing lane + bytes
-            mbar_init(smem_addr(bars + kQuads * kStages + i), 4);            // empty: the quad's warps
+            mbar_init(smem_addr(bars + kQuads * kStages + i), kBoxWarps);    // empty: the box's warps
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -491,7 +522,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     const bool issuer = (wq == 0 && lane == 0);     // issues the quad's copies
     uint64_t* full = bars + quad * kStages;
     uint64_t* empty = bars + kQuads * kStages + quad * kStages;
-    const uint32_t qring = ring_s + (uint32_t)(quad * kStages * kStageBytes);
+    const uint32_t qring = quad == 0 ? lay.ring[0] : quad == 1 ? lay.ring[1] : quad == 2 ? lay.ring[2] : lay.ring[3];
 
     // unit u -> (active expert a, first weight row n0, first routed row of the pass mc);
     // a only moves forward along a quad's units, so it is found by walking
@@ -538,27 +569,35 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     // scale cursor (every warp, its own rows): one chunk ahead of the math
     int sc_left = nsteps, sc_c = c_lo, sc_a = 0;
     int64_t sc_u = U0 + gi;
-    const uint8_t* sc_p = nullptr;
+    const uint8_t* sc_p[kTPW];
     auto sc_unit = [&]() {
         int n0, mc;
         locate(sc_u, sc_a, n0, mc);
-        // rows past N (a short last tile) read row 0 of the expert instead: in bounds, unused
-        const int rr = (n0 + 16 * wq < p.N) ? n0 + 16 * wq + g : g;
-        const int64_t row = (int64_t)s_e[sc_a] * p.N + rr;
-        sc_p = Sb + (row * pl.nblk + (int64_t)c_lo * G::NB) * SSZ;
+#pragma unroll
+        for (int tt = 0; tt < kTPW; ++tt) {
+            // rows past N (a short last box) read row g of the expert instead: in bounds, unused
+            const int r16 = n0 + row0 + 16 * tt;
+            const int rr = (r16 < p.N) ? r16 + g : g;
+            const int64_t row = (int64_t)s_e[sc_a] * p.N + rr;
+            sc_p[tt] = Sb + (row * pl.nblk + (int64_t)c_lo * G::NB) * SSZ;
+        }
         sc_c = c_lo;
     };
-    auto scales_next = [&](Scales<SCL>& sc) {
+    auto scales_next = [&](Scales<SCL> (&sc)[kTPW]) {
         if (sc_left <= 0) return;
-        load_scales<SCL>(sc, sc_p, s8, min(G::NB, pl.nblk - sc_c * G::NB), vec);
+        const int nb = min(G::NB, pl.nblk - sc_c * G::NB);
+#pragma unroll
+        for (int tt = 0; tt < kTPW; ++tt) {
+            load_scales<SCL>(sc[tt], sc_p[tt], s8, nb, vec);
+            sc_p[tt] += G::NB * SSZ;
+        }
         --sc_left;
-        sc_p += G::NB * SSZ;
         if (++sc_c == c_hi && sc_left > 0) {
             sc_u += ngroups;
             sc_unit();
         }
     };
-    Scales<SCL> scN;                                 // the next chunk's scales
+    Scales<SCL> scN[kTPW];                           // the next chunk's scales
     if (nsteps > 0) {
         sc_unit();
         scales_next(scN);
@@ -615,8 +654,8 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     // ---- math cursor ----
     int mt_ck = 0, mt_a = 0, mt_n0 = 0, mt_mc = 0, mt_unit = 0, nvalid = 0, ng = 0;
     int64_t mt_u = U0 + gi, mt_r0 = 0;
-    bool rows_ok = false;                           // this warp's 16 rows exist (n0 + 16 wq < N)
-    float acc[NG][4];
+    int ntl = 0;                                    // this warp's tiles that exist in the unit (rows < N)
+    float acc[kTPW][NG][4];
     const uint16_t* xp[NG];
     bool dead = false;
 
@@ -625,19 +664,21 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
         mt_r0 = s_r0[mt_a];
         nvalid = min(8 * NG, s_m[mt_a] - mt_mc);
         ng = (nvalid + 7) >> 3;
-        rows_ok = mt_n0 + 16 * wq < p.N;
+        ntl = min(kTPW, max(0, (p.N - mt_n0 - row0) / 16));
 #pragma unroll
         for (int j = 0; j < NG; ++j) {
             xp[j] = nullptr;
             const int jr = 8 * j + g;
             if (jr < nvalid)
                 xp[j] = p.x + (int64_t)tok_of(mt_r0 + mt_mc + jr) * p.K + c_lo * kChunkK + t * (G::SB / 4);
-            acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+#pragma unroll
+            for (int tt = 0; tt < kTPW; ++tt) acc[tt][j][0] = acc[tt][j][1] = acc[tt][j][2] = acc[tt][j][3] = 0.f;
         }
     };
-    // store one lane's four sums (rows n0 + 16 wq + lg and + 8; routed columns 2 lt, 2 lt + 1 of group grp)
-    auto store4 = [&](const float4& v, int lg, int lt, int grp) {
-        const int n_a = mt_n0 + 16 * wq + lg, n_b = n_a + 8;
+    // store one lane's four sums (rows n0 + row0 + 16 tt + lg and + 8; routed columns 2 lt,
+    // 2 lt + 1 of group grp)
+    auto store4 = [&](const float4& v, int tt, int lg, int lt, int grp) {
+        const int n_a = mt_n0 + row0 + 16 * tt + lg, n_b = n_a + 8;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int jc = 8 * grp + 2 * lt + h;
@@ -652,32 +693,39 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     };
     auto unit_end = [&]() {
         if (np == 1) {
-            if (rows_ok && !dead) {
+            if (!dead) {
 #pragma unroll
-                for (int j = 0; j < NG; ++j)
-                    if (j < ng) store4(make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]), g, t, j);
+                for (int tt = 0; tt < kTPW; ++tt)
+#pragma unroll
+                    for (int j = 0; j < NG; ++j)
+                        if (tt < ntl && j < ng)
+                            store4(make_float4(acc[tt][j][0], acc[tt][j][1], acc[tt][j][2], acc[tt][j][3]), tt, g, t, j);
             }
             return;
         }
-        // hand the part sums to the group (slot of parity, warp, group, lane), then
+        // hand the part sums to the group (slot of parity, warp, tile, group, lane), then
         // reduce a share of this warp's rows in part order
         const int par = mt_unit & 1;
 #pragma unroll
-        for (int j = 0; j < NG; ++j)
-            if (j < ng) *slot_ptr(((par * kWarps + warp) * NG + j) * 32 + lane) = make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
-        asm volatile("bar.sync %0, %1;" ::"r"(1 + gi), "r"(np * 128) : "memory");
-        const int ipw = (NG * 32) / np;             // items (one lane's float4 of one group) per warp
-        if (lane < ipw && rows_ok && !dead) {
-            const int q = part * ipw + lane;
-            const int src = q & 31, grp = q >> 5;
-            if (grp < ng) {
-                // warp wq of quad (gi * np + pp) holds part pp of these rows
-                float4 v = *slot_ptr(((par * kWarps + (gi * np) * 4 + wq) * NG + grp) * 32 + src);
+        for (int tt = 0; tt < kTPW; ++tt)
+#pragma unroll
+            for (int j = 0; j < NG; ++j)
+                if (j < ng)
+                    *slot_ptr((((par * kWarps + warp) * kTPW + tt) * NG + j) * 32 + lane) =
+                        make_float4(acc[tt][j][0], acc[tt][j][1], acc[tt][j][2], acc[tt][j][3]);
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + gi), "r"(np * kBoxWarps * 32) : "memory");
+        const int ipw = (kTPW * NG * 32) / np;      // items (one lane's float4 of one tile and group) per warp
+        for (int i = lane; i < ipw && !dead; i += 32) {
+            const int q = part * ipw + i;
+            const int src = q & 31, grp = (q >> 5) % NG, tt = (q >> 5) / NG;
+            if (grp < ng && tt < ntl) {
+                // warp wq of box (gi * np + pp) holds part pp of these rows
+                float4 v = *slot_ptr((((par * kWarps + (gi * np) * kBoxWarps + wq) * kTPW + tt) * NG + grp) * 32 + src);
                 for (int pp = 1; pp < np; ++pp) {
-                    const float4 w = *slot_ptr(((par * kWarps + (gi * np + pp) * 4 + wq) * NG + grp) * 32 + src);
+                    const float4 w = *slot_ptr((((par * kWarps + (gi * np + pp) * kBoxWarps + wq) * kTPW + tt) * NG + grp) * 32 + src);
                     v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
                 }
-                store4(v, src >> 2, src & 3, grp);
+                store4(v, tt, src >> 2, src & 3, grp);
             }
         }
     };
@@ -688,7 +736,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     for (int b = 0; b < G::NB; ++b)
         woff[b] = (G::LW == 2) ? (((uint32_t)((2 * b + (t >> 1)) ^ g) << 4) + (uint32_t)(t & 1) * 8u)
                                : (((uint32_t)(b ^ g) << 4) + (uint32_t)t * 4u);
-    const uint32_t lane_row = (uint32_t)(16 * wq + g) * kBoxBytes;
+    const uint32_t lane_row = (uint32_t)(row0 + g) * kBoxBytes;
     const int nfull = pl.nblk / G::NB;              // chunks with every block present
     int cs = 0;                                     // stage of the current chunk
     uint32_t cph = 0;                               // its full-barrier parity
@@ -696,24 +744,28 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     uint32_t rph = 0;                               // parity of that stage's release
 
     auto step = [&]() {
-        const Scales<SCL> use = scN;                // this chunk's scales (loaded a step ago)
+        Scales<SCL> use[kTPW];                      // this chunk's scales (loaded a step ago)
+#pragma unroll
+        for (int tt = 0; tt < kTPW; ++tt) use[tt] = scN[tt];
         scales_next(scN);
         if (mt_ck == 0) unit_begin();
         if (!dead && !wait_bounded(smem_addr(full + cs), cph, abort_flag)) dead = true;
-        if (!dead && rows_ok) {
+        if (!dead && ntl > 0) {
             const int c = c_lo + mt_ck;
-            const uint32_t rowa = qring + (uint32_t)cs * kStageBytes + lane_row;
+            uint32_t rowa[kTPW];
+#pragma unroll
+            for (int tt = 0; tt < kTPW; ++tt) rowa[tt] = qring + (uint32_t)cs * kStageBytes + lane_row + tt * 16 * kBoxBytes;
             if (c < nfull) {
                 if (NG == 1 || ng == 1)
-                    chunk_math<FMT, SCL, XH, 1, NG, true>(rowa, woff, use, lane_sel, xp, G::NB, acc);
+                    chunk_math<FMT, SCL, XH, 1, NG, TPW, true>(rowa, woff, use, lane_sel, xp, G::NB, acc);
                 else
-                    chunk_math<FMT, SCL, XH, (NG > 1 ? 2 : 1), NG, true>(rowa, woff, use, lane_sel, xp, G::NB, acc);
+                    chunk_math<FMT, SCL, XH, (NG > 1 ? 2 : 1), NG, TPW, true>(rowa, woff, use, lane_sel, xp, G::NB, acc);
             } else {
                 const int nb = pl.nblk - c * G::NB;
                 if (NG == 1 || ng == 1)
-                    chunk_math<FMT, SCL, XH, 1, NG, false>(rowa, woff, use, lane_sel, xp, nb, acc);
+                    chunk_math<FMT, SCL, XH, 1, NG, TPW, false>(rowa, woff, use, lane_sel, xp, nb, acc);
                 else
-                    chunk_math<FMT, SCL, XH, (NG > 1 ? 2 : 1), NG, false>(rowa, woff, use, lane_sel, xp, nb, acc);
+                    chunk_math<FMT, SCL, XH, (NG > 1 ? 2 : 1), NG, TPW, false>(rowa, woff, use, lane_sel, xp, nb, acc);
             }
         }
         __syncwarp();
@@ -722,7 +774,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
             cs = 0;
             cph ^= 1u;
         }
-        // the issuing lane refills the oldest stage once all four warps released it
+        // the issuing lane refills the oldest stage once every warp of the box released it
         // (the chunk kStages before the one it now receives)
         if (issuer && cp_left > 0 && cp_j >= kStages) {
             if (!dead && !wait_bounded(smem_addr(empty + rs), rph, abort_flag)) dead = true;
@@ -784,7 +836,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn_db() {
     return fn;
 }
 
-template <int FMT, int SCL, int XH, int NG>
+template <int FMT, int SCL, int XH, int NG, int TPW>
 static cudaError_t launch_db(const GroupedArgs& a, db::Plan& pl, cudaStream_t s) {
     const int dev = current_device();
     // the dynamic shared memory starts after the per-block reserved bytes (this kernel
@@ -809,7 +861,7 @@ static cudaError_t launch_db(const GroupedArgs& a, db::Plan& pl, cudaStream_t s)
     pl.smem_bytes = (int)bytes;
     static std::atomic<bool> attr_done[64];          // per device: dynamic shared memory opted in
     if (!attr_done[dev].load(std::memory_order_acquire)) {
-        cudaError_t e = cudaFuncSetAttribute(decode_band_kernel<FMT, SCL, XH, NG>,
+        cudaError_t e = cudaFuncSetAttribute(decode_band_kernel<FMT, SCL, XH, NG, TPW>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, db::kMaxSmem);
         if (e != cudaSuccess) return e;
         attr_done[dev].store(true, std::memory_order_release);
@@ -827,7 +879,7 @@ static cudaError_t launch_db(const GroupedArgs& a, db::Plan& pl, cudaStream_t s)
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     const int grid = device_sm_count();
-    decode_band_kernel<FMT, SCL, XH, NG><<<grid, db::kThreads, bytes, s>>>(a, pl, wmap);
+    decode_band_kernel<FMT, SCL, XH, NG, TPW><<<grid, 512 / TPW, bytes, s>>>(a, pl, wmap);
     return cudaGetLastError();
 }
 
@@ -844,13 +896,20 @@ cudaError_t launch_decode_band(int fmt, const GroupedArgs& a, cudaStream_t s) {
     const uintptr_t sbase = reinterpret_cast<uintptr_t>(a.scales);
     if (fmt == FMT_NF4) pl.vec_scales = (pl.nblk % 4 == 0) && (sbase % 16 == 0);
     else pl.vec_scales = (pl.nblk % per_chunk == 0) && (sbase % 8 == 0);
+    // 8 routed rows per pass when no group can exceed 8, or when groups are small on
+    // average (fewer than 4 rows an expert: the rare larger group takes extra passes);
+    // 16 per pass otherwise. Both give a row the same bits (one MMA chain per block and
+    // group either way), so the choice never changes a result.
     const int64_t mmax = a.R < (int64_t)a.m_hi ? a.R : (int64_t)a.m_hi;      // no group exceeds this
+    const bool one = mmax <= 8 || a.R < 4 * (int64_t)a.E;
+    // NF4 (4 blocks a chunk): two tiles a warp, 8 warps; MXFP4 (8 blocks a chunk, twice
+    // the code and registers per tile): one tile a warp, 16 warps (measured faster each)
     if (fmt == FMT_NF4) {
-        if (mmax <= GNF4_DB_NG1_MAX) return launch_db<FMT_NF4, db::SC_F32, 0, 1>(a, pl, s);
-        return launch_db<FMT_NF4, db::SC_F32, 0, 2>(a, pl, s);
+        if (one) return launch_db<FMT_NF4, db::SC_F32, 0, 1, 2>(a, pl, s);
+        return launch_db<FMT_NF4, db::SC_F32, 0, 2, 2>(a, pl, s);
     }
-    if (mmax <= GNF4_DB_NG1_MAX) return launch_db<FMT_MXFP4, db::SC_E8M0, 0, 1>(a, pl, s);
-    return launch_db<FMT_MXFP4, db::SC_E8M0, 0, 2>(a, pl, s);
+    if (one) return launch_db<FMT_MXFP4, db::SC_E8M0, 0, 1, 1>(a, pl, s);
+    return launch_db<FMT_MXFP4, db::SC_E8M0, 0, 2, 1>(a, pl, s);
 }
 
 unsigned take_decode_error(cudaError_t* err) {
