@@ -57,6 +57,11 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--absmax", default="f32", choices=["f32", "bf16"],
+                    help="NF4 absmax storage: f32, or bf16 (the weights are then drawn as bf16 values, a "
+                         "bf16 source, so the cast is lossless)")
+    ap.add_argument("--x-dtype", default="bf16", choices=["bf16", "f16"],
+                    help="activations (and output) type")
     ap.add_argument("--no-sub-records", action="store_true",
                     help="default workload only: skip the prefill and MXFP4 sub-records")
     ap.add_argument("--top-k", type=int, default=None, help="sweep workload: top_k (default first)")
@@ -81,8 +86,12 @@ def workload_calls(wl, seed, top_k=None, tokens=None):
     return calls, k
 
 
-def call_bytes(fmt, proj, b):
+def call_bytes(fmt, proj, b, absmax="f32"):
+    """Algorithmic bytes of one call: the packed codes and scales of the experts it
+    touches (bf16 absmax: 2 bytes a block instead of 4)."""
     pb = expert_bytes(fmt, proj.N, proj.K)
+    if fmt == "nf4" and absmax == "bf16":
+        pb = dict(pb, scales=pb["scales"] // 2)
     n_act = int((np.diff(b.offsets) > 0).sum())
     return n_act * (pb["nibbles"] + pb["scales"]), n_act * pb["nibbles"]
 
@@ -332,6 +341,9 @@ def measure_step(args, wl, dev, world, rank, headline=True):
     prefill = wl.name in PREFILL_WORKLOADS
     tokens = _tokens(args) if headline else None
     top_k = args.top_k if headline else None
+    absmax = args.absmax if (headline and wl.fmt == "nf4") else "f32"
+    xf16 = headline and args.x_dtype == "f16"
+    xdt = torch.float16 if xf16 else torch.bfloat16
 
     calls, k = workload_calls(wl, args.seed, top_k, tokens)
     props = torch.cuda.get_device_properties(dev)
@@ -346,7 +358,10 @@ def measure_step(args, wl, dev, world, rank, headline=True):
         Wl, Sl = [], []
         for e in range(wl.E):
             w = torch.randn((proj.N, proj.K), generator=gen, device=dev, dtype=torch.float32) * 0.02
-            if wl.fmt == "nf4":
+            if wl.fmt == "nf4" and absmax == "bf16":
+                p, s = g.quantize_nf4(w.to(torch.bfloat16).to(torch.float32))   # a bf16 source
+                s = g.absmax_to_bf16(s)                                         # lossless: exact cast
+            elif wl.fmt == "nf4":
                 p, s = g.quantize_nf4(w)
             else:
                 p, s = g.quantize_mxfp4(w)
@@ -358,7 +373,7 @@ def measure_step(args, wl, dev, world, rank, headline=True):
         stacks[proj.name] = [(W, S)]
         stack_bytes += W.numel() + S.numel() * S.element_size()
     # copies so that two uses of one copy are > 2 x L2 apart
-    step_bytes = sum(call_bytes(wl.fmt, p, b)[0] for _, p, b in calls)
+    step_bytes = sum(call_bytes(wl.fmt, p, b, absmax)[0] for _, p, b in calls)
     ncopies = max(1, min(8, int(np.ceil(2.0 * l2 / max(1, step_bytes))) + 1))
     free = torch.cuda.mem_get_info(dev)[0]
     while ncopies > 1 and (ncopies - 1) * stack_bytes > 0.5 * free:
@@ -379,14 +394,16 @@ def measure_step(args, wl, dev, world, rank, headline=True):
         else:
             xb = synth.activations_bf16(args.seed, b.R, proj.K, tag="x_down")
             tok, wt, dst, T_out = None, b.row_weight, b.row_dest, T * b.k
-        xh = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).pin_memory()
+        if xf16:      # the same draw, rounded to fp16 instead
+            xb = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).float().to(torch.float16).numpy().view(np.uint16)
+        xh = torch.from_numpy(xb.view(np.int16)).view(xdt).pin_memory()
         h = {"x": xh, "off": torch.from_numpy(b.offsets).pin_memory()}
         for nm, a in (("tok", tok), ("wt", wt), ("dst", dst)):
             h[nm] = None if a is None else torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
         d = {nm: (None if t is None else t.to(dev)) for nm, t in h.items()}
-        out = torch.zeros((T_out, proj.N), dtype=torch.bfloat16, device=dev)
-        outh = torch.empty((T_out, proj.N), dtype=torch.bfloat16).pin_memory()
-        nb, nn = call_bytes(wl.fmt, proj, b)
+        out = torch.zeros((T_out, proj.N), dtype=xdt, device=dev)
+        outh = torch.empty((T_out, proj.N), dtype=xdt).pin_memory()
+        nb, nn = call_bytes(wl.fmt, proj, b, absmax)
         prepared.append(dict(T=T, proj=proj, b=b, h=h, d=d, out=out, outh=outh, bytes=nb, nib=nn,
                              flop=2.0 * b.R * proj.N * proj.K))
 
@@ -501,8 +518,9 @@ def measure_step(args, wl, dev, world, rank, headline=True):
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": describe(wl, k), "format": wl.fmt,
+        "vs_baseline": None, "dtype": "f16" if xf16 else "bf16", "data": "synthetic",
+        "config": {"workload": describe(wl, k), "format": wl.fmt, "absmax": absmax if wl.fmt == "nf4" else "e8m0",
+                   "activations": "f16" if xf16 else "bf16",
                    "algorithmic_bytes_per_step": work_bytes, "nibble_bytes_per_step": work_nib,
                    "flop_per_step": work_flop,
                    "l2": f"rotating {ncopies} weight-stack copies ({ncopies * stack_bytes / 1e6:.0f} MB; "

@@ -22,6 +22,10 @@ GNF4_CHECK = 0x1
 GNF4_FORCE_DECODE = 0x2
 GNF4_FORCE_PREFILL = 0x4
 
+GNF4_DTYPE_BF16 = 0
+GNF4_DTYPE_F16 = 1
+GNF4_DTYPE_F32 = 2
+
 STATUS_NAMES = {0: "GNF4_OK", 1: "GNF4_ERR_INVALID_ARG", 2: "GNF4_ERR_UNSUPPORTED_SHAPE",
                 3: "GNF4_ERR_MISALIGNED", 4: "GNF4_ERR_CUDA", 5: "GNF4_ERR_DEVICE_STATUS"}
 
@@ -29,7 +33,8 @@ STATUS_NAMES = {0: "GNF4_OK", 1: "GNF4_ERR_INVALID_ARG", 2: "GNF4_ERR_UNSUPPORTE
 EXPORTED = ("gnf4_last_error", "gnf4_version", "gnf4_quantize_nf4", "gnf4_quantize_mxfp4",
             "gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4", "gnf4_grouped_gemm_launches",
             "gnf4_device_status", "gnf4_swiglu", "gnf4_combine_topk", "gnf4_dgrad_nf4",
-            "gnf4_dgrad_mxfp4", "gnf4_routing_metadata")
+            "gnf4_dgrad_mxfp4", "gnf4_routing_metadata", "gnf4_grouped_gemm_nf4_ex",
+            "gnf4_grouped_gemm_mxfp4_ex", "gnf4_absmax_to_bf16")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
@@ -50,6 +55,14 @@ for _name in ("gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4"):
     getattr(lib, _name).restype = _i32
     getattr(lib, _name).argtypes = [_p, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _i64, _i64,
                                     _p, _i32, _p]
+lib.gnf4_grouped_gemm_nf4_ex.restype = _i32
+lib.gnf4_grouped_gemm_nf4_ex.argtypes = [_p, _i32, _p, _p, _i32, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _i64,
+                                         _i64, _p, _i32, _p]
+lib.gnf4_grouped_gemm_mxfp4_ex.restype = _i32
+lib.gnf4_grouped_gemm_mxfp4_ex.argtypes = [_p, _i32, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _i64,
+                                           _i64, _p, _i32, _p]
+lib.gnf4_absmax_to_bf16.restype = _i32
+lib.gnf4_absmax_to_bf16.argtypes = [_p, _i64, _p, _p]
 for _name in ("gnf4_dgrad_nf4", "gnf4_dgrad_mxfp4"):
     getattr(lib, _name).restype = _i32
     getattr(lib, _name).argtypes = [_p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _i64, _p, _i32, _p]

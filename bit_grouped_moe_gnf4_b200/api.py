@@ -75,12 +75,21 @@ def grouped_gemm(fmt: str, x: torch.Tensor, W: torch.Tensor, scales: torch.Tenso
                  R: Optional[int] = None, stream=None) -> torch.Tensor:
     """One grouped GEMM call (see include/gnf4.h). ``R`` (the routed row count) is
     taken from ``row_token``/``row_weight``/``row_dest`` when one is given, else it
-    must be passed (it is never read back from the device)."""
+    must be passed (it is never read back from the device). ``x`` is bf16 or fp16 (the
+    output has its type); NF4 ``scales`` (absmax) are fp32 or bf16 (the bf16-absmax
+    storage, see ``absmax_to_bf16``)."""
     if fmt not in ("nf4", "mxfp4"):
         raise ValueError("fmt must be 'nf4' or 'mxfp4'")
-    _need(x, torch.bfloat16, "x")
+    if x.dtype not in (torch.bfloat16, torch.float16):
+        raise TypeError(f"x must be torch.bfloat16 or torch.float16, got {x.dtype}")
+    _need(x, x.dtype, "x")
     _need(W, torch.uint8, "W")
-    _need(scales, torch.float32 if fmt == "nf4" else torch.uint8, "scales")
+    if fmt == "nf4":
+        if scales.dtype not in (torch.float32, torch.bfloat16):
+            raise TypeError(f"NF4 absmax must be torch.float32 or torch.bfloat16, got {scales.dtype}")
+        _need(scales, scales.dtype, "scales")
+    else:
+        _need(scales, torch.uint8, "scales")
     _need(expert_offsets, torch.int64, "expert_offsets")
     for name, t, dt in (("row_token", row_token, torch.int32), ("row_weight", row_weight, torch.float32),
                         ("row_dest", row_dest, torch.int32)):
@@ -99,14 +108,34 @@ def grouped_gemm(fmt: str, x: torch.Tensor, W: torch.Tensor, scales: torch.Tenso
         raise ValueError("pass R (routed rows) when row_token, row_weight and row_dest are all None")
     if out is None:
         T_out = R if T_out is None else T_out
-        out = torch.empty((T_out, N), dtype=torch.bfloat16, device=x.device)
+        out = torch.empty((T_out, N), dtype=x.dtype, device=x.device)
+    else:
+        _need(out, x.dtype, "out")
+        T_out = out.shape[0]
+    xdt = _lib.GNF4_DTYPE_F16 if x.dtype == torch.float16 else _lib.GNF4_DTYPE_BF16
+    if fmt == "nf4":
+        sdt = _lib.GNF4_DTYPE_BF16 if scales.dtype == torch.bfloat16 else _lib.GNF4_DTYPE_F32
+        st = lib.gnf4_grouped_gemm_nf4_ex(_ptr(x), xdt, _ptr(W), _ptr(scales), sdt, _ptr(expert_offsets),
+                                          _ptr(row_token), _ptr(row_weight), _ptr(row_dest), E, N, K, R,
+                                          x.shape[0], T_out, _ptr(out), flags, _stream(stream))
+    else:
+        st = lib.gnf4_grouped_gemm_mxfp4_ex(_ptr(x), xdt, _ptr(W), _ptr(scales), _ptr(expert_offsets),
+                                            _ptr(row_token), _ptr(row_weight), _ptr(row_dest), E, N, K, R,
+                                            x.shape[0], T_out, _ptr(out), flags, _stream(stream))
+    check(st, f"gnf4_grouped_gemm_{fmt}_ex")
+    return out
+
+
+def absmax_to_bf16(absmax: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The lossless fp32 -> bf16 NF4 absmax cast (include/gnf4.h, gnf4_absmax_to_bf16):
+    raises Gnf4Error if any value has no bf16 equal (an fp32 source)."""
+    _need(absmax, torch.float32, "absmax")
+    if out is None:
+        out = torch.empty(absmax.shape, dtype=torch.bfloat16, device=absmax.device)
     else:
         _need(out, torch.bfloat16, "out")
-        T_out = out.shape[0]
-    fn = lib.gnf4_grouped_gemm_nf4 if fmt == "nf4" else lib.gnf4_grouped_gemm_mxfp4
-    check(fn(_ptr(x), _ptr(W), _ptr(scales), _ptr(expert_offsets), _ptr(row_token), _ptr(row_weight),
-             _ptr(row_dest), E, N, K, R, x.shape[0], T_out, _ptr(out), flags, _stream(stream)),
-          f"gnf4_grouped_gemm_{fmt}")
+    check(lib.gnf4_absmax_to_bf16(_ptr(absmax), absmax.numel(), _ptr(out), _stream(stream)),
+          "gnf4_absmax_to_bf16")
     return out
 
 

@@ -83,7 +83,25 @@ static uint16_t host_bf16_rne(float f) {
     return (uint16_t)(u >> 16);
 }
 
-LutPlanes make_lut(int fmt) {
+// fp32 -> IEEE binary16 bits, round to nearest even; the codebook values are all
+// zero or normal binary16 numbers, which is all this handles
+static uint16_t host_f16_rne(float f) {
+    uint32_t u;
+    std::memcpy(&u, &f, 4);
+    const uint32_t sign = (u >> 16) & 0x8000u;
+    if ((u & 0x7FFFFFFFu) == 0) return (uint16_t)sign;
+    int exp = (int)((u >> 23) & 0xFFu) - 127 + 15;
+    uint32_t m = (u & 0x7FFFFFu) >> 13;
+    const uint32_t rem = u & 0x1FFFu;
+    if (rem > 0x1000u || (rem == 0x1000u && (m & 1u))) ++m;
+    if (m == 0x400u) {
+        m = 0;
+        ++exp;
+    }
+    return (uint16_t)(sign | ((uint32_t)exp << 10) | m);
+}
+
+LutPlanes make_lut(int fmt, int f16) {
     // NF4 values (QLoRA / bitsandbytes NF4) and the OCP e2m1 magnitudes
     static const float nf4[16] = {
         -1.0f, -0.6961928009986877f, -0.5250730514526367f, -0.39491748809814453f,
@@ -96,7 +114,8 @@ LutPlanes make_lut(int fmt) {
     std::memset(&L, 0, sizeof(L));
     const int n = (fmt == FMT_NF4) ? 16 : 8;
     for (int i = 0; i < n; ++i) {
-        const uint16_t b = host_bf16_rne(fmt == FMT_NF4 ? nf4[i] : e2m1[i]);
+        const float v = fmt == FMT_NF4 ? nf4[i] : e2m1[i];
+        const uint16_t b = f16 ? host_f16_rne(v) : host_bf16_rne(v);
         L.lo[i >> 2] |= (uint32_t)(b & 0xFFu) << (8 * (i & 3));
         L.hi[i >> 2] |= (uint32_t)(b >> 8) << (8 * (i & 3));
     }
@@ -158,12 +177,43 @@ cudaError_t launch_check_routing(const GroupedArgs& a, int64_t T_in, int64_t T_o
     return cudaStreamSynchronize(s);
 }
 
-static gnf4_status grouped(int fmt, const void* x, const uint8_t* W, const void* scales,
-                           const int64_t* offsets, const int32_t* row_token,
+// The lossless fp32 -> bf16 absmax cast: the high half of each value; any value whose
+// low half is not zero (bf16 cannot hold it) marks the call's status slot.
+__global__ void absmax_to_bf16_kernel(const uint32_t* a, int64_t n, uint16_t* out, int slot) {
+    unsigned bad = 0;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const uint32_t v = a[i];
+        bad |= (v & 0xFFFFu) ? 1u : 0u;
+        out[i] = (uint16_t)(v >> 16);
+    }
+    if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0) atomicOr(&g_check_status[slot], 1u);
+}
+
+cudaError_t launch_absmax_to_bf16(const float* a, int64_t n, uint16_t* out, unsigned* inexact, cudaStream_t s) {
+    const int slot = (int)(g_check_next.fetch_add(1u, std::memory_order_relaxed) % kCheckSlots);
+    const size_t off = sizeof(unsigned) * (size_t)slot;
+    const unsigned zero = 0;
+    cudaError_t e = cudaMemcpyToSymbolAsync(g_check_status, &zero, sizeof(zero), off, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return e;
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 4 * (int64_t)device_sm_count()) blocks = 4 * (int64_t)device_sm_count();
+    absmax_to_bf16_kernel<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const uint32_t*>(a), n, out, slot);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbolAsync(inexact, g_check_status, sizeof(unsigned), off, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return e;
+    return cudaStreamSynchronize(s);
+}
+
+static gnf4_status grouped(int fmt, const void* x, int x_dtype, const uint8_t* W, const void* scales,
+                           int scale_dtype, const int64_t* offsets, const int32_t* row_token,
                            const float* row_weight, const int32_t* row_dest, int64_t E,
                            int64_t N, int64_t K, int64_t R, int64_t T_in, int64_t T_out,
                            void* out, int flags, void* stream) {
     const int64_t kmul = (fmt == FMT_NF4) ? 64 : 32;
+    if (x_dtype != GNF4_DTYPE_BF16 && x_dtype != GNF4_DTYPE_F16)
+        return fail(GNF4_ERR_INVALID_ARG, "x_dtype must be GNF4_DTYPE_BF16 or GNF4_DTYPE_F16");
+    if (fmt == FMT_NF4 && scale_dtype != GNF4_DTYPE_F32 && scale_dtype != GNF4_DTYPE_BF16)
+        return fail(GNF4_ERR_INVALID_ARG, "NF4 absmax_dtype must be GNF4_DTYPE_F32 or GNF4_DTYPE_BF16");
     if (!x || !W || !scales || !offsets || !out) return fail(GNF4_ERR_INVALID_ARG, "null pointer argument");
     if (E < 1 || N < 1 || K < 1 || R < 0 || T_in < 0 || T_out < 0)
         return fail(GNF4_ERR_INVALID_ARG, "sizes must be E,N,K >= 1 and R,T_in,T_out >= 0");
@@ -181,8 +231,10 @@ static gnf4_status grouped(int fmt, const void* x, const uint8_t* W, const void*
     if (R > 0 && (T_in == 0 || T_out == 0)) return fail(GNF4_ERR_INVALID_ARG, "R > 0 needs T_in, T_out >= 1");
     if (!aligned16(x) || !aligned16(W) || !aligned16(out))
         return fail(GNF4_ERR_MISALIGNED, "x, W and out must be 16-byte aligned");
-    if (fmt == FMT_NF4 && (reinterpret_cast<uintptr_t>(scales) & 3u))
+    if (fmt == FMT_NF4 && scale_dtype == GNF4_DTYPE_F32 && (reinterpret_cast<uintptr_t>(scales) & 3u))
         return fail(GNF4_ERR_MISALIGNED, "absmax must be 4-byte aligned (fp32)");
+    if (fmt == FMT_NF4 && scale_dtype == GNF4_DTYPE_BF16 && (reinterpret_cast<uintptr_t>(scales) & 1u))
+        return fail(GNF4_ERR_MISALIGNED, "absmax must be 2-byte aligned (bf16)");
     if ((reinterpret_cast<uintptr_t>(offsets) & 7u) || (row_token && (reinterpret_cast<uintptr_t>(row_token) & 3u)) ||
         (row_weight && (reinterpret_cast<uintptr_t>(row_weight) & 3u)) ||
         (row_dest && (reinterpret_cast<uintptr_t>(row_dest) & 3u)))
@@ -207,9 +259,11 @@ static gnf4_status grouped(int fmt, const void* x, const uint8_t* W, const void*
     a.E = (int)E;
     a.N = (int)N;
     a.K = (int)K;
-    static const LutPlanes lut_nf4 = make_lut(FMT_NF4);
-    static const LutPlanes lut_mx = make_lut(FMT_MXFP4);
-    a.lut = (fmt == FMT_NF4) ? lut_nf4 : lut_mx;
+    static const LutPlanes lut_nf4 = make_lut(FMT_NF4, 0), lut_nf4_h = make_lut(FMT_NF4, 1);
+    static const LutPlanes lut_mx = make_lut(FMT_MXFP4, 0), lut_mx_h = make_lut(FMT_MXFP4, 1);
+    a.x_f16 = (x_dtype == GNF4_DTYPE_F16) ? 1 : 0;
+    a.scale_bf16 = (fmt == FMT_NF4 && scale_dtype == GNF4_DTYPE_BF16) ? 1 : 0;
+    a.lut = (fmt == FMT_NF4) ? (a.x_f16 ? lut_nf4_h : lut_nf4) : (a.x_f16 ? lut_mx_h : lut_mx);
 
     if (flags & GNF4_CHECK) {
         unsigned st = 0;
@@ -268,8 +322,8 @@ static gnf4_status dgrad(int fmt, const void* grad_out, const uint8_t* W, const 
         return fail(GNF4_ERR_INVALID_ARG, "every buffer must be device memory of the current device");
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    static const LutPlanes lut_nf4 = make_lut(FMT_NF4);
-    static const LutPlanes lut_mx = make_lut(FMT_MXFP4);
+    static const LutPlanes lut_nf4 = make_lut(FMT_NF4, 0);
+    static const LutPlanes lut_mx = make_lut(FMT_MXFP4, 0);
     if (flags & GNF4_CHECK) {
         GroupedArgs c;
         std::memset(&c, 0, sizeof(c));
@@ -333,8 +387,8 @@ gnf4_status gnf4_grouped_gemm_nf4(const void* x, const uint8_t* W, const float* 
                                   const float* row_weight, const int32_t* row_dest, int64_t E,
                                   int64_t N, int64_t K, int64_t R, int64_t T_in, int64_t T_out,
                                   void* out, int flags, void* stream) {
-    return grouped(FMT_NF4, x, W, absmax, expert_offsets, row_token, row_weight, row_dest, E, N,
-                   K, R, T_in, T_out, out, flags, stream);
+    return grouped(FMT_NF4, x, GNF4_DTYPE_BF16, W, absmax, GNF4_DTYPE_F32, expert_offsets, row_token, row_weight,
+                   row_dest, E, N, K, R, T_in, T_out, out, flags, stream);
 }
 
 gnf4_status gnf4_grouped_gemm_mxfp4(const void* x, const uint8_t* W, const uint8_t* scales,
@@ -342,8 +396,44 @@ gnf4_status gnf4_grouped_gemm_mxfp4(const void* x, const uint8_t* W, const uint8
                                     const float* row_weight, const int32_t* row_dest, int64_t E,
                                     int64_t N, int64_t K, int64_t R, int64_t T_in, int64_t T_out,
                                     void* out, int flags, void* stream) {
-    return grouped(FMT_MXFP4, x, W, scales, expert_offsets, row_token, row_weight, row_dest, E,
-                   N, K, R, T_in, T_out, out, flags, stream);
+    return grouped(FMT_MXFP4, x, GNF4_DTYPE_BF16, W, scales, GNF4_DTYPE_BF16, expert_offsets, row_token,
+                   row_weight, row_dest, E, N, K, R, T_in, T_out, out, flags, stream);
+}
+
+gnf4_status gnf4_grouped_gemm_nf4_ex(const void* x, int x_dtype, const uint8_t* W, const void* absmax,
+                                     int absmax_dtype, const int64_t* expert_offsets, const int32_t* row_token,
+                                     const float* row_weight, const int32_t* row_dest, int64_t E, int64_t N,
+                                     int64_t K, int64_t R, int64_t T_in, int64_t T_out, void* out, int flags,
+                                     void* stream) {
+    return grouped(FMT_NF4, x, x_dtype, W, absmax, absmax_dtype, expert_offsets, row_token, row_weight,
+                   row_dest, E, N, K, R, T_in, T_out, out, flags, stream);
+}
+
+gnf4_status gnf4_grouped_gemm_mxfp4_ex(const void* x, int x_dtype, const uint8_t* W, const uint8_t* scales,
+                                       const int64_t* expert_offsets, const int32_t* row_token,
+                                       const float* row_weight, const int32_t* row_dest, int64_t E, int64_t N,
+                                       int64_t K, int64_t R, int64_t T_in, int64_t T_out, void* out, int flags,
+                                       void* stream) {
+    return grouped(FMT_MXFP4, x, x_dtype, W, scales, GNF4_DTYPE_BF16, expert_offsets, row_token, row_weight,
+                   row_dest, E, N, K, R, T_in, T_out, out, flags, stream);
+}
+
+gnf4_status gnf4_absmax_to_bf16(const float* absmax, int64_t n, uint16_t* absmax_bf16, void* stream) {
+    if (n < 0) return fail(GNF4_ERR_INVALID_ARG, "n must be >= 0");
+    if (n == 0) return GNF4_OK;
+    if (!absmax || !absmax_bf16) return fail(GNF4_ERR_INVALID_ARG, "null pointer argument");
+    if ((reinterpret_cast<uintptr_t>(absmax) & 3u) || (reinterpret_cast<uintptr_t>(absmax_bf16) & 1u))
+        return fail(GNF4_ERR_MISALIGNED, "absmax must be 4-byte and absmax_bf16 2-byte aligned");
+    if (!is_device_ptr(absmax) || !is_device_ptr(absmax_bf16))
+        return fail(GNF4_ERR_INVALID_ARG, "absmax and absmax_bf16 must be device memory of the current device");
+    unsigned inexact = 0;
+    cudaError_t e = launch_absmax_to_bf16(absmax, n, absmax_bf16, &inexact, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "absmax_to_bf16");
+    if (inexact)
+        return fail(GNF4_ERR_INVALID_ARG,
+                    "some absmax values are not exactly representable in bf16 (the source is not bf16); "
+                    "refused, absmax_bf16 holds unspecified values");
+    return GNF4_OK;
 }
 
 gnf4_status gnf4_device_status(void* stream) {

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 namespace gnf4 {
@@ -30,12 +31,14 @@ struct GroupedArgs {
     int64_t R;
     int E, N, K;
     int m_lo, m_hi;             // this band takes groups with m_lo <= rows <= m_hi
-    LutPlanes lut;
+    int x_f16;                  // activations and output: 0 bf16, 1 fp16
+    int scale_bf16;             // NF4 absmax stored as bf16 (1) or fp32 (0)
+    LutPlanes lut;              // codebook in the activations' 16-bit type
 };
 
-// Host-side: the decode tables of each format (bf16 of the codebook values,
-// round to nearest even from the fp32 values).
-LutPlanes make_lut(int fmt);
+// Host-side: the decode tables of each format: the codebook values rounded to
+// nearest even from fp32, to bf16 (f16 = 0) or to IEEE binary16 (f16 = 1).
+LutPlanes make_lut(int fmt, int f16 = 0);
 
 // ---------------------------------------------------------------------------
 // device helpers
@@ -90,10 +93,15 @@ __device__ __forceinline__ float e8m0_to_f32(uint32_t s) {
     return __uint_as_float(s << 23);
 }
 
-template <int FMT>
+// block scale idx as fp32: NF4 absmax stored as fp32 (SBF16 = false) or bf16 (widened
+// exactly), MXFP4 e8m0
+template <int FMT, bool SBF16 = false>
 __device__ __forceinline__ float load_scale(const void* scales, int64_t idx) {
     if constexpr (FMT == FMT_NF4) {
-        return __ldg(reinterpret_cast<const float*>(scales) + idx);
+        if constexpr (SBF16)
+            return __uint_as_float((uint32_t)__ldg(reinterpret_cast<const uint16_t*>(scales) + idx) << 16);
+        else
+            return __ldg(reinterpret_cast<const float*>(scales) + idx);
     } else {
         return e8m0_to_f32(__ldg(reinterpret_cast<const uint8_t*>(scales) + idx));
     }
@@ -105,6 +113,13 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rne(float v) {
     if ((u & 0x7FFFFFFFu) > 0x7F800000u) return (uint16_t)((u >> 16) | 0x40u);
     u += 0x7FFFu + ((u >> 16) & 1u);
     return (uint16_t)(u >> 16);
+}
+
+// fp32 -> the output's 16-bit type (XH = 0: bf16, 1: IEEE binary16), nearest even
+template <int XH>
+__device__ __forceinline__ uint16_t f32_to_out16(float v) {
+    if constexpr (XH == 0) return f32_to_bf16_rne(v);
+    else return __half_as_ushort(__float2half_rn(v));
 }
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,

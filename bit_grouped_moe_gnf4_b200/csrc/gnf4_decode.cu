@@ -350,11 +350,6 @@ __device__ __forceinline__ void chunk_math(const uint32_t (&rowa)[TPW], const ui
     }
 }
 
-template <int XH>
-__device__ __forceinline__ uint16_t to_out16(float v) {
-    if constexpr (XH == 0) return f32_to_bf16_rne(v);
-    else return __half_as_ushort(__float2half_rn(v));
-}
 
 // bytes of the shared memory other than the table and the rings: barriers and abort
 // flag, expert tables, scan scratch, row table (16-byte multiple)
@@ -686,8 +681,8 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
                 const int64_t r = mt_r0 + mt_mc + jc;
                 const float w = wt_of(r);
                 const int64_t d = dst_of(r) * p.N;
-                out[d + n_a] = to_out16<XH>((h ? v.y : v.x) * w);
-                out[d + n_b] = to_out16<XH>((h ? v.w : v.z) * w);
+                out[d + n_a] = f32_to_out16<XH>((h ? v.y : v.x) * w);
+                out[d + n_b] = f32_to_out16<XH>((h ? v.w : v.z) * w);
             }
         }
     };
@@ -894,7 +889,8 @@ cudaError_t launch_decode_band(int fmt, const GroupedArgs& a, cudaStream_t s) {
     // one vector load per row for a chunk's scales when every chunk's scales start
     // on a vector boundary (16 bytes of f32 x 4, 8 bytes of e8m0 x 8); else scalar loads
     const uintptr_t sbase = reinterpret_cast<uintptr_t>(a.scales);
-    if (fmt == FMT_NF4) pl.vec_scales = (pl.nblk % 4 == 0) && (sbase % 16 == 0);
+    if (fmt == FMT_NF4 && !a.scale_bf16) pl.vec_scales = (pl.nblk % 4 == 0) && (sbase % 16 == 0);
+    else if (fmt == FMT_NF4) pl.vec_scales = (pl.nblk % 4 == 0) && (sbase % 8 == 0);   // 8-byte bf16 x 4
     else pl.vec_scales = (pl.nblk % per_chunk == 0) && (sbase % 8 == 0);
     // 8 routed rows per pass when no group can exceed 8, or when groups are small on
     // average (fewer than 4 rows an expert: the rare larger group takes extra passes);
@@ -905,11 +901,15 @@ cudaError_t launch_decode_band(int fmt, const GroupedArgs& a, cudaStream_t s) {
     // NF4 (4 blocks a chunk): two tiles a warp, 8 warps; MXFP4 (8 blocks a chunk, twice
     // the code and registers per tile): one tile a warp, 16 warps (measured faster each)
     if (fmt == FMT_NF4) {
-        if (one) return launch_db<FMT_NF4, db::SC_F32, 0, 1, 2>(a, pl, s);
-        return launch_db<FMT_NF4, db::SC_F32, 0, 2, 2>(a, pl, s);
+        if (a.scale_bf16) {
+            if (a.x_f16) return one ? launch_db<FMT_NF4, db::SC_BF16, 1, 1, 2>(a, pl, s) : launch_db<FMT_NF4, db::SC_BF16, 1, 2, 2>(a, pl, s);
+            return one ? launch_db<FMT_NF4, db::SC_BF16, 0, 1, 2>(a, pl, s) : launch_db<FMT_NF4, db::SC_BF16, 0, 2, 2>(a, pl, s);
+        }
+        if (a.x_f16) return one ? launch_db<FMT_NF4, db::SC_F32, 1, 1, 2>(a, pl, s) : launch_db<FMT_NF4, db::SC_F32, 1, 2, 2>(a, pl, s);
+        return one ? launch_db<FMT_NF4, db::SC_F32, 0, 1, 2>(a, pl, s) : launch_db<FMT_NF4, db::SC_F32, 0, 2, 2>(a, pl, s);
     }
-    if (one) return launch_db<FMT_MXFP4, db::SC_E8M0, 0, 1, 1>(a, pl, s);
-    return launch_db<FMT_MXFP4, db::SC_E8M0, 0, 2, 1>(a, pl, s);
+    if (a.x_f16) return one ? launch_db<FMT_MXFP4, db::SC_E8M0, 1, 1, 1>(a, pl, s) : launch_db<FMT_MXFP4, db::SC_E8M0, 1, 2, 1>(a, pl, s);
+    return one ? launch_db<FMT_MXFP4, db::SC_E8M0, 0, 1, 1>(a, pl, s) : launch_db<FMT_MXFP4, db::SC_E8M0, 0, 2, 1>(a, pl, s);
 }
 
 unsigned take_decode_error(cudaError_t* err) {

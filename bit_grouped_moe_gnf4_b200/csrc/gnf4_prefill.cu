@@ -109,9 +109,12 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
     return d;
 }
 
-// Instruction descriptor, kind::f16: bf16 A and B, fp32 D, both K-major, M = 128.
-__device__ __forceinline__ uint32_t idesc_bf16(int n) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+// Instruction descriptor, kind::f16: A and B both bf16 (XH = 0) or both fp16 (XH = 1),
+// fp32 D, both K-major, M = 128.
+template <int XH>
+__device__ __forceinline__ uint32_t idesc_f16kind(int n) {
+    const uint32_t ab = (XH == 0) ? ((1u << 7) | (1u << 10)) : 0u;   // operand formats: 1 = bf16, 0 = f16
+    return (1u << 4) | ab | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -216,7 +219,7 @@ __device__ __forceinline__ Tile tile_at(const GroupedArgs& p, const Sched& s, in
 
 }  // namespace pf
 
-template <int FMT>
+template <int FMT, bool SBF16, int XH>
 __global__ void __maxnreg__(80)
 prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xmap,
                     const __grid_constant__ CUtensorMap wmap,
@@ -317,7 +320,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
             uint32_t stage_ctr = 0, acc_ctr = 0;
             for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
                 const Tile tl = tile_at(p, sch, t, nnt);
-                const uint32_t idesc = idesc_bf16(tl.bn);
+                const uint32_t idesc = idesc_f16kind<XH>(tl.bn);
                 for (int s = 0; s < nst; ++s, ++stage_ctr) {
                     const uint32_t slot = stage_ctr % kStages, ph = (stage_ctr / kStages) & 1u;
                     if (!mbar_wait_bounded(bar_afull + 8 * slot, ph, abort_flag, err, 1u)) goto mma_done;
@@ -473,14 +476,14 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
                 for (int c = 0; c < 16; ++c) acc[j][c] = 0.f;
             float sring[kScaleAhead];                 // scales of blocks b .. b+kScaleAhead-1
 #pragma unroll
-            for (int u = 0; u < kScaleAhead; ++u) sring[u] = (u < nsbk) ? load_scale<FMT>(p.scales, srow + u) : 0.f;
+            for (int u = 0; u < kScaleAhead; ++u) sring[u] = (u < nsbk) ? load_scale<FMT, SBF16>(p.scales, srow + u) : 0.f;
             for (int b0 = 0; b0 < nsbk; b0 += kScaleAhead) {
 #pragma unroll
                 for (int u = 0; u < kScaleAhead; ++u) {
                     const int b = b0 + u;
                     if (b < nsbk) {
                         const float sc = sring[u];
-                        if (b + kScaleAhead < nsbk) sring[u] = load_scale<FMT>(p.scales, srow + b + kScaleAhead);
+                        if (b + kScaleAhead < nsbk) sring[u] = load_scale<FMT, SBF16>(p.scales, srow + b + kScaleAhead);
                         const uint32_t buf = acc_ctr % kAccBufs, ph = (acc_ctr / kAccBufs) & 1u;
                         ++acc_ctr;
                         if (!mbar_wait_bounded(bar_accfull + 8 * buf, ph, abort_flag, err, 128u)) goto epi_done;
@@ -518,7 +521,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
                                 float v = acc[j][c];
                                 if (p.row_weight) v *= __ldg(p.row_weight + r);
                                 const int64_t dst = p.row_dest ? (int64_t)__ldg(p.row_dest + r) : r;
-                                p.out[dst * p.N + n] = f32_to_bf16_rne(v);
+                                p.out[dst * p.N + n] = f32_to_out16<XH>(v);
                             }
                         }
                     }
@@ -551,12 +554,12 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-template <int FMT>
+template <int FMT, bool SBF16, int XH>
 static cudaError_t launch_pf(const GroupedArgs& a, int64_t T_in, cudaStream_t s) {
     static std::atomic<bool> configured[64];         // per device: dynamic shared memory opted in
     const int dev = current_device();
     if (!configured[dev].load(std::memory_order_acquire)) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_band_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(prefill_band_kernel<FMT, SBF16, XH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              pf::kSmemBytes);
         if (e != cudaSuccess) return e;
         configured[dev].store(true, std::memory_order_release);
@@ -566,12 +569,13 @@ static cudaError_t launch_pf(const GroupedArgs& a, int64_t T_in, cudaStream_t s)
     const int gather = a.row_token != nullptr;
     CUtensorMap xmap, wmap;
     {
-        // activations: bf16 [T_in, K], boxes of 64 K x 128 rows, 128B swizzle
+        // activations: bf16 or fp16 [T_in, K], boxes of 64 K x 128 rows, 128B swizzle
         cuuint64_t dims[2] = {(cuuint64_t)a.K, (cuuint64_t)T_in};
         cuuint64_t strides[1] = {(cuuint64_t)a.K * 2};
         cuuint32_t box[2] = {64, (cuuint32_t)pf::kBNMax};
         cuuint32_t estr[2] = {1, 1};
-        CUresult r = enc(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a.x), dims, strides, box,
+        CUresult r = enc(&xmap, XH ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                         const_cast<uint16_t*>(a.x), dims, strides, box,
                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
@@ -593,12 +597,16 @@ static cudaError_t launch_pf(const GroupedArgs& a, int64_t T_in, cudaStream_t s)
     const int64_t max_tiles = (int64_t)((a.N + pf::kBM - 1) / pf::kBM) * (a.R / pf::kBNMax + a.R / mlo + 1);
     int grid = device_sm_count();
     if (max_tiles < grid) grid = (int)max_tiles;
-    prefill_band_kernel<FMT><<<grid, pf::kThreads, pf::kSmemBytes, s>>>(a, xmap, wmap, gather);
+    prefill_band_kernel<FMT, SBF16, XH><<<grid, pf::kThreads, pf::kSmemBytes, s>>>(a, xmap, wmap, gather);
     return cudaGetLastError();
 }
 
 cudaError_t launch_prefill_band(int fmt, const GroupedArgs& a, int64_t T_in, cudaStream_t s) {
-    return fmt == FMT_NF4 ? launch_pf<FMT_NF4>(a, T_in, s) : launch_pf<FMT_MXFP4>(a, T_in, s);
+    if (fmt == FMT_NF4) {
+        if (a.scale_bf16) return a.x_f16 ? launch_pf<FMT_NF4, true, 1>(a, T_in, s) : launch_pf<FMT_NF4, true, 0>(a, T_in, s);
+        return a.x_f16 ? launch_pf<FMT_NF4, false, 1>(a, T_in, s) : launch_pf<FMT_NF4, false, 0>(a, T_in, s);
+    }
+    return a.x_f16 ? launch_pf<FMT_MXFP4, false, 1>(a, T_in, s) : launch_pf<FMT_MXFP4, false, 0>(a, T_in, s);
 }
 
 unsigned take_prefill_error(cudaError_t* err) {

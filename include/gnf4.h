@@ -45,6 +45,11 @@ typedef enum gnf4_status {
 #define GNF4_FORCE_DECODE   0x2  /* run every group through the decode band (testing) */
 #define GNF4_FORCE_PREFILL  0x4  /* run every group through the prefill band (testing) */
 
+/* storage types of the *_ex entry points */
+#define GNF4_DTYPE_BF16 0    /* bfloat16 */
+#define GNF4_DTYPE_F16  1    /* IEEE binary16 */
+#define GNF4_DTYPE_F32  2    /* IEEE binary32 */
+
 /* Message describing the last failure on the calling thread ("" if none). */
 const char* gnf4_last_error(void);
 
@@ -145,6 +150,50 @@ gnf4_status gnf4_grouped_gemm_mxfp4(const void* x, const uint8_t* W, const uint8
                                     int64_t E, int64_t N, int64_t K, int64_t R,
                                     int64_t T_in, int64_t T_out, void* out,
                                     int flags, void* stream);
+
+/*
+ * Storage variants of the two grouped GEMMs (the same op, contract and errors as
+ * gnf4_grouped_gemm_nf4 / _mxfp4 above, plus the checks of the two type arguments):
+ *  - x_dtype: the activations and the output are bf16 (GNF4_DTYPE_BF16) or IEEE
+ *    binary16 (GNF4_DTYPE_F16): `a_cat [T, K]` bf16/fp16 on the solution page,
+ *    "Supported scope". With fp16 the codebook is decoded to fp16 (rounded to
+ *    nearest even once; the e2m1 values are exact), the tensor-core operands are
+ *    fp16, accumulation stays fp32, and out[...] is rounded once to fp16 (the
+ *    output type follows the activations).
+ *  - absmax_dtype (NF4): fp32 (GNF4_DTYPE_F32, 4-byte aligned) or bf16
+ *    (GNF4_DTYPE_BF16, 2-byte aligned): the grouped-nf4-gemm README (0.11.0), "Which
+ *    entry point? Pick by where the weights live", the --absmax-dtype bf16 paragraph:
+ *    5.6 % fewer bytes per NF4 row, lossless for a bf16 source (see
+ *    gnf4_absmax_to_bf16). The bf16 absmax is widened exactly to fp32 on chip; the
+ *    block scaling is still fp32, outside the MMA.
+ * gnf4_grouped_gemm_nf4_ex(x, GNF4_DTYPE_BF16, W, absmax, GNF4_DTYPE_F32, ...) is
+ * gnf4_grouped_gemm_nf4(x, W, absmax, ...) bit for bit.
+ * Errors: as above; INVALID_ARG for an unknown type, MISALIGNED for an absmax off
+ * its type's alignment.
+ */
+gnf4_status gnf4_grouped_gemm_nf4_ex(const void* x, int x_dtype, const uint8_t* W, const void* absmax,
+                                     int absmax_dtype, const int64_t* expert_offsets,
+                                     const int32_t* row_token, const float* row_weight,
+                                     const int32_t* row_dest, int64_t E, int64_t N, int64_t K, int64_t R,
+                                     int64_t T_in, int64_t T_out, void* out, int flags, void* stream);
+gnf4_status gnf4_grouped_gemm_mxfp4_ex(const void* x, int x_dtype, const uint8_t* W, const uint8_t* scales,
+                                       const int64_t* expert_offsets, const int32_t* row_token,
+                                       const float* row_weight, const int32_t* row_dest, int64_t E,
+                                       int64_t N, int64_t K, int64_t R, int64_t T_in, int64_t T_out,
+                                       void* out, int flags, void* stream);
+
+/*
+ * The lossless absmax cast of the bf16-absmax storage (README 0.11.0, "Which entry
+ * point?", the --absmax-dtype bf16 paragraph: the cast refuses rather than rounds).
+ * absmax_bf16[i] = the bf16 pattern of absmax[i] (its high 16 bits); an fp32 value
+ * whose low 16 bits are not all zero has no bf16 equal, and then the call returns
+ * GNF4_ERR_INVALID_ARG and absmax_bf16 holds unspecified values. For the NF4 absmax
+ * of a bf16 source every value passes (each is one of its block's magnitudes).
+ * absmax device fp32 [n] (4-byte aligned); absmax_bf16 device uint16 [n] (2-byte
+ * aligned). Synchronises `stream` (it reads the verdict back). n == 0 does nothing.
+ * Errors: INVALID_ARG, MISALIGNED, CUDA.
+ */
+gnf4_status gnf4_absmax_to_bf16(const float* absmax, int64_t n, uint16_t* absmax_bf16, void* stream);
 
 /*
  * Synchronise `stream` and report whether any grouped GEMM kernel since the last
