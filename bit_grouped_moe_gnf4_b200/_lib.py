@@ -34,7 +34,8 @@ EXPORTED = ("gnf4_last_error", "gnf4_version", "gnf4_quantize_nf4", "gnf4_quanti
             "gnf4_grouped_gemm_nf4", "gnf4_grouped_gemm_mxfp4", "gnf4_grouped_gemm_launches",
             "gnf4_device_status", "gnf4_swiglu", "gnf4_combine_topk", "gnf4_dgrad_nf4",
             "gnf4_dgrad_mxfp4", "gnf4_routing_metadata", "gnf4_grouped_gemm_nf4_ex",
-            "gnf4_grouped_gemm_mxfp4_ex", "gnf4_absmax_to_bf16")
+            "gnf4_grouped_gemm_mxfp4_ex", "gnf4_absmax_to_bf16", "gnf4_grouped_gemm_swiglu_nf4",
+            "gnf4_grouped_gemm_swiglu_mxfp4")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
@@ -61,6 +62,10 @@ lib.gnf4_grouped_gemm_nf4_ex.argtypes = [_p, _i32, _p, _p, _i32, _p, _p, _p, _p,
 lib.gnf4_grouped_gemm_mxfp4_ex.restype = _i32
 lib.gnf4_grouped_gemm_mxfp4_ex.argtypes = [_p, _i32, _p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i64, _i64,
                                            _i64, _p, _i32, _p]
+lib.gnf4_grouped_gemm_swiglu_nf4.restype = _i32
+lib.gnf4_grouped_gemm_swiglu_nf4.argtypes = lib.gnf4_grouped_gemm_nf4_ex.argtypes
+lib.gnf4_grouped_gemm_swiglu_mxfp4.restype = _i32
+lib.gnf4_grouped_gemm_swiglu_mxfp4.argtypes = lib.gnf4_grouped_gemm_mxfp4_ex.argtypes
 lib.gnf4_absmax_to_bf16.restype = _i32
 lib.gnf4_absmax_to_bf16.argtypes = [_p, _i64, _p, _p]
 for _name in ("gnf4_dgrad_nf4", "gnf4_dgrad_mxfp4"):

@@ -126,6 +126,62 @@ def grouped_gemm(fmt: str, x: torch.Tensor, W: torch.Tensor, scales: torch.Tenso
     return out
 
 
+def grouped_gemm_swiglu(fmt: str, x: torch.Tensor, W: torch.Tensor, scales: torch.Tensor,
+                        expert_offsets: torch.Tensor, row_token: Optional[torch.Tensor] = None,
+                        row_weight: Optional[torch.Tensor] = None, row_dest: Optional[torch.Tensor] = None,
+                        out: Optional[torch.Tensor] = None, T_out: Optional[int] = None, flags: int = 0,
+                        R: Optional[int] = None, stream=None) -> torch.Tensor:
+    """gate_up grouped GEMM with the SwiGLU fused into its epilogue (include/gnf4.h,
+    gnf4_grouped_gemm_swiglu_*): ``W`` is the fused gate_up stack ``[E, 2I, K/2]``, the
+    result ``[T_out, I]`` holds silu(gate) * up in the activations' type."""
+    if fmt not in ("nf4", "mxfp4"):
+        raise ValueError("fmt must be 'nf4' or 'mxfp4'")
+    if x.dtype not in (torch.bfloat16, torch.float16):
+        raise TypeError(f"x must be torch.bfloat16 or torch.float16, got {x.dtype}")
+    _need(x, x.dtype, "x")
+    _need(W, torch.uint8, "W")
+    if fmt == "nf4":
+        if scales.dtype not in (torch.float32, torch.bfloat16):
+            raise TypeError(f"NF4 absmax must be torch.float32 or torch.bfloat16, got {scales.dtype}")
+        _need(scales, scales.dtype, "scales")
+    else:
+        _need(scales, torch.uint8, "scales")
+    _need(expert_offsets, torch.int64, "expert_offsets")
+    for name, t, dt in (("row_token", row_token, torch.int32), ("row_weight", row_weight, torch.float32),
+                        ("row_dest", row_dest, torch.int32)):
+        if t is not None:
+            _need(t, dt, name)
+    E, N, K2 = W.shape
+    K = x.shape[1]
+    if K2 * 2 != K:
+        raise ValueError(f"W is [E, N, K/2] = {tuple(W.shape)} but x has K = {K}")
+    if R is None:
+        for t in (row_token, row_weight, row_dest):
+            if t is not None:
+                R = t.numel()
+                break
+    if R is None:
+        raise ValueError("pass R (routed rows) when row_token, row_weight and row_dest are all None")
+    if out is None:
+        T_out = R if T_out is None else T_out
+        out = torch.empty((T_out, N // 2), dtype=x.dtype, device=x.device)
+    else:
+        _need(out, x.dtype, "out")
+        T_out = out.shape[0]
+    xdt = _lib.GNF4_DTYPE_F16 if x.dtype == torch.float16 else _lib.GNF4_DTYPE_BF16
+    if fmt == "nf4":
+        sdt = _lib.GNF4_DTYPE_BF16 if scales.dtype == torch.bfloat16 else _lib.GNF4_DTYPE_F32
+        st = lib.gnf4_grouped_gemm_swiglu_nf4(_ptr(x), xdt, _ptr(W), _ptr(scales), sdt, _ptr(expert_offsets),
+                                              _ptr(row_token), _ptr(row_weight), _ptr(row_dest), E, N, K, R,
+                                              x.shape[0], T_out, _ptr(out), flags, _stream(stream))
+    else:
+        st = lib.gnf4_grouped_gemm_swiglu_mxfp4(_ptr(x), xdt, _ptr(W), _ptr(scales), _ptr(expert_offsets),
+                                                _ptr(row_token), _ptr(row_weight), _ptr(row_dest), E, N, K, R,
+                                                x.shape[0], T_out, _ptr(out), flags, _stream(stream))
+    check(st, f"gnf4_grouped_gemm_swiglu_{fmt}")
+    return out
+
+
 def absmax_to_bf16(absmax: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """The lossless fp32 -> bf16 NF4 absmax cast (include/gnf4.h, gnf4_absmax_to_bf16):
     raises Gnf4Error if any value has no bf16 equal (an fp32 source)."""

@@ -208,7 +208,7 @@ static gnf4_status grouped(int fmt, const void* x, int x_dtype, const uint8_t* W
                            int scale_dtype, const int64_t* offsets, const int32_t* row_token,
                            const float* row_weight, const int32_t* row_dest, int64_t E,
                            int64_t N, int64_t K, int64_t R, int64_t T_in, int64_t T_out,
-                           void* out, int flags, void* stream) {
+                           void* out, int flags, void* stream, bool fuse_swiglu = false) {
     const int64_t kmul = (fmt == FMT_NF4) ? 64 : 32;
     if (x_dtype != GNF4_DTYPE_BF16 && x_dtype != GNF4_DTYPE_F16)
         return fail(GNF4_ERR_INVALID_ARG, "x_dtype must be GNF4_DTYPE_BF16 or GNF4_DTYPE_F16");
@@ -223,6 +223,9 @@ static gnf4_status grouped(int fmt, const void* x, int x_dtype, const uint8_t* W
         return fail(GNF4_ERR_INVALID_ARG, "GNF4_FORCE_DECODE and GNF4_FORCE_PREFILL exclude each other");
     if (K % kmul) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K must be a multiple of %lld", (long long)kmul);
     if (N % 16) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "N must be a multiple of 16");
+    if (fuse_swiglu && N % 32) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "the fused gate_up width N = 2I must be a multiple of 32");
+    if (fuse_swiglu && (flags & GNF4_FORCE_PREFILL))
+        return fail(GNF4_ERR_INVALID_ARG, "the fused SwiGLU runs in the decode band only");
     if (E > 2048) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "at most 2048 experts");
     if (K > (int64_t)INT_MAX / 2 || E * N > (int64_t)INT_MAX || T_in > INT_MAX || T_out > INT_MAX)
         return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K, E*N, T_in and T_out must fit in int32");
@@ -275,6 +278,12 @@ static gnf4_status grouped(int fmt, const void* x, int x_dtype, const uint8_t* W
                             "16 non-finite row_weight)", st);
     }
 
+    if (fuse_swiglu) {
+        a.m_lo = 1;
+        a.m_hi = INT_MAX;
+        cudaError_t e = launch_decode_band(fmt, a, s, true);
+        return e == cudaSuccess ? GNF4_OK : cuda_fail(e, "fused gate_up + SwiGLU launch");
+    }
     // band split by rows per group; decided on the device from the offsets
     int split = kDecodeMaxRows;
     if (R <= kDecodeOnlyRows) split = INT_MAX;
@@ -416,6 +425,24 @@ gnf4_status gnf4_grouped_gemm_mxfp4_ex(const void* x, int x_dtype, const uint8_t
                                        void* stream) {
     return grouped(FMT_MXFP4, x, x_dtype, W, scales, GNF4_DTYPE_BF16, expert_offsets, row_token, row_weight,
                    row_dest, E, N, K, R, T_in, T_out, out, flags, stream);
+}
+
+gnf4_status gnf4_grouped_gemm_swiglu_nf4(const void* x, int x_dtype, const uint8_t* W, const void* absmax,
+                                         int absmax_dtype, const int64_t* expert_offsets, const int32_t* row_token,
+                                         const float* row_weight, const int32_t* row_dest, int64_t E, int64_t N,
+                                         int64_t K, int64_t R, int64_t T_in, int64_t T_out, void* out, int flags,
+                                         void* stream) {
+    return grouped(FMT_NF4, x, x_dtype, W, absmax, absmax_dtype, expert_offsets, row_token, row_weight,
+                   row_dest, E, N, K, R, T_in, T_out, out, flags, stream, true);
+}
+
+gnf4_status gnf4_grouped_gemm_swiglu_mxfp4(const void* x, int x_dtype, const uint8_t* W, const uint8_t* scales,
+                                           const int64_t* expert_offsets, const int32_t* row_token,
+                                           const float* row_weight, const int32_t* row_dest, int64_t E,
+                                           int64_t N, int64_t K, int64_t R, int64_t T_in, int64_t T_out,
+                                           void* out, int flags, void* stream) {
+    return grouped(FMT_MXFP4, x, x_dtype, W, scales, GNF4_DTYPE_BF16, expert_offsets, row_token, row_weight,
+                   row_dest, E, N, K, R, T_in, T_out, out, flags, stream, true);
 }
 
 gnf4_status gnf4_absmax_to_bf16(const float* absmax, int64_t n, uint16_t* absmax_bf16, void* stream) {

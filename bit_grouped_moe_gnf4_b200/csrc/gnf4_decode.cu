@@ -398,11 +398,17 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
 
 }  // namespace db
 
-template <int FMT, int SCL, int XH, int NG, int TPW>
+template <int FMT, int SCL, int XH, int NG, int TPW, int FUSE>
 __global__ void __launch_bounds__(512 / TPW, 1)
 decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant__ CUtensorMap wmap) {
     using namespace db;
+    static_assert(!FUSE || TPW == 2, "the fused SwiGLU pairs a gate tile with its up tile in one warp");
     constexpr int kTPW = TPW;
+    // FUSE: a unit is 32 gate rows [n0, n0 + 32) and their up rows [I + n0, I + n0 + 32) of
+    // the fused gate_up matrix (two 32-row boxes per stage: gate in stage rows 0..31, up in
+    // 32..63); warp wq takes gate rows n0 + 16 wq .. + 15 as tile 0 and the matching up rows
+    // as tile 1, and writes silu(gate) * up into the [.., I] output
+    constexpr int kUnitRows = FUSE ? 32 : kTileRows;
     constexpr int kBoxWarps = 4 / TPW;              // warps reading one box
     constexpr int kWarps = kQuads * kBoxWarps;
     constexpr int kThreads = kWarps * 32;
@@ -434,7 +440,9 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     const int g = lane >> 2, t = lane & 3;
     const int quad = warp / kBoxWarps, wq = warp % kBoxWarps;   // box ring, warp within it
     const int row0 = 16 * kTPW * wq;                 // the warp's first row inside a unit's 64
-    const int ntile = (p.N + kTileRows - 1) / kTileRows;
+    const int I = p.N / 2;                           // FUSE: output columns (the gate half)
+    const int nrows = FUSE ? I : p.N;                 // rows that units cover
+    const int ntile = (nrows + kUnitRows - 1) / kUnitRows;
 
     if (tid == 0) {
         for (int i = 0; i < kQuads * kStages; ++i) {
@@ -531,7 +539,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
             tile = local / npass;
             pass = local - tile * npass;
         }
-        n0 = tile * kTileRows;
+        n0 = tile * kUnitRows;
         mc = pass * 8 * NG;
     };
 
@@ -548,6 +556,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
         const uint32_t fb = smem_addr(full + cp_s);
         mbar_arrive_tx(fb, (uint32_t)kStageBytes);
         tma_2d(qring + (uint32_t)cp_s * kStageBytes, &wmap, cp_c * kBoxBytes, cp_y, fb);
+        if (FUSE) tma_2d(qring + (uint32_t)cp_s * kStageBytes + kStageBytes / 2, &wmap, cp_c * kBoxBytes, cp_y + I, fb);
         if (++cp_s == kStages) cp_s = 0;
         ++cp_j;
         --cp_left;
@@ -570,9 +579,10 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
         locate(sc_u, sc_a, n0, mc);
 #pragma unroll
         for (int tt = 0; tt < kTPW; ++tt) {
-            // rows past N (a short last box) read row g of the expert instead: in bounds, unused
-            const int r16 = n0 + row0 + 16 * tt;
-            const int rr = (r16 < p.N) ? r16 + g : g;
+            // rows past the end (a short last unit) read row g of the expert instead: in
+            // bounds, unused
+            const int r16 = FUSE ? n0 + 16 * wq : n0 + row0 + 16 * tt;
+            const int rr = (r16 < nrows) ? r16 + g + (FUSE && tt == 1 ? I : 0) : g;
             const int64_t row = (int64_t)s_e[sc_a] * p.N + rr;
             sc_p[tt] = Sb + (row * pl.nblk + (int64_t)c_lo * G::NB) * SSZ;
         }
@@ -659,7 +669,8 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
         mt_r0 = s_r0[mt_a];
         nvalid = min(8 * NG, s_m[mt_a] - mt_mc);
         ng = (nvalid + 7) >> 3;
-        ntl = min(kTPW, max(0, (p.N - mt_n0 - row0) / 16));
+        if (FUSE) ntl = (mt_n0 + 16 * wq < I) ? 2 : 0;
+        else ntl = min(kTPW, max(0, (p.N - mt_n0 - row0) / 16));
 #pragma unroll
         for (int j = 0; j < NG; ++j) {
             xp[j] = nullptr;
@@ -686,15 +697,42 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
             }
         }
     };
+    // FUSE: the same four places of the gate tile (vg) and the up tile (vu) become
+    // silu(w gate) * (w up) in output columns n0 + 16 wq + lg and + 8
+    auto store4_fused = [&](const float4& vg, const float4& vu, int lg, int lt, int grp) {
+        const int c_a = mt_n0 + 16 * wq + lg, c_b = c_a + 8;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int jc = 8 * grp + 2 * lt + h;
+            if (jc < nvalid) {
+                const int64_t r = mt_r0 + mt_mc + jc;
+                const float w = wt_of(r);
+                const int64_t d = dst_of(r) * I;
+                out[d + c_a] = f32_to_out16<XH>(silu_mul((h ? vg.y : vg.x) * w, (h ? vu.y : vu.x) * w));
+                out[d + c_b] = f32_to_out16<XH>(silu_mul((h ? vg.w : vg.z) * w, (h ? vu.w : vu.z) * w));
+            }
+        }
+    };
     auto unit_end = [&]() {
         if (np == 1) {
             if (!dead) {
-#pragma unroll
-                for (int tt = 0; tt < kTPW; ++tt)
+                if (FUSE) {
 #pragma unroll
                     for (int j = 0; j < NG; ++j)
-                        if (tt < ntl && j < ng)
-                            store4(make_float4(acc[tt][j][0], acc[tt][j][1], acc[tt][j][2], acc[tt][j][3]), tt, g, t, j);
+                        if (ntl == 2 && j < ng)
+                            store4_fused(make_float4(acc[0][j][0], acc[0][j][1], acc[0][j][2], acc[0][j][3]),
+                                         make_float4(acc[kTPW - 1][j][0], acc[kTPW - 1][j][1], acc[kTPW - 1][j][2],
+                                                     acc[kTPW - 1][j][3]),
+                                         g, t, j);
+                } else {
+#pragma unroll
+                    for (int tt = 0; tt < kTPW; ++tt)
+#pragma unroll
+                        for (int j = 0; j < NG; ++j)
+                            if (tt < ntl && j < ng)
+                                store4(make_float4(acc[tt][j][0], acc[tt][j][1], acc[tt][j][2], acc[tt][j][3]), tt, g, t,
+                                       j);
+                }
             }
             return;
         }
@@ -709,18 +747,29 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
                     *slot_ptr((((par * kWarps + warp) * kTPW + tt) * NG + j) * 32 + lane) =
                         make_float4(acc[tt][j][0], acc[tt][j][1], acc[tt][j][2], acc[tt][j][3]);
         asm volatile("bar.sync %0, %1;" ::"r"(1 + gi), "r"(np * kBoxWarps * 32) : "memory");
-        const int ipw = (kTPW * NG * 32) / np;      // items (one lane's float4 of one tile and group) per warp
-        for (int i = lane; i < ipw && !dead; i += 32) {
-            const int q = part * ipw + i;
-            const int src = q & 31, grp = (q >> 5) % NG, tt = (q >> 5) / NG;
-            if (grp < ng && tt < ntl) {
-                // warp wq of box (gi * np + pp) holds part pp of these rows
-                float4 v = *slot_ptr((((par * kWarps + (gi * np) * kBoxWarps + wq) * kTPW + tt) * NG + grp) * 32 + src);
-                for (int pp = 1; pp < np; ++pp) {
-                    const float4 w = *slot_ptr((((par * kWarps + (gi * np + pp) * kBoxWarps + wq) * kTPW + tt) * NG + grp) * 32 + src);
-                    v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
-                }
-                store4(v, tt, src >> 2, src & 3, grp);
+        auto part_sum = [&](int tt, int grp, int src) {
+            // warp wq of box (gi * np + pp) holds part pp of these rows
+            float4 v = *slot_ptr((((par * kWarps + (gi * np) * kBoxWarps + wq) * kTPW + tt) * NG + grp) * 32 + src);
+            for (int pp = 1; pp < np; ++pp) {
+                const float4 w = *slot_ptr((((par * kWarps + (gi * np + pp) * kBoxWarps + wq) * kTPW + tt) * NG + grp) * 32 + src);
+                v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+            }
+            return v;
+        };
+        if (FUSE) {
+            const int ipw = (NG * 32) / np;         // items (one lane's gate and up float4s of one group)
+            for (int i = lane; i < ipw && !dead; i += 32) {
+                const int q = part * ipw + i;
+                const int src = q & 31, grp = q >> 5;
+                if (grp < ng && ntl == 2)
+                    store4_fused(part_sum(0, grp, src), part_sum(kTPW - 1, grp, src), src >> 2, src & 3, grp);
+            }
+        } else {
+            const int ipw = (kTPW * NG * 32) / np;  // items (one lane's float4 of one tile and group) per warp
+            for (int i = lane; i < ipw && !dead; i += 32) {
+                const int q = part * ipw + i;
+                const int src = q & 31, grp = (q >> 5) % NG, tt = (q >> 5) / NG;
+                if (grp < ng && tt < ntl) store4(part_sum(tt, grp, src), tt, src >> 2, src & 3, grp);
             }
         }
     };
@@ -749,7 +798,9 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
             const int c = c_lo + mt_ck;
             uint32_t rowa[kTPW];
 #pragma unroll
-            for (int tt = 0; tt < kTPW; ++tt) rowa[tt] = qring + (uint32_t)cs * kStageBytes + lane_row + tt * 16 * kBoxBytes;
+            for (int tt = 0; tt < kTPW; ++tt)
+                rowa[tt] = qring + (uint32_t)cs * kStageBytes +
+                           (FUSE ? (uint32_t)(32 * tt + 16 * wq + g) * kBoxBytes : lane_row + tt * 16 * kBoxBytes);
             if (c < nfull) {
                 if (NG == 1 || ng == 1)
                     chunk_math<FMT, SCL, XH, 1, NG, TPW, true>(rowa, woff, use, lane_sel, xp, G::NB, acc);
@@ -831,7 +882,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn_db() {
     return fn;
 }
 
-template <int FMT, int SCL, int XH, int NG, int TPW>
+template <int FMT, int SCL, int XH, int NG, int TPW, int FUSE = 0>
 static cudaError_t launch_db(const GroupedArgs& a, db::Plan& pl, cudaStream_t s) {
     const int dev = current_device();
     // the dynamic shared memory starts after the per-block reserved bytes (this kernel
@@ -856,29 +907,30 @@ static cudaError_t launch_db(const GroupedArgs& a, db::Plan& pl, cudaStream_t s)
     pl.smem_bytes = (int)bytes;
     static std::atomic<bool> attr_done[64];          // per device: dynamic shared memory opted in
     if (!attr_done[dev].load(std::memory_order_acquire)) {
-        cudaError_t e = cudaFuncSetAttribute(decode_band_kernel<FMT, SCL, XH, NG, TPW>,
+        cudaError_t e = cudaFuncSetAttribute(decode_band_kernel<FMT, SCL, XH, NG, TPW, FUSE>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, db::kMaxSmem);
         if (e != cudaSuccess) return e;
         attr_done[dev].store(true, std::memory_order_release);
     }
     auto enc = encode_fn_db();
     if (!enc) return cudaErrorNotSupported;
-    // packed weights as bytes [E*N, K/2]: boxes of 128 bytes x 64 rows, 128B swizzle
+    // packed weights as bytes [E*N, K/2]: boxes of 128 bytes x 64 rows (x 32 rows, two a
+    // stage, for the fused SwiGLU), 128B swizzle
     CUtensorMap wmap;
     cuuint64_t dims[2] = {(cuuint64_t)(a.K / 2), (cuuint64_t)a.E * (cuuint64_t)a.N};
     cuuint64_t strides[1] = {(cuuint64_t)(a.K / 2)};
-    cuuint32_t box[2] = {(cuuint32_t)db::kBoxBytes, (cuuint32_t)db::kTileRows};
+    cuuint32_t box[2] = {(cuuint32_t)db::kBoxBytes, (cuuint32_t)(FUSE ? db::kTileRows / 2 : db::kTileRows)};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.W), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     const int grid = device_sm_count();
-    decode_band_kernel<FMT, SCL, XH, NG, TPW><<<grid, 512 / TPW, bytes, s>>>(a, pl, wmap);
+    decode_band_kernel<FMT, SCL, XH, NG, TPW, FUSE><<<grid, 512 / TPW, bytes, s>>>(a, pl, wmap);
     return cudaGetLastError();
 }
 
-cudaError_t launch_decode_band(int fmt, const GroupedArgs& a, cudaStream_t s) {
+cudaError_t launch_decode_band(int fmt, const GroupedArgs& a, cudaStream_t s, bool fuse_swiglu) {
     db::Plan pl;
     const int SB = (fmt == FMT_NF4) ? 64 : 32;
     pl.nblk = a.K / SB;
@@ -898,6 +950,19 @@ cudaError_t launch_decode_band(int fmt, const GroupedArgs& a, cudaStream_t s) {
     // group either way), so the choice never changes a result.
     const int64_t mmax = a.R < (int64_t)a.m_hi ? a.R : (int64_t)a.m_hi;      // no group exceeds this
     const bool one = mmax <= 8 || a.R < 4 * (int64_t)a.E;
+    if (fuse_swiglu) {
+        // gate tile and up tile in one warp: two tiles a warp for both formats
+        if (fmt == FMT_NF4) {
+            if (a.scale_bf16) {
+                if (a.x_f16) return one ? launch_db<FMT_NF4, db::SC_BF16, 1, 1, 2, 1>(a, pl, s) : launch_db<FMT_NF4, db::SC_BF16, 1, 2, 2, 1>(a, pl, s);
+                return one ? launch_db<FMT_NF4, db::SC_BF16, 0, 1, 2, 1>(a, pl, s) : launch_db<FMT_NF4, db::SC_BF16, 0, 2, 2, 1>(a, pl, s);
+            }
+            if (a.x_f16) return one ? launch_db<FMT_NF4, db::SC_F32, 1, 1, 2, 1>(a, pl, s) : launch_db<FMT_NF4, db::SC_F32, 1, 2, 2, 1>(a, pl, s);
+            return one ? launch_db<FMT_NF4, db::SC_F32, 0, 1, 2, 1>(a, pl, s) : launch_db<FMT_NF4, db::SC_F32, 0, 2, 2, 1>(a, pl, s);
+        }
+        if (a.x_f16) return one ? launch_db<FMT_MXFP4, db::SC_E8M0, 1, 1, 2, 1>(a, pl, s) : launch_db<FMT_MXFP4, db::SC_E8M0, 1, 2, 2, 1>(a, pl, s);
+        return one ? launch_db<FMT_MXFP4, db::SC_E8M0, 0, 1, 2, 1>(a, pl, s) : launch_db<FMT_MXFP4, db::SC_E8M0, 0, 2, 2, 1>(a, pl, s);
+    }
     // NF4 (4 blocks a chunk): two tiles a warp, 8 warps; MXFP4 (8 blocks a chunk, twice
     // the code and registers per tile): one tile a warp, 16 warps (measured faster each)
     if (fmt == FMT_NF4) {

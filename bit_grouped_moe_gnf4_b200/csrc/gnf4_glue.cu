@@ -41,26 +41,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return d;
 }
 
-// e^x for x <= 0 as 2^(x log2 e) on the hardware base-2 exponential (ex2.approx.f32:
-// about 2^-22 relative error, subnormal results kept). Rounding x log2 e to fp32 adds
-// at most 2^-24 |x log2 e| to the exponent, i.e. 2^-17.5 relative for |x| <= 88 (below
-// that the result is subnormal and only the absolute error matters).
-__device__ __forceinline__ float exp_via_ex2(float x) {
-    float y;
-    asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x * 1.4426950408889634f));
-    return y;
-}
-
-// silu(g) = g * sigmoid(g), with e = exp(-|g|) in (0, 1] so that nothing overflows:
-// sigmoid(g) = 1 / (1 + e) for g >= 0 and e / (1 + e) for g < 0. The divisor is in
-// [1, 2], where the fast division is within 2 ulp. For g far below zero g * e underflows
-// gradually, as the exact value does.
-__device__ __forceinline__ float silu_mul(float g, float u) {
-    const float e = exp_via_ex2(-fabsf(g));
-    const float num = g >= 0.0f ? g : g * e;
-    return __fdividef(num, 1.0f + e) * u;
-}
-
 __device__ __forceinline__ uint32_t swiglu_word(uint32_t g, uint32_t u) {
     return pack_bf16x2(silu_mul(bf16_lo(g), bf16_lo(u)), silu_mul(bf16_hi(g), bf16_hi(u)));
 }

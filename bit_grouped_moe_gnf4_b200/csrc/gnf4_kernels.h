@@ -13,9 +13,10 @@ cudaError_t launch_quantize_nf4(const float* w, int64_t rows, int64_t K, uint8_t
 cudaError_t launch_quantize_mxfp4(const float* w, int64_t rows, int64_t K, uint8_t* blocks,
                                   uint8_t* scales, cudaStream_t s);
 
-// Decode band: register-decoded warp MMAs, K split across the warps of a CTA.
-// Takes the groups whose row count m satisfies a.m_lo <= m <= a.m_hi.
-cudaError_t launch_decode_band(int fmt, const GroupedArgs& a, cudaStream_t s);
+// Decode band: TMA-fed warp MMAs over table-decoded nibbles. Takes the groups whose
+// row count m satisfies a.m_lo <= m <= a.m_hi. fuse_swiglu: a.N is the fused gate_up
+// width 2I and the output [.., I] holds silu(gate) * up.
+cudaError_t launch_decode_band(int fmt, const GroupedArgs& a, cudaStream_t s, bool fuse_swiglu = false);
 
 // Prefill band: tcgen05 MMAs into tensor memory with the per-block fp32
 // rescale outside the MMA. Takes the groups with a.m_lo <= m <= a.m_hi.

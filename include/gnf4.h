@@ -183,6 +183,35 @@ gnf4_status gnf4_grouped_gemm_mxfp4_ex(const void* x, int x_dtype, const uint8_t
                                        void* out, int flags, void* stream);
 
 /*
+ * gate_up grouped GEMM with the SwiGLU fused into its epilogue: the step between the
+ * gate_up and down projections of a SwiGLU MoE layer (the decode glue "swiglu_rows" of
+ * the status page "MoE Software Status & Known Limits", "Correctness contracts"; the
+ * SwiGLU architectures of the experts4bit-qlora README, "Scope") done where the gate_up
+ * sums are still fp32 in registers, so the [R, 2I] gate_up rows never reach memory.
+ * For routed row r, with G and U the gate_up call's fp32 results before rounding
+ * (row j of W[e] the gate of column j, row I + j its up; routing weight included):
+ *   out[dest(r), j] = round16( silu(w(r) G[r, j]) * (w(r) U[r, j]) ),  j < I = N / 2
+ * i.e. gnf4_swiglu applied to gnf4_grouped_gemm_*_ex's output without rounding the
+ * gate_up rows in between (silu as in gnf4_swiglu). Arguments as in
+ * gnf4_grouped_gemm_{nf4,mxfp4}_ex, with N = 2I the fused gate_up width (N % 32 == 0)
+ * and out [T_out, I] of the activations' type. Every group runs in the decode band
+ * (one launch; groups above 8 or 16 rows take several passes over their weights), so
+ * for prefill-sized groups the unfused GEMM + gnf4_swiglu is the faster pair.
+ * flags: 0, GNF4_CHECK or GNF4_FORCE_DECODE (a no-op); GNF4_FORCE_PREFILL is refused.
+ * Errors: as for the grouped GEMM; UNSUPPORTED_SHAPE if N % 32.
+ */
+gnf4_status gnf4_grouped_gemm_swiglu_nf4(const void* x, int x_dtype, const uint8_t* W, const void* absmax,
+                                         int absmax_dtype, const int64_t* expert_offsets,
+                                         const int32_t* row_token, const float* row_weight,
+                                         const int32_t* row_dest, int64_t E, int64_t N, int64_t K, int64_t R,
+                                         int64_t T_in, int64_t T_out, void* out, int flags, void* stream);
+gnf4_status gnf4_grouped_gemm_swiglu_mxfp4(const void* x, int x_dtype, const uint8_t* W, const uint8_t* scales,
+                                           const int64_t* expert_offsets, const int32_t* row_token,
+                                           const float* row_weight, const int32_t* row_dest, int64_t E,
+                                           int64_t N, int64_t K, int64_t R, int64_t T_in, int64_t T_out,
+                                           void* out, int flags, void* stream);
+
+/*
  * The lossless absmax cast of the bf16-absmax storage (README 0.11.0, "Which entry
  * point?", the --absmax-dtype bf16 paragraph: the cast refuses rather than rounds).
  * absmax_bf16[i] = the bf16 pattern of absmax[i] (its high 16 bits); an fp32 value
