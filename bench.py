@@ -62,6 +62,8 @@ def parse():
                          "bf16 source, so the cast is lossless)")
     ap.add_argument("--x-dtype", default="bf16", choices=["bf16", "f16"],
                     help="activations (and output) type")
+    ap.add_argument("--unfused-swiglu", action="store_true",
+                    help="--op layer: run gate_up and the SwiGLU as two kernels (default: fused)")
     ap.add_argument("--no-sub-records", action="store_true",
                     help="default workload only: skip the prefill and MXFP4 sub-records")
     ap.add_argument("--top-k", type=int, default=None, help="sweep workload: top_k (default first)")
@@ -991,11 +993,16 @@ def run_layer_bench(args, wl):
         nbytes = call_bytes(wl.fmt, gu, b)[0] + call_bytes(wl.fmt, dn, b)[0]
         layers.append((T, d, nbytes, b))
 
+    fused = not args.unfused_swiglu
+
     def layer(d, T):
         st = torch.cuda.current_stream()
         off, tok, wt, dst = g.routing_metadata(d["ids"], d["w"], wl.E, stream=st)
-        g.grouped_gemm(wl.fmt, d["x"], Wg, Sg, off, row_token=tok, out=d["h"], R=T * k, stream=st)
-        g.swiglu(d["h"], out=d["a"], stream=st)
+        if fused:       # gate_up with the SwiGLU in its epilogue: no [R, 2I] round trip
+            g.grouped_gemm_swiglu(wl.fmt, d["x"], Wg, Sg, off, row_token=tok, out=d["a"], R=T * k, stream=st)
+        else:
+            g.grouped_gemm(wl.fmt, d["x"], Wg, Sg, off, row_token=tok, out=d["h"], R=T * k, stream=st)
+            g.swiglu(d["h"], out=d["a"], stream=st)
         g.grouped_gemm(wl.fmt, d["a"], Wd, Sd, off, row_weight=wt, row_dest=dst, out=d["y"], R=T * k, stream=st)
         g.combine_topk(d["y"], T, k, out=d["out"], stream=st)
 
@@ -1037,8 +1044,9 @@ def run_layer_bench(args, wl):
             "warmup": args.warmup, "ms_per_step": float(ms.sum()), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": "layer of " + describe(wl, k), "l2": "flushed (256 MB write) before each layer",
+                       "swiglu": "fused into the gate_up epilogue" if fused else "separate kernel",
                        "layers": [f"T={T}" for T, _, _, _ in layers]},
-            "gpu_launches": 5 * len(layers) * args.steps,
+            "gpu_launches": (4 if fused else 5) * len(layers) * args.steps,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                          "peak_source": f"{src} HBM copy", "traffic": None,
                          "note": "packed-weight bytes of both projections over the whole layer's time",

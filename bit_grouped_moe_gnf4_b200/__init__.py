@@ -8,7 +8,7 @@ it is missing -- there is no fallback implementation.
 _API = ("quantize_nf4", "quantize_mxfp4", "grouped_gemm", "grouped_gemm_nf4", "grouped_gemm_mxfp4",
         "launches_per_call", "device_status", "version", "swiglu", "combine_topk", "dgrad", "routing_metadata",
         "absmax_to_bf16", "grouped_gemm_swiglu")
-_LIB = ("Gnf4Error", "GNF4_CHECK", "GNF4_FORCE_DECODE", "GNF4_FORCE_PREFILL", "GNF4_DTYPE_BF16", "GNF4_DTYPE_F16",
+_LIB = ("Gnf4Error", "GNF4_CHECK", "GNF4_FORCE_DECODE", "GNF4_FORCE_PREFILL", "GNF4_TEST_STALL", "GNF4_DTYPE_BF16", "GNF4_DTYPE_F16",
         "GNF4_DTYPE_F32")
 
 __all__ = list(_API + _LIB)

@@ -21,6 +21,7 @@ GNF4_ERR_DEVICE_STATUS = 5
 GNF4_CHECK = 0x1
 GNF4_FORCE_DECODE = 0x2
 GNF4_FORCE_PREFILL = 0x4
+GNF4_TEST_STALL = 0x100
 
 GNF4_DTYPE_BF16 = 0
 GNF4_DTYPE_F16 = 1

@@ -217,8 +217,10 @@ static gnf4_status grouped(int fmt, const void* x, int x_dtype, const uint8_t* W
     if (!x || !W || !scales || !offsets || !out) return fail(GNF4_ERR_INVALID_ARG, "null pointer argument");
     if (E < 1 || N < 1 || K < 1 || R < 0 || T_in < 0 || T_out < 0)
         return fail(GNF4_ERR_INVALID_ARG, "sizes must be E,N,K >= 1 and R,T_in,T_out >= 0");
-    if (flags & ~(GNF4_CHECK | GNF4_FORCE_DECODE | GNF4_FORCE_PREFILL))
+    if (flags & ~(GNF4_CHECK | GNF4_FORCE_DECODE | GNF4_FORCE_PREFILL | GNF4_TEST_STALL))
         return fail(GNF4_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+    if ((flags & GNF4_TEST_STALL) && (flags & GNF4_FORCE_PREFILL))
+        return fail(GNF4_ERR_INVALID_ARG, "GNF4_TEST_STALL runs the decode band only");
     if ((flags & GNF4_FORCE_DECODE) && (flags & GNF4_FORCE_PREFILL))
         return fail(GNF4_ERR_INVALID_ARG, "GNF4_FORCE_DECODE and GNF4_FORCE_PREFILL exclude each other");
     if (K % kmul) return fail(GNF4_ERR_UNSUPPORTED_SHAPE, "K must be a multiple of %lld", (long long)kmul);
@@ -265,6 +267,7 @@ static gnf4_status grouped(int fmt, const void* x, int x_dtype, const uint8_t* W
     static const LutPlanes lut_nf4 = make_lut(FMT_NF4, 0), lut_nf4_h = make_lut(FMT_NF4, 1);
     static const LutPlanes lut_mx = make_lut(FMT_MXFP4, 0), lut_mx_h = make_lut(FMT_MXFP4, 1);
     a.x_f16 = (x_dtype == GNF4_DTYPE_F16) ? 1 : 0;
+    a.test_stall = (flags & GNF4_TEST_STALL) ? 1 : 0;
     a.scale_bf16 = (fmt == FMT_NF4 && scale_dtype == GNF4_DTYPE_BF16) ? 1 : 0;
     a.lut = (fmt == FMT_NF4) ? (a.x_f16 ? lut_nf4_h : lut_nf4) : (a.x_f16 ? lut_mx_h : lut_mx);
 
@@ -287,7 +290,7 @@ static gnf4_status grouped(int fmt, const void* x, int x_dtype, const uint8_t* W
     // band split by rows per group; decided on the device from the offsets
     int split = kDecodeMaxRows;
     if (R <= kDecodeOnlyRows) split = INT_MAX;
-    if (flags & GNF4_FORCE_DECODE) split = INT_MAX;
+    if (flags & (GNF4_FORCE_DECODE | GNF4_TEST_STALL)) split = INT_MAX;
     if (flags & GNF4_FORCE_PREFILL) split = 0;
 #ifndef GNF4_HAVE_PREFILL
     split = INT_MAX;
@@ -553,7 +556,7 @@ int gnf4_grouped_gemm_launches(int64_t R, int flags) {
     if (R <= 0) return 0;
     int n = (flags & GNF4_CHECK) ? 1 : 0;
 #ifdef GNF4_HAVE_PREFILL
-    if (flags & GNF4_FORCE_DECODE) return n + 1;
+    if (flags & (GNF4_FORCE_DECODE | GNF4_TEST_STALL)) return n + 1;
     if (flags & GNF4_FORCE_PREFILL) return n + 1;
     return n + 1 + (R > kDecodeOnlyRows ? 1 : 0);
 #else

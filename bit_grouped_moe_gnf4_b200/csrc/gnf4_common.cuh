@@ -32,6 +32,7 @@ struct GroupedArgs {
     int E, N, K;
     int m_lo, m_hi;             // this band takes groups with m_lo <= rows <= m_hi
     int x_f16;                  // activations and output: 0 bf16, 1 fp16
+    int test_stall;             // testing: the decode band issues no copies and waits at most 2^17 cycles
     int scale_bf16;             // NF4 absmax stored as bf16 (1) or fp32 (0)
     LutPlanes lut;              // codebook in the activations' 16-bit type
 };
@@ -178,14 +179,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uin
 // has given up) it records `code` in *err, raises the CTA's abort flag and
 // returns false. The clock and the flag are polled only every 8th attempt.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                                  unsigned* err, unsigned code) {
+                                                  unsigned* err, unsigned code,
+                                                  long long limit = kWaitTimeoutCycles) {
     if (mbar_try_wait(bar, parity, 0u)) return true;
     const long long t0 = clock64();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity, 2000u)) return true;
         if ((it & 7u) == 0u) {
             if (*abort_flag) return false;
-            if (clock64() - t0 > kWaitTimeoutCycles) {
+            if (clock64() - t0 > limit) {
                 *abort_flag = 1;
                 atomicOr(err, code);
                 return false;

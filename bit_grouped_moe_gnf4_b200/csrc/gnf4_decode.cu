@@ -87,6 +87,10 @@ constexpr int kLutBytes = 256 * 256;           // byte b, lane l -> b*256 + l*4 
 constexpr int kMaxTableRows = 1024;            // routed rows whose metadata the CTA stages in shared memory
 constexpr int kMaxSmem = 227 * 1024;
 
+// independent MMA chains per scale block (their sums are added in order afterwards)
+#ifndef GNF4_DB_CHAINS
+#define GNF4_DB_CHAINS 1
+#endif
 // most K parts of a tile (a power of two, at most kQuads)
 #ifndef GNF4_DB_MAXPARTS
 #define GNF4_DB_MAXPARTS 2
@@ -313,14 +317,18 @@ __device__ __forceinline__ void chunk_math(const uint32_t (&rowa)[TPW], const ui
             uint32_t (&xw)[NGC][XW] = (b & 1) ? xb : xa;
             uint32_t (&xn)[NGC][XW] = (b & 1) ? xa : xb;
             if (b + 1 < G::NB && (FULL || b + 1 < nb)) load_x(xn, b + 1);
-            float c[TPW][NGC][4];
+            // CH independent MMA chains per block, tile and group (the block's k16 steps dealt
+            // round robin), added in chain order: the same for every group count and tile
+            // count, so a row's sum never depends on what shares its pass. The A operand of
+            // step st is bytes 2st and 2st + 1 of rows ra and rb, decoded in operand order.
+            constexpr int CH = GNF4_DB_CHAINS < STEPS ? GNF4_DB_CHAINS : STEPS;
+            float c[TPW][NGC][CH][4];
 #pragma unroll
             for (int tt = 0; tt < TPW; ++tt)
 #pragma unroll
-                for (int j = 0; j < NGC; ++j) c[tt][j][0] = c[tt][j][1] = c[tt][j][2] = c[tt][j][3] = 0.f;
-            // one MMA chain per block, tile and group, the same for every group count and
-            // tile count, so a row's sum never depends on what shares its pass. The A operand
-            // of step st is bytes 2st and 2st + 1 of rows ra and rb, decoded in operand order.
+                for (int j = 0; j < NGC; ++j)
+#pragma unroll
+                    for (int h = 0; h < CH; ++h) c[tt][j][h][0] = c[tt][j][h][1] = c[tt][j][h][2] = c[tt][j][h][3] = 0.f;
 #pragma unroll
             for (int st = 0; st < STEPS; ++st) {
 #pragma unroll
@@ -331,19 +339,27 @@ __device__ __forceinline__ void chunk_math(const uint32_t (&rowa)[TPW], const ui
                     const uint32_t a3 = lut_lookup(w[tt][1][G::LW * b + ((2 * st + 1) >> 2)], lane_sel, (2 * st + 1) & 3);
 #pragma unroll
                     for (int j = 0; j < NGC; ++j)
-                        mma16816<XH>(c[tt][j], a0, a1, a2, a3, xw[j][2 * st], xw[j][2 * st + 1]);
+                        mma16816<XH>(c[tt][j][st % CH], a0, a1, a2, a3, xw[j][2 * st], xw[j][2 * st + 1]);
                 }
             }
+#pragma unroll
+            for (int tt = 0; tt < TPW; ++tt)
+#pragma unroll
+                for (int j = 0; j < NGC; ++j)
+#pragma unroll
+                    for (int h = 1; h < CH; ++h)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) c[tt][j][0][q] += c[tt][j][h][q];
 #pragma unroll
             for (int tt = 0; tt < TPW; ++tt) {
                 const float sa = scale_of<SCL>(sc[tt].s[0], b);
                 const float sb = scale_of<SCL>(sc[tt].s[1], b);
 #pragma unroll
                 for (int j = 0; j < NGC; ++j) {
-                    acc[tt][j][0] = fmaf(c[tt][j][0], sa, acc[tt][j][0]);
-                    acc[tt][j][1] = fmaf(c[tt][j][1], sa, acc[tt][j][1]);
-                    acc[tt][j][2] = fmaf(c[tt][j][2], sb, acc[tt][j][2]);
-                    acc[tt][j][3] = fmaf(c[tt][j][3], sb, acc[tt][j][3]);
+                    acc[tt][j][0] = fmaf(c[tt][j][0][0], sa, acc[tt][j][0]);
+                    acc[tt][j][1] = fmaf(c[tt][j][0][1], sa, acc[tt][j][1]);
+                    acc[tt][j][2] = fmaf(c[tt][j][0][2], sb, acc[tt][j][2]);
+                    acc[tt][j][3] = fmaf(c[tt][j][0][3], sb, acc[tt][j][3]);
                 }
             }
         }
@@ -392,8 +408,12 @@ __host__ __device__ inline bool make_layout(uint32_t base, uint32_t bytes, int E
     return true;
 }
 
-__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-    return mbar_wait_bounded(bar, parity, abort_flag, &g_decode_error, 1u);
+// the stall test's limit: long enough for nothing, short enough to end the test fast
+constexpr long long kStallTestWaitCycles = 1LL << 17;
+
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag, bool stall_test) {
+    return mbar_wait_bounded(bar, parity, abort_flag, &g_decode_error, 1u,
+                             stall_test ? kStallTestWaitCycles : kWaitTimeoutCycles);
 }
 
 }  // namespace db
@@ -522,7 +542,10 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     const int64_t s8 = 8 * (int64_t)pl.nblk * SSZ;
     const bool vec = pl.vec_scales != 0;
     const uint8_t* Sb = reinterpret_cast<const uint8_t*>(p.scales);
-    const bool issuer = (wq == 0 && lane == 0);     // issues the quad's copies
+    // the stall test (a documented test flag) issues no copy at all: every first wait for
+    // a stage gives up after a short limit, and the abort path runs with nothing in flight
+    const bool stall_test = p.test_stall != 0;
+    const bool issuer = (wq == 0 && lane == 0) && !stall_test;   // issues the box's copies
     uint64_t* full = bars + quad * kStages;
     uint64_t* empty = bars + kQuads * kStages + quad * kStages;
     const uint32_t qring = quad == 0 ? lay.ring[0] : quad == 1 ? lay.ring[1] : quad == 2 ? lay.ring[2] : lay.ring[3];
@@ -793,7 +816,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
         for (int tt = 0; tt < kTPW; ++tt) use[tt] = scN[tt];
         scales_next(scN);
         if (mt_ck == 0) unit_begin();
-        if (!dead && !wait_bounded(smem_addr(full + cs), cph, abort_flag)) dead = true;
+        if (!dead && !wait_bounded(smem_addr(full + cs), cph, abort_flag, stall_test)) dead = true;
         if (!dead && ntl > 0) {
             const int c = c_lo + mt_ck;
             uint32_t rowa[kTPW];
@@ -823,7 +846,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
         // the issuing lane refills the oldest stage once every warp of the box released it
         // (the chunk kStages before the one it now receives)
         if (issuer && cp_left > 0 && cp_j >= kStages) {
-            if (!dead && !wait_bounded(smem_addr(empty + rs), rph, abort_flag)) dead = true;
+            if (!dead && !wait_bounded(smem_addr(empty + rs), rph, abort_flag, stall_test)) dead = true;
             if (!dead) issue_next();
             if (++rs == kStages) {
                 rs = 0;

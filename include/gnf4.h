@@ -44,6 +44,12 @@ typedef enum gnf4_status {
                                     results as long as fewer than 256 are in flight */
 #define GNF4_FORCE_DECODE   0x2  /* run every group through the decode band (testing) */
 #define GNF4_FORCE_PREFILL  0x4  /* run every group through the prefill band (testing) */
+#define GNF4_TEST_STALL   0x100  /* testing the error path: every group runs in the decode
+                                    band, which issues none of its weight copies and waits at
+                                    most 2^17 cycles, so its first wait gives up; the kernel
+                                    records the event, skips the math and returns. The output
+                                    is unspecified and gnf4_device_status then reports
+                                    GNF4_ERR_DEVICE_STATUS; the next call runs normally */
 
 /* storage types of the *_ex entry points */
 #define GNF4_DTYPE_BF16 0    /* bfloat16 */

@@ -316,3 +316,50 @@ def test_host_pointers_are_refused():
     with pytest.raises(g.Gnf4Error) as ei:
         g.grouped_gemm("nf4", x_host, Wd, Sd, to_dev(np.array([0, 2, 4], np.int64)), R=4)
     assert ei.value.status == 1
+
+
+def test_bounded_wait_abort_path_reports_and_recovers():
+    """GNF4_TEST_STALL: the decode band issues no weight copy, so every wait for a stage
+    gives up after a short limit; the kernel records it, skips the math and drains
+    nothing (nothing was issued). gnf4_device_status reports it once, and the next call
+    on the same context returns correct results."""
+    import bit_grouped_moe_gnf4_b200 as g
+    E, k, T, K, N = 4, 2, 8, 256, 128
+    Wd, Sd, Wh, Sh = build_stack("nf4", E, N, K)
+    b = synth.make_routed_batch(0, T, E, k)
+    x = synth.activations_bf16(0, T, K)
+    args = dict(row_token=to_dev(b.row_token), row_weight=to_dev(b.row_weight), row_dest=to_dev(b.row_dest))
+    for fused in (False, True):
+        fn = g.grouped_gemm_swiglu if fused else g.grouped_gemm
+        fn("nf4", bf16_dev(x), Wd, Sd, to_dev(b.offsets), T_out=T * k, flags=g.GNF4_TEST_STALL, **args)
+        with pytest.raises(g.Gnf4Error) as ei:
+            g.device_status()
+        assert ei.value.status == 5
+        g.device_status()                                # the record was cleared
+    out = run_gemm("nf4", x, Wd, Sd, b.offsets, b.row_token, b.row_weight, b.row_dest, T_out=T * k)
+    ref = O.grouped_rows_f64("nf4", x, Wh, Sh, b.offsets, b.row_token, b.row_weight, K, np.arange(b.R))
+    check_rows(out[b.row_dest], ref, "after the stall test")
+
+
+def test_default_mode_row_count_invariance():
+    """A token's rows keep their bits whether it is routed alone or inside 16-, 17- and
+    160-token calls with softmax top-8 routing, in the default band choice: every group
+    of these calls has at most 64 rows, so every row runs in the decode band, whose fp32
+    summation order depends on K alone."""
+    import bit_grouped_moe_gnf4_b200 as g
+    wl = WORKLOADS["olmoe_decode_nf4"]
+    gu = wl.projections[0]
+    E, k = wl.E, 8
+    ids, w = G.route_softmax_topk(11, 160, E, k)
+    x_all = synth.activations_bf16(12, 160, gu.K)
+    Wd, Sd, _, _ = build_stack("nf4", E, gu.N, gu.K, seed=0, oracle_experts=[int(e) for e in ids[0]])
+    rows0 = []
+    for T in (1, 16, 17, 160):
+        off, tok, wt, dst = G.routing_metadata(ids[:T].astype(np.int32), w[:T], E)
+        assert np.diff(off).max() <= 64
+        out = g.grouped_gemm("nf4", bf16_dev(x_all[:T]), Wd, Sd, to_dev(off), row_token=to_dev(tok),
+                             row_dest=to_dev(dst), T_out=T * k)
+        rows0.append(bf16_host_bits(out)[:k])             # token 0's k slots
+    g.device_status()
+    for r in rows0[1:]:
+        assert np.array_equal(r, rows0[0])
