@@ -15,7 +15,10 @@ namespace gnf4 {
 
 // Groups with more than this many routed rows go to the prefill (tensor-core)
 // band; the rest to the decode band.
-constexpr int kDecodeMaxRows = 64;
+#ifndef GNF4_DECODE_MAX_ROWS
+#define GNF4_DECODE_MAX_ROWS 64
+#endif
+constexpr int kDecodeMaxRows = GNF4_DECODE_MAX_ROWS;
 // at most this many routed rows in the whole call: every group runs in the decode band
 // (at most one group can exceed kDecodeMaxRows, and a second launch costs more than
 // the decode band's extra passes over that group)

@@ -425,9 +425,15 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
                 // (waits are made warp-uniform: the tensor-memory stores below need the whole warp)
                 if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_wfull + 8 * wslot, wph, abort_flag, err, 32u)))
                     goto dec_done;
+                // the row's 32 bytes as two 16-byte halves; lanes 4..7 of every 8 read the second
+                // half first, so that the 8 rows of a group of lanes cover all 32 banks and
+                // each load is 4 wavefronts (rows are 32 bytes apart)
                 const uint8_t* wrow = smem + kOffW + wslot * kWStageBytes + i * 32;
-                const uint4 c0 = *reinterpret_cast<const uint4*>(wrow);
-                const uint4 c1 = *reinterpret_cast<const uint4*>(wrow + 16);
+                const int sw = (lane >> 2) & 1;
+                const uint4 q0 = *reinterpret_cast<const uint4*>(wrow + 16 * sw);
+                const uint4 q1 = *reinterpret_cast<const uint4*>(wrow + 16 * (sw ^ 1));
+                const uint4 c0 = sw ? q1 : q0;
+                const uint4 c1 = sw ? q0 : q1;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_wempty + 8 * wslot);
                 const uint32_t slot = stage_ctr % kStages, ph = ((stage_ctr / kStages) & 1u) ^ 1u;
