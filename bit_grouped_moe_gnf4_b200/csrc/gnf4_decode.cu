@@ -72,7 +72,10 @@ namespace db {
 // A warp computes TPW tiles of 16 rows per chunk (1 or 2, a kernel template
 // parameter): the 64-row box of a unit is shared by 4 / TPW warps, and a CTA has
 // kQuads boxes in flight side by side (one ring each), so 16 / TPW warps.
-constexpr int kQuads = 4;
+#ifndef GNF4_DB_BOXES
+#define GNF4_DB_BOXES 4
+#endif
+constexpr int kQuads = GNF4_DB_BOXES;
 constexpr int kMaxWarps = 16;
 constexpr int kTileRows = 64;                  // weight rows of a unit: 16 per warp of a quad
 constexpr int kChunkK = 256;                   // K per chunk: 128 packed bytes of every row
@@ -419,10 +422,11 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
 }  // namespace db
 
 template <int FMT, int SCL, int XH, int NG, int TPW, int FUSE>
-__global__ void __launch_bounds__(512 / TPW, 1)
+__global__ void __launch_bounds__(db::kQuads * 128 / TPW, 1)
 decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant__ CUtensorMap wmap) {
     using namespace db;
     static_assert(!FUSE || TPW == 2, "the fused SwiGLU pairs a gate tile with its up tile in one warp");
+    static_assert(2 * kQuads * 4 * NG * 32 <= 256 * 8, "the part-sum slots must fit the table's spare halves");
     constexpr int kTPW = TPW;
     // FUSE: a unit is 32 gate rows [n0, n0 + 32) and their up rows [I + n0, I + n0 + 32) of
     // the fused gate_up matrix (two 32-row boxes per stage: gate in stage rows 0..31, up in
@@ -548,7 +552,10 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     const bool issuer = (wq == 0 && lane == 0) && !stall_test;   // issues the box's copies
     uint64_t* full = bars + quad * kStages;
     uint64_t* empty = bars + kQuads * kStages + quad * kStages;
-    const uint32_t qring = quad == 0 ? lay.ring[0] : quad == 1 ? lay.ring[1] : quad == 2 ? lay.ring[2] : lay.ring[3];
+    uint32_t qring = lay.ring[0];
+#pragma unroll
+    for (int q = 1; q < kQuads; ++q)
+        if (quad == q) qring = lay.ring[q];
 
     // unit u -> (active expert a, first weight row n0, first routed row of the pass mc);
     // a only moves forward along a quad's units, so it is found by walking
@@ -949,7 +956,7 @@ static cudaError_t launch_db(const GroupedArgs& a, db::Plan& pl, cudaStream_t s)
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     const int grid = device_sm_count();
-    decode_band_kernel<FMT, SCL, XH, NG, TPW, FUSE><<<grid, 512 / TPW, bytes, s>>>(a, pl, wmap);
+    decode_band_kernel<FMT, SCL, XH, NG, TPW, FUSE><<<grid, db::kQuads * 128 / TPW, bytes, s>>>(a, pl, wmap);
     return cudaGetLastError();
 }
 
