@@ -557,8 +557,22 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     for (int q = 1; q < kQuads; ++q)
         if (quad == q) qring = lay.ring[q];
 
+    // the active expert that holds unit u: the last a with s_up[a] <= u (s_up rises
+    // strictly: every active expert has at least one unit); a binary search, so that a
+    // CTA late in the band does not walk every expert before it
+    auto find_active = [&](int64_t u) -> int {
+        int lo = 0, hi = nact - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_up[mid] <= u) lo = mid;
+            else hi = mid - 1;
+        }
+        return lo;
+    };
+    const int a_first = find_active(U0);             // the expert of the CTA's first unit
+
     // unit u -> (active expert a, first weight row n0, first routed row of the pass mc);
-    // a only moves forward along a quad's units, so it is found by walking
+    // a only moves forward along a quad's units (from a_first), so it is found by walking
     auto locate = [&](int64_t u, int& a, int& n0, int& mc) {
         while (s_up[a + 1] <= u) ++a;
         const int m = s_m[a];
@@ -574,7 +588,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     };
 
     // copy cursor (issuing lane only): chunk j of the quad's sequence into stage j % kStages
-    int cp_left = nsteps, cp_c = c_lo, cp_a = 0, cp_y = 0, cp_j = 0, cp_s = 0;
+    int cp_left = nsteps, cp_c = c_lo, cp_a = a_first, cp_y = 0, cp_j = 0, cp_s = 0;
     int64_t cp_u = U0 + gi;
     auto cp_unit = [&]() {
         int n0, mc;
@@ -601,7 +615,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     }
 
     // scale cursor (every warp, its own rows): one chunk ahead of the math
-    int sc_left = nsteps, sc_c = c_lo, sc_a = 0;
+    int sc_left = nsteps, sc_c = c_lo, sc_a = a_first;
     int64_t sc_u = U0 + gi;
     const uint8_t* sc_p[kTPW];
     auto sc_unit = [&]() {
@@ -650,9 +664,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     int64_t rlo = 0;
     bool table = false;
     {
-        int a0 = 0, a1 = 0, n0, mc;
-        locate(U0, a0, n0, mc);
-        locate(U1 - 1, a1, n0, mc);
+        const int a0 = a_first, a1 = find_active(U1 - 1);
         rlo = s_r0[a0];
         const int64_t rhi = s_r0[a1] + s_m[a1];
         table = (rhi - rlo) <= kMaxTableRows;
@@ -687,7 +699,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     };
 
     // ---- math cursor ----
-    int mt_ck = 0, mt_a = 0, mt_n0 = 0, mt_mc = 0, mt_unit = 0, nvalid = 0, ng = 0;
+    int mt_ck = 0, mt_a = a_first, mt_n0 = 0, mt_mc = 0, mt_unit = 0, nvalid = 0, ng = 0;
     int64_t mt_u = U0 + gi, mt_r0 = 0;
     int ntl = 0;                                    // this warp's tiles that exist in the unit (rows < N)
     float acc[kTPW][NG][4];
