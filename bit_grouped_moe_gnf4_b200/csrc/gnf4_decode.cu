@@ -436,6 +436,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     constexpr int kBoxWarps = 4 / TPW;              // warps reading one box
     constexpr int kWarps = kQuads * kBoxWarps;
     constexpr int kThreads = kWarps * 32;
+    static_assert(kWarps <= kMaxWarps, "the scan scratch holds one word per warp");
     using G = ChunkGeom<FMT>;
     constexpr int SSZ = (SCL == SC_F32) ? 4 : (SCL == SC_BF16) ? 2 : 1;   // bytes per scale
 
@@ -477,6 +478,36 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap)) : "memory");
     }
+    // the lookup table comes from the kernel parameters alone, so it is built before
+    // anything is read from global memory: under a programmatic dependent launch this
+    // overlaps the tail of the kernel before; the wait below is the first point where
+    // that kernel's results (offsets, routing rows, activations, even weights) are read
+    {
+        const LutPlanes L = p.lut;
+        if constexpr (kWarps == 8 || kWarps == 16 || kWarps == 32) {
+            // each of the 256 entries computed once (warp w % 8 owns bytes 32 (w % 8) ..
+            // + 31, one a lane), then handed by shuffle to the lanes that store it: a store
+            // instruction writes four entries' 128-byte rows, eight lanes a row (no conflict)
+            constexpr int kShare = kWarps / 8;          // warps sharing one byte range
+            const int wb = warp & 7, half = warp >> 3;
+            const uint32_t v = byte_bf16x2<FMT>((uint32_t)(32 * wb + lane), L);
+#pragma unroll
+            for (int k = half * (8 / kShare); k < (half + 1) * (8 / kShare); ++k) {
+                const uint32_t u = __shfl_sync(0xffffffffu, v, 4 * k + (lane >> 3));
+                const int b = 32 * wb + 4 * k + (lane >> 3), q = lane & 7;
+                *reinterpret_cast<uint4*>(lut + b * 256 + q * 16) = make_uint4(u, u, u, u);
+            }
+        } else {
+            for (int i = tid; i < 256 * 8; i += kThreads) {
+                const int b = i >> 3, q = i & 7;
+                const uint32_t v = byte_bf16x2<FMT>((uint32_t)b, L);
+                *reinterpret_cast<uint4*>(lut + b * 256 + q * 16) = make_uint4(v, v, v, v);
+            }
+        }
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // the next kernel of the stream may start its own prologue as SMs free up
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     // ---- active experts of this band and their unit counts (every CTA derives the same list) ----
     int nact = 0;
@@ -571,6 +602,25 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     };
     const int a_first = find_active(U0);             // the expert of the CTA's first unit
 
+    // routed rows [rlo, rhi) of the CTA's experts: staged in shared memory when few
+    // enough. Each thread's first row is loaded now, so that the loads do not queue
+    // behind the first weight copies; they land in the table after the copies went out.
+    const int64_t rlo = s_r0[a_first];
+    const int64_t rhi = [&] {
+        const int a1 = find_active(U1 - 1);
+        return s_r0[a1] + s_m[a1];
+    }();
+    const bool table = (rhi - rlo) <= kMaxTableRows;
+    const bool m_have = table && rlo + tid < rhi;
+    int m_tok = 0, m_dst = 0;
+    float m_wt = 0.f;
+    if (m_have) {
+        const int64_t r = rlo + tid;
+        m_tok = p.row_token ? __ldg(p.row_token + r) : (int)r;
+        m_wt = p.row_weight ? __ldg(p.row_weight + r) : 1.f;
+        m_dst = p.row_dest ? __ldg(p.row_dest + r) : (int)r;
+    }
+
     // unit u -> (active expert a, first weight row n0, first routed row of the pass mc);
     // a only moves forward along a quad's units (from a_first), so it is found by walking
     auto locate = [&](int64_t u, int& a, int& n0, int& mc) {
@@ -611,7 +661,9 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     };
     if (issuer && nsteps > 0) {
         cp_unit();
-        for (int j = 0; j < kStages && cp_left > 0; ++j) issue_next();
+        // stage 0 of every ring now, the other stages once the table is up: the grid's
+        // first chunks then land ahead of the rest of the opening burst
+        if (cp_left > 0) issue_next();
     }
 
     // scale cursor (every warp, its own rows): one chunk ahead of the math
@@ -652,33 +704,24 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
         scales_next(scN);
     }
 
-    // ---- lookup table and the CTA's routing metadata, while the first copies fly ----
-    {
-        const LutPlanes L = p.lut;
-        for (int i = tid; i < 256 * 8; i += kThreads) {
-            const int b = i >> 3, q = i & 7;
-            const uint32_t v = byte_bf16x2<FMT>((uint32_t)b, L);
-            *reinterpret_cast<uint4*>(lut + b * 256 + q * 16) = make_uint4(v, v, v, v);
+    // ---- the CTA's routing metadata: the first rows' loads went out before the copies ----
+    if (table) {
+        if (m_have) {
+            t_tok[tid] = m_tok;
+            t_wt[tid] = m_wt;
+            t_dst[tid] = m_dst;
         }
-    }
-    int64_t rlo = 0;
-    bool table = false;
-    {
-        const int a0 = a_first, a1 = find_active(U1 - 1);
-        rlo = s_r0[a0];
-        const int64_t rhi = s_r0[a1] + s_m[a1];
-        table = (rhi - rlo) <= kMaxTableRows;
-        if (table) {
-            for (int64_t r = rlo + tid; r < rhi; r += kThreads) {
-                const int k = (int)(r - rlo);
-                t_tok[k] = p.row_token ? __ldg(p.row_token + r) : (int)r;
-                t_wt[k] = p.row_weight ? __ldg(p.row_weight + r) : 1.f;
-                t_dst[k] = p.row_dest ? __ldg(p.row_dest + r) : (int)r;
-            }
+        for (int64_t r = rlo + kThreads + tid; r < rhi; r += kThreads) {
+            const int k = (int)(r - rlo);
+            t_tok[k] = p.row_token ? __ldg(p.row_token + r) : (int)r;
+            t_wt[k] = p.row_weight ? __ldg(p.row_weight + r) : 1.f;
+            t_dst[k] = p.row_dest ? __ldg(p.row_dest + r) : (int)r;
         }
     }
     __syncthreads();
 
+    if (issuer)
+        while (cp_j < kStages && cp_left > 0) issue_next();
     // selector word of this lane's table lookups, made after the barrier (the volatile
     // move keeps every lookup, which depends on it, below the table fill)
     uint32_t lane_sel;
@@ -968,7 +1011,21 @@ static cudaError_t launch_db(const GroupedArgs& a, db::Plan& pl, cudaStream_t s)
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     const int grid = device_sm_count();
-    decode_band_kernel<FMT, SCL, XH, NG, TPW, FUSE><<<grid, db::kQuads * 128 / TPW, bytes, s>>>(a, pl, wmap);
+    // programmatic dependent launch: the kernel builds its table while the previous
+    // kernel of the stream drains, and waits for it (griddepcontrol.wait) before its
+    // first global read
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)(db::kQuads * 128 / TPW));
+    cfg.dynamicSmemBytes = bytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_band_kernel<FMT, SCL, XH, NG, TPW, FUSE>, a, pl, wmap);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
