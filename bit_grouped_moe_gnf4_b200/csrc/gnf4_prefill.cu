@@ -72,14 +72,19 @@ constexpr int kScaleAhead = 4;       // block scales held ahead in epilogue regi
 constexpr int kOffB = 0;
 constexpr int kOffW = kOffB + kStages * kBStageBytes;
 constexpr int kOffBar = kOffW + kWStages * kWStageBytes;
-constexpr int kNumBars = 3 * kStages + 2 * kWStages + 2 * kAccBufs;
+constexpr int kNumBars = 3 * kStages + 2 * kWStages + 2 * kAccBufs + 1;
 constexpr int kOffTmem = kOffBar + kNumBars * 8;
 constexpr int kOffAbort = kOffTmem + 4;
 constexpr int kOffRows = kOffTmem + 16;                       // int[kBNMax] gathered rows of the loader's tile
 constexpr int kOffList = kOffRows + kBNMax * 4;               // int[kMaxExperts] experts of the band
 constexpr int kOffCum = kOffList + kMaxExperts * 4;           // int[kMaxExperts+1] tile prefix
 constexpr int kOffCount = kOffCum + (kMaxExperts + 1) * 4;
-constexpr int kSmemBytes = kOffCount + 16 + 1024;             // + alignment slack
+// a tile's outputs, staged for the bulk stores: [routed row][weight row] rounded values,
+// two tiles deep (the stores of one tile drain while the next is computed)
+constexpr int kOutRowBytes = kBM * 2;
+constexpr int kOutBufBytes = kBNMax * kOutRowBytes;
+constexpr int kOffOut = (kOffCount + 16 + 127) & ~127;
+constexpr int kSmemBytes = kOffOut + 2 * kOutBufBytes + 1024;  // + alignment slack
 
 struct Tile {
     int e;          // expert
@@ -169,6 +174,18 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
+// shared -> global bulk copy (async proxy), tracked by this thread's bulk groups
+__device__ __forceinline__ void bulk_store(void* gdst, uint32_t ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 ::"l"(reinterpret_cast<uint64_t>(gdst)), "r"(ssrc), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// every bulk group of this thread has finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
@@ -239,6 +256,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
     const uint32_t bar_wempty = bar_wfull + 8 * kWStages;        // [kWStages] decoders -> weight loader
     const uint32_t bar_accfull = bar_wempty + 8 * kWStages;      // [kAccBufs] MMA -> epilogue
     const uint32_t bar_accempty = bar_accfull + 8 * kAccBufs;    // [kAccBufs] epilogue -> MMA
+    const uint32_t bar_ostaged = bar_accempty + 8 * kAccBufs;    // epilogue warps: a tile's outputs are staged
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffTmem);
     int* s_list = reinterpret_cast<int*>(smem + kOffList);
@@ -296,6 +314,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
             mbar_init(bar_accfull + 8 * i, 1);
             mbar_init(bar_accempty + 8 * i, kEpiWarps);
         }
+        mbar_init(bar_ostaged, kEpiWarps);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -468,7 +487,7 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
         const int cq = (warp - kEpiWarp0) >> 2;       // its 16-column chunks: cq and cq + 4
         const int i = q4 * 32 + lane;                 // tile row = tensor-memory lane
         const int nsbk = p.K / SB;                    // scale blocks per row
-        uint32_t acc_ctr = 0;
+        uint32_t acc_ctr = 0, tile_ctr = 0;
         float acc[2][16];
         for (int t = blockIdx.x; t < sch.total; t += gridDim.x) {
             const Tile tl = tile_at(p, sch, t, nnt);
@@ -492,7 +511,8 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
                         if (b + kScaleAhead < nsbk) sring[u] = load_scale<FMT, SBF16>(p.scales, srow + b + kScaleAhead);
                         const uint32_t buf = acc_ctr % kAccBufs, ph = (acc_ctr / kAccBufs) & 1u;
                         ++acc_ctr;
-                        if (!mbar_wait_bounded(bar_accfull + 8 * buf, ph, abort_flag, err, 128u)) goto epi_done;
+                        if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_accfull + 8 * buf, ph, abort_flag, err, 128u)))
+                            goto epi_done;
                         tc_fence_after();
                         const uint32_t taddr = tmem + ((uint32_t)(q4 * 32) << 16) + buf * kBNMax;
 #pragma unroll
@@ -513,7 +533,17 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
                     }
                 }
             }
-            // outputs of this tile: row n, routed rows r0 .. r0+cnt-1
+            // outputs of this tile: weight row n of routed rows r0 .. r0+cnt-1. Each thread
+            // stages its rounded values in [routed row][weight row] order (a warp's 32 lanes
+            // write 64 contiguous bytes); then routed row c's slice of up to 128 weight rows,
+            // contiguous in the output, goes out with one bulk copy (thread c), so the warps
+            // return to the next tile's blocks while the copies drain. The epilogue warps meet
+            // once a tile, on an mbarrier (bounded, warp-uniform waits: an abort anywhere leaves
+            // no warp waiting forever). Before arriving, each thread waits until its copies of
+            // the tile before have read their source; so when the meeting completes, the
+            // buffer this tile's writes will reuse two tiles on is free.
+            const uint32_t obuf = sbase + kOffOut + (uint32_t)(tile_ctr & 1) * kOutBufBytes;
+            const uint32_t oph = tile_ctr & 1u;
             if (valid) {
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
@@ -523,18 +553,35 @@ prefill_band_kernel(const GroupedArgs p, const __grid_constant__ CUtensorMap xma
                         for (int c = 0; c < 16; ++c) {
                             const int slot = c0 * 16 + c;
                             if (slot < tl.cnt) {
-                                const int64_t r = tl.r0 + slot;
                                 float v = acc[j][c];
-                                if (p.row_weight) v *= __ldg(p.row_weight + r);
-                                const int64_t dst = p.row_dest ? (int64_t)__ldg(p.row_dest + r) : r;
-                                p.out[dst * p.N + n] = f32_to_out16<XH>(v);
+                                if (p.row_weight) v *= __ldg(p.row_weight + tl.r0 + slot);
+                                const uint16_t h = f32_to_out16<XH>(v);
+                                asm volatile("st.shared.u16 [%0], %1;" ::"r"(obuf + (uint32_t)slot * kOutRowBytes + (uint32_t)i * 2u),
+                                             "h"(h) : "memory");
                             }
                         }
                     }
                 }
             }
+            fence_proxy_async();
+            bulk_wait_read_all();                     // this thread's earlier copies have read their source
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_ostaged);
+            if (!__all_sync(0xffffffffu, mbar_wait_bounded(bar_ostaged, oph, abort_flag, err, 256u))) goto epi_done;
+            {
+                const int c = (warp - kEpiWarp0) * 32 + lane;      // one routed row per thread
+                if (c < tl.cnt) {
+                    const int64_t r = tl.r0 + c;
+                    const int64_t dst = p.row_dest ? (int64_t)__ldg(p.row_dest + r) : r;
+                    const uint32_t bytes = (uint32_t)min(kBM, p.N - tl.n0) * 2u;
+                    bulk_store(p.out + dst * p.N + tl.n0, obuf + (uint32_t)c * kOutRowBytes, bytes);
+                }
+                bulk_commit();
+            }
+            ++tile_ctr;
         }
-    epi_done:;
+    epi_done:
+        bulk_wait_all();                              // every output copy has landed
     }
 
     tc_fence_before();
