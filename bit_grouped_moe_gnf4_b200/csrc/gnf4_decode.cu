@@ -85,7 +85,13 @@ constexpr int kStageBytes = kTileRows * kBoxBytes;   // 8 KB: one TMA box
 #define GNF4_DB_STAGES 3
 #endif
 constexpr int kStages = GNF4_DB_STAGES;       // ring stages per quad
-constexpr int kRingBytes = kStages * kStageBytes;
+// with the scales in the stage (ST): a second box of the chunk's block scales of the same
+// 64 rows, 16 bytes a row, after the 8 KB of packed weights (stages stay 1024-aligned)
+constexpr int kScaleBoxBytes = kTileRows * 16;
+template <bool ST>
+__host__ __device__ constexpr uint32_t stage_stride() { return ST ? kStageBytes + kScaleBoxBytes : kStageBytes; }
+template <bool ST>
+__host__ __device__ constexpr uint32_t ring_bytes() { return kStages * stage_stride<ST>(); }
 constexpr int kLutBytes = 256 * 256;           // byte b, lane l -> b*256 + l*4 (bytes 128..255 of each row hold the part slots)
 constexpr int kMaxTableRows = 1024;            // routed rows whose metadata the CTA stages in shared memory
 constexpr int kMaxSmem = 227 * 1024;
@@ -258,6 +264,11 @@ __device__ __forceinline__ uint2 lds_v2(uint32_t a) {
     asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
     return v;
 }
+__device__ __forceinline__ uint4 lds_v4(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
 __device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
     uint32_t v;
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
@@ -385,7 +396,7 @@ __host__ __device__ constexpr uint32_t other_bytes(int E) {
 struct Layout {
     uint32_t lut, ring[kQuads], other;
 };
-__host__ __device__ inline bool make_layout(uint32_t base, uint32_t bytes, int E, Layout& L) {
+__host__ __device__ inline bool make_layout(uint32_t base, uint32_t bytes, int E, uint32_t kRingBytes, Layout& L) {
     const uint32_t end = base + bytes;
     const uint32_t lut = (base + 0xFFFFu) & ~0xFFFFu;
     if (lut + kLutBytes > end) return false;
@@ -421,9 +432,10 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
 
 }  // namespace db
 
-template <int FMT, int SCL, int XH, int NG, int TPW, int FUSE>
+template <int FMT, int SCL, int XH, int NG, int TPW, int FUSE, bool ST>
 __global__ void __launch_bounds__(db::kQuads * 128 / TPW, 1)
-decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant__ CUtensorMap wmap) {
+decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant__ CUtensorMap wmap,
+                   const __grid_constant__ CUtensorMap smap) {
     using namespace db;
     static_assert(!FUSE || TPW == 2, "the fused SwiGLU pairs a gate tile with its up tile in one warp");
     static_assert(2 * kQuads * 4 * NG * 32 <= 256 * 8, "the part-sum slots must fit the table's spare halves");
@@ -443,7 +455,8 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     extern __shared__ uint8_t smem_raw[];
     const uint32_t smem_s = smem_addr(smem_raw);
     Layout lay;
-    if (!make_layout(smem_s, (uint32_t)pl.smem_bytes, p.E, lay)) {
+    constexpr uint32_t kStride = stage_stride<ST>();    // bytes of one ring stage
+    if (!make_layout(smem_s, (uint32_t)pl.smem_bytes, p.E, ring_bytes<ST>(), lay)) {
         if (threadIdx.x == 0) atomicOr(&g_decode_error, 0x100u);
         return;
     }
@@ -477,6 +490,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap)) : "memory");
+        if (ST) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&smap)) : "memory");
     }
     // the lookup table comes from the kernel parameters alone, so it is built before
     // anything is read from global memory: under a programmatic dependent launch this
@@ -648,9 +662,17 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     };
     auto issue_next = [&]() {
         const uint32_t fb = smem_addr(full + cp_s);
-        mbar_arrive_tx(fb, (uint32_t)kStageBytes);
-        tma_2d(qring + (uint32_t)cp_s * kStageBytes, &wmap, cp_c * kBoxBytes, cp_y, fb);
-        if (FUSE) tma_2d(qring + (uint32_t)cp_s * kStageBytes + kStageBytes / 2, &wmap, cp_c * kBoxBytes, cp_y + I, fb);
+        const uint32_t sdst = qring + (uint32_t)cp_s * kStride;
+        mbar_arrive_tx(fb, (uint32_t)(kStageBytes + (ST ? kScaleBoxBytes : 0)));
+        tma_2d(sdst, &wmap, cp_c * kBoxBytes, cp_y, fb);
+        if (FUSE) tma_2d(sdst + kStageBytes / 2, &wmap, cp_c * kBoxBytes, cp_y + I, fb);
+        if constexpr (ST) {
+            // the 16 bytes holding this chunk's scales (8-byte formats: the pair of chunks
+            // 2j, 2j+1, whose half the math picks)
+            const int sx = (SSZ == 4) ? cp_c * 16 : (cp_c & ~1) * 8;
+            tma_2d(sdst + kStageBytes, &smap, sx, cp_y, fb);
+            if (FUSE) tma_2d(sdst + kStageBytes + kScaleBoxBytes / 2, &smap, sx, cp_y + I, fb);
+        }
         if (++cp_s == kStages) cp_s = 0;
         ++cp_j;
         --cp_left;
@@ -698,10 +720,12 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
             sc_unit();
         }
     };
-    Scales<SCL> scN[kTPW];                           // the next chunk's scales
-    if (nsteps > 0) {
-        sc_unit();
-        scales_next(scN);
+    Scales<SCL> scN[kTPW];                           // the next chunk's scales (scales not in the stage)
+    if constexpr (!ST) {
+        if (nsteps > 0) {
+            sc_unit();
+            scales_next(scN);
+        }
     }
 
     // ---- the CTA's routing metadata: the first rows' loads went out before the copies ----
@@ -873,10 +897,12 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     uint32_t rph = 0;                               // parity of that stage's release
 
     auto step = [&]() {
-        Scales<SCL> use[kTPW];                      // this chunk's scales (loaded a step ago)
+        Scales<SCL> use[kTPW];                      // this chunk's scales (loaded a step ago, or from the stage)
+        if constexpr (!ST) {
 #pragma unroll
-        for (int tt = 0; tt < kTPW; ++tt) use[tt] = scN[tt];
-        scales_next(scN);
+            for (int tt = 0; tt < kTPW; ++tt) use[tt] = scN[tt];
+            scales_next(scN);
+        }
         if (mt_ck == 0) unit_begin();
         if (!dead && !wait_bounded(smem_addr(full + cs), cph, abort_flag, stall_test)) dead = true;
         if (!dead && ntl > 0) {
@@ -884,8 +910,26 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
             uint32_t rowa[kTPW];
 #pragma unroll
             for (int tt = 0; tt < kTPW; ++tt)
-                rowa[tt] = qring + (uint32_t)cs * kStageBytes +
+                rowa[tt] = qring + (uint32_t)cs * kStride +
                            (FUSE ? (uint32_t)(32 * tt + 16 * wq + g) * kBoxBytes : lane_row + tt * 16 * kBoxBytes);
+            if constexpr (ST) {
+                // rows g and g + 8 of each tile, 16 bytes a row after the stage's weights
+                const uint32_t sb = qring + (uint32_t)cs * kStride + kStageBytes;
+#pragma unroll
+                for (int tt = 0; tt < kTPW; ++tt) {
+                    const uint32_t ra = sb + (uint32_t)(FUSE ? 32 * tt + 16 * wq + g : row0 + 16 * tt + g) * 16u;
+                    if constexpr (SCL == SC_F32) {
+                        const uint4 va = lds_v4(ra), vb = lds_v4(ra + 128u);
+                        use[tt].s[0][0] = va.x; use[tt].s[0][1] = va.y; use[tt].s[0][2] = va.z; use[tt].s[0][3] = va.w;
+                        use[tt].s[1][0] = vb.x; use[tt].s[1][1] = vb.y; use[tt].s[1][2] = vb.z; use[tt].s[1][3] = vb.w;
+                    } else {
+                        const uint32_t h = (uint32_t)(c & 1) * 8u;
+                        const uint2 va = lds_v2(ra + h), vb = lds_v2(ra + 128u + h);
+                        use[tt].s[0][0] = va.x; use[tt].s[0][1] = va.y;
+                        use[tt].s[1][0] = vb.x; use[tt].s[1][1] = vb.y;
+                    }
+                }
+            }
             if (c < nfull) {
                 if (NG == 1 || ng == 1)
                     chunk_math<FMT, SCL, XH, 1, NG, TPW, true>(rowa, woff, use, lane_sel, xp, G::NB, acc);
@@ -967,8 +1011,8 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn_db() {
     return fn;
 }
 
-template <int FMT, int SCL, int XH, int NG, int TPW, int FUSE = 0>
-static cudaError_t launch_db(const GroupedArgs& a, db::Plan& pl, cudaStream_t s) {
+template <int FMT, int SCL, int XH, int NG, int TPW, int FUSE, bool ST>
+static cudaError_t launch_db_st(const GroupedArgs& a, db::Plan& pl, cudaStream_t s) {
     const int dev = current_device();
     // the dynamic shared memory starts after the per-block reserved bytes (this kernel
     // has no static shared memory); size the launch so that the layout fits there
@@ -984,7 +1028,7 @@ static cudaError_t launch_db(const GroupedArgs& a, db::Plan& pl, cudaStream_t s)
     db::Layout lay;
     uint32_t bytes = 0;
     for (uint32_t b = 64 * 1024; b <= (uint32_t)db::kMaxSmem; b += 1024)
-        if (db::make_layout((uint32_t)rsv, b, a.E, lay)) {
+        if (db::make_layout((uint32_t)rsv, b, a.E, db::ring_bytes<ST>(), lay)) {
             bytes = b;
             break;
         }
@@ -992,7 +1036,7 @@ static cudaError_t launch_db(const GroupedArgs& a, db::Plan& pl, cudaStream_t s)
     pl.smem_bytes = (int)bytes;
     static std::atomic<bool> attr_done[64];          // per device: dynamic shared memory opted in
     if (!attr_done[dev].load(std::memory_order_acquire)) {
-        cudaError_t e = cudaFuncSetAttribute(decode_band_kernel<FMT, SCL, XH, NG, TPW, FUSE>,
+        cudaError_t e = cudaFuncSetAttribute(decode_band_kernel<FMT, SCL, XH, NG, TPW, FUSE, ST>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, db::kMaxSmem);
         if (e != cudaSuccess) return e;
         attr_done[dev].store(true, std::memory_order_release);
@@ -1001,15 +1045,32 @@ static cudaError_t launch_db(const GroupedArgs& a, db::Plan& pl, cudaStream_t s)
     if (!enc) return cudaErrorNotSupported;
     // packed weights as bytes [E*N, K/2]: boxes of 128 bytes x 64 rows (x 32 rows, two a
     // stage, for the fused SwiGLU), 128B swizzle
-    CUtensorMap wmap;
-    cuuint64_t dims[2] = {(cuuint64_t)(a.K / 2), (cuuint64_t)a.E * (cuuint64_t)a.N};
-    cuuint64_t strides[1] = {(cuuint64_t)(a.K / 2)};
-    cuuint32_t box[2] = {(cuuint32_t)db::kBoxBytes, (cuuint32_t)(FUSE ? db::kTileRows / 2 : db::kTileRows)};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.W), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    const cuuint32_t box_rows = (cuuint32_t)(FUSE ? db::kTileRows / 2 : db::kTileRows);
+    CUtensorMap wmap, smap;
+    {
+        cuuint64_t dims[2] = {(cuuint64_t)(a.K / 2), (cuuint64_t)a.E * (cuuint64_t)a.N};
+        cuuint64_t strides[1] = {(cuuint64_t)(a.K / 2)};
+        cuuint32_t box[2] = {(cuuint32_t)db::kBoxBytes, box_rows};
+        cuuint32_t estr[2] = {1, 1};
+        CUresult r = enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a.W), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    }
+    if (ST) {
+        // block scales as bytes [E*N, nblk * scale size]: boxes of 16 bytes x the weight box's rows
+        constexpr int SSZ = (SCL == db::SC_F32) ? 4 : (SCL == db::SC_BF16) ? 2 : 1;
+        cuuint64_t dims[2] = {(cuuint64_t)pl.nblk * SSZ, (cuuint64_t)a.E * (cuuint64_t)a.N};
+        cuuint64_t strides[1] = {(cuuint64_t)pl.nblk * SSZ};
+        cuuint32_t box[2] = {16, box_rows};
+        cuuint32_t estr[2] = {1, 1};
+        CUresult r = enc(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(a.scales), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    } else {
+        smap = wmap;                                 // not read
+    }
     const int grid = device_sm_count();
     // programmatic dependent launch: the kernel builds its table while the previous
     // kernel of the stream drains, and waits for it (griddepcontrol.wait) before its
@@ -1024,9 +1085,21 @@ static cudaError_t launch_db(const GroupedArgs& a, db::Plan& pl, cudaStream_t s)
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_band_kernel<FMT, SCL, XH, NG, TPW, FUSE>, a, pl, wmap);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, decode_band_kernel<FMT, SCL, XH, NG, TPW, FUSE, ST>, a, pl, wmap, smap);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+// The chunk's block scales ride in the stage with the weights (a second TMA box) when
+// every row's scales can be a TMA tensor: a row pitch of a multiple of 16 bytes and a
+// 16-byte-aligned array; else each lane loads its rows' scales itself, a chunk ahead.
+template <int FMT, int SCL, int XH, int NG, int TPW, int FUSE = 0>
+static cudaError_t launch_db(const GroupedArgs& a, db::Plan& pl, cudaStream_t s) {
+    constexpr int SSZ = (SCL == db::SC_F32) ? 4 : (SCL == db::SC_BF16) ? 2 : 1;
+    const bool st = ((int64_t)pl.nblk * SSZ) % 16 == 0 && (reinterpret_cast<uintptr_t>(a.scales) & 15u) == 0 &&
+                    (int64_t)a.E * a.N < ((int64_t)1 << 31);
+    return st ? launch_db_st<FMT, SCL, XH, NG, TPW, FUSE, true>(a, pl, s)
+              : launch_db_st<FMT, SCL, XH, NG, TPW, FUSE, false>(a, pl, s);
 }
 
 cudaError_t launch_decode_band(int fmt, const GroupedArgs& a, cudaStream_t s, bool fuse_swiglu) {
