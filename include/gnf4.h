@@ -115,7 +115,9 @@ gnf4_status gnf4_quantize_mxfp4(const float* w, int64_t rows, int64_t K,
  * x              device bf16 [T_in, K], 16-byte aligned
  * W              device uint8 [E, N, K/2] (NF4 codes as gnf4_quantize_nf4 writes them), 16-byte aligned
  * absmax         device fp32  [E, N, K/64], 4-byte aligned (any offset into a float
- *                array); 16-byte alignment lets the kernels use vector loads
+ *                array). With 16-byte alignment and K % 256 == 0 the decode band brings
+ *                each chunk's scales in with its weight copies (TMA); otherwise each lane
+ *                loads them itself. Both ways give the same bits.
  * expert_offsets device int64 [E+1], 8-byte aligned: offsets[0] = 0, non-decreasing,
  *                offsets[E] = R; empty experts (equal neighbours) are legal and cost nothing
  * row_token      device int32 [R] in [0, T_in), or NULL (then T_in >= R); 4-byte aligned
@@ -146,7 +148,8 @@ gnf4_status gnf4_grouped_gemm_nf4(const void* x, const uint8_t* W, const float* 
  * Grouped GEMM on MXFP4-packed expert weights: identical contract, with
  *   What[e, n, k] = e2m1[code(e, n, k)] * 2^(scales[e, n, k/32] - 127)
  * W      device uint8 [E, N, K/2] (element 2j in the low nibble of byte j)
- * scales device uint8 [E, N, K/32] (e8m0; 255 decodes to NaN)
+ * scales device uint8 [E, N, K/32] (e8m0; 255 decodes to NaN), any alignment; with
+ *        16-byte alignment and K % 512 == 0 the decode band copies them by TMA (same bits)
  * K % 32 == 0. The README's "MXFP4 native-byte lane": the same mainloop by
  * table swap, on the released bytes.
  */
@@ -171,7 +174,8 @@ gnf4_status gnf4_grouped_gemm_mxfp4(const void* x, const uint8_t* W, const uint8
  *    entry point? Pick by where the weights live", the --absmax-dtype bf16 paragraph:
  *    5.6 % fewer bytes per NF4 row, lossless for a bf16 source (see
  *    gnf4_absmax_to_bf16). The bf16 absmax is widened exactly to fp32 on chip; the
- *    block scaling is still fp32, outside the MMA.
+ *    block scaling is still fp32, outside the MMA. (The decode band copies bf16
+ *    absmax by TMA when it is 16-byte aligned and K % 512 == 0; same bits otherwise.)
  * gnf4_grouped_gemm_nf4_ex(x, GNF4_DTYPE_BF16, W, absmax, GNF4_DTYPE_F32, ...) is
  * gnf4_grouped_gemm_nf4(x, W, absmax, ...) bit for bit.
  * Errors: as above; INVALID_ARG for an unknown type, MISALIGNED for an absmax off
