@@ -19,10 +19,12 @@
 // accumulators of lane (g, t) end up as the 16 contiguous columns 16t..16t+15 of
 // rows g and g+8.
 //
-// Block scale: the contraction crosses rows with different scales, so the
-// scale is applied to the decoded bf16 pair before the MMA (bf16x2 multiply,
-// round to nearest). For MXFP4 the e8m0 scale is a power of two and the product
-// is exact; for NF4 the fp32 absmax is rounded to bf16 and the product once more.
+// Block scale: the contraction crosses rows with different scales, so the scale
+// is applied before the MMA (bf16x2 multiply, round to nearest), to the decoded
+// weight pair; for MXFP4 the e8m0 scale is a power of two and the product is exact,
+// for NF4 the fp32 absmax is rounded to bf16 and the product once more. NF4 items of
+// two row tiles instead scale the gradient: an item's 64 output columns are one NF4
+// scale block, so the absmax of contraction row n multiplies the gradient's column n.
 #include <climits>
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -135,14 +137,38 @@ __device__ __forceinline__ void compute_stage(uint32_t ring, int slot, uint32_t 
         for (int j = 0; j < 4; ++j)
             asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a[r][j]) : "r"(base + (uint32_t)((4 + 4 * r + j) * 128)));
     uint32_t dec[4][4];
+    if constexpr (FMT == FMT_NF4 && RT == 2) {
+        // the 64 output columns of an item lie in one NF4 scale block, so the scale of
+        // contraction row n can multiply the gradient's column n (the A fragments: 8 bf16
+        // pair multiplies for the two row tiles) instead of every decoded weight pair (16).
+        // With one row tile the saving is smaller than the latency it puts in front of the
+        // first MMA (measured), so that case scales the weights.
+        const float s0 = __uint_as_float(__shfl_sync(0xffffffffu, sraw, 2 * t));
+        const float s1 = __uint_as_float(__shfl_sync(0xffffffffu, sraw, 2 * t + 1));
+        const float s8 = __uint_as_float(__shfl_sync(0xffffffffu, sraw, 2 * t + 8));
+        const float s9 = __uint_as_float(__shfl_sync(0xffffffffu, sraw, 2 * t + 9));
+        const uint32_t sp_lo = pack_bf16x2(s0, s1), sp_hi = pack_bf16x2(s8, s9);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int row = 2 * t + (j & 1) + 8 * (j >> 1);
-        const int src_lane = (FMT == FMT_NF4) ? row : row + 16 * (g >> 2);
-        const uint32_t sp = scale_pair<FMT>(__shfl_sync(0xffffffffu, sraw, src_lane));
-        decode_word<FMT>(w[j], lut, dec[j]);
+        for (int r = 0; r < RT; ++r) {
+            a[r][0] = mul_bf16x2(a[r][0], sp_lo);
+            a[r][1] = mul_bf16x2(a[r][1], sp_lo);
+            a[r][2] = mul_bf16x2(a[r][2], sp_hi);
+            a[r][3] = mul_bf16x2(a[r][3], sp_hi);
+        }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) dec[j][i] = mul_bf16x2(dec[j][i], sp);
+        for (int j = 0; j < 4; ++j) decode_word<FMT>(w[j], lut, dec[j]);
+    } else {
+        // each decoded weight pair is scaled (MXFP4: an item's 64 columns span two scale
+        // blocks; its e8m0 scale is a power of two, so the product is exact)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int row = 2 * t + (j & 1) + 8 * (j >> 1);
+            const int src_lane = (FMT == FMT_NF4) ? row : row + 16 * (g >> 2);
+            const uint32_t sp = scale_pair<FMT>(__shfl_sync(0xffffffffu, sraw, src_lane));
+            decode_word<FMT>(w[j], lut, dec[j]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dec[j][i] = mul_bf16x2(dec[j][i], sp);
+        }
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
