@@ -100,10 +100,6 @@ constexpr int kMaxSmem = 227 * 1024;
 #ifndef GNF4_DB_CHAINS
 #define GNF4_DB_CHAINS 1
 #endif
-// most K parts of a tile (a power of two, at most kQuads)
-#ifndef GNF4_DB_MAXPARTS
-#define GNF4_DB_MAXPARTS 2
-#endif
 
 struct Plan {
     int np;          // K parts
@@ -440,6 +436,13 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     static_assert(!FUSE || TPW == 2, "the fused SwiGLU pairs a gate tile with its up tile in one warp");
     static_assert(2 * kQuads * 4 * NG * 32 <= 256 * 8, "the part-sum slots must fit the table's spare halves");
     constexpr int kTPW = TPW;
+    // A row's K sum is fixed by K alone: one chain for a single chunk, else the sum of its
+    // two halves (chunks [0, nc/2) and [nc/2, nc)), half 0 + half 1 in fp32. With two K
+    // parts each ring of a group computes one half and the hand-over adds them; with one
+    // part (only in the variants with the registers for it: NF4, 8 routed rows a pass) a
+    // ring keeps half 0 aside at the boundary and adds it at the unit's end. Either way the
+    // same bits, so the host can pick the part count from the call's load.
+    constexpr bool kHalvesInRing = (FMT == FMT_NF4) && (NG == 1);
     // FUSE: a unit is 32 gate rows [n0, n0 + 32) and their up rows [I + n0, I + n0 + 32) of
     // the fused gate_up matrix (two 32-row boxes per stage: gate in stage rows 0..31, up in
     // 32..63); warp wq takes gate rows n0 + 16 wq .. + 15 as tile 0 and the matching up rows
@@ -770,6 +773,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     int64_t mt_u = U0 + gi, mt_r0 = 0;
     int ntl = 0;                                    // this warp's tiles that exist in the unit (rows < N)
     float acc[kTPW][NG][4];
+    float half0[kHalvesInRing ? kTPW : 1][NG][4];   // one part: the unit's half-0 sums
     const uint16_t* xp[NG];
     bool dead = false;
 
@@ -824,6 +828,16 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     };
     auto unit_end = [&]() {
         if (np == 1) {
+            if constexpr (kHalvesInRing) {
+                if (pl.nc >= 2) {
+#pragma unroll
+                    for (int tt = 0; tt < kTPW; ++tt)
+#pragma unroll
+                        for (int j = 0; j < NG; ++j)
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) acc[tt][j][q] = half0[tt][j][q] + acc[tt][j][q];
+                }
+            }
             if (!dead) {
                 if (FUSE) {
 #pragma unroll
@@ -962,6 +976,20 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
 #pragma unroll
         for (int q = 0; q < NG; ++q)
             if (xp[q] != nullptr) xp[q] += kChunkK;
+        if constexpr (kHalvesInRing) {
+            // one part: the end of half 0 (chunk nc/2 - 1) puts its sums aside
+            if (np == 1 && pl.nc >= 2 && c_lo + mt_ck + 1 == pl.nc / 2) {
+#pragma unroll
+                for (int tt = 0; tt < kTPW; ++tt)
+#pragma unroll
+                    for (int j = 0; j < NG; ++j)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            half0[tt][j][q] = acc[tt][j][q];
+                            acc[tt][j][q] = 0.f;
+                        }
+            }
+        }
         if (++mt_ck == nck) {
             unit_end();
             mt_ck = 0;
@@ -986,17 +1014,6 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
                 }
         }
     }
-}
-
-static int pick_parts(int nc) {
-    // the largest power of two (at most GNF4_DB_MAXPARTS, at most nc) whose parts are
-    // within 15 % of even
-    for (int np = GNF4_DB_MAXPARTS; np > 1; np >>= 1) {
-        if (np > nc) continue;
-        const int per = (nc + np - 1) / np;
-        if (per * np * 100 <= nc * 115) return np;
-    }
-    return 1;
 }
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn_db() {
@@ -1107,7 +1124,7 @@ cudaError_t launch_decode_band(int fmt, const GroupedArgs& a, cudaStream_t s, bo
     const int SB = (fmt == FMT_NF4) ? 64 : 32;
     pl.nblk = a.K / SB;
     pl.nc = (a.K + db::kChunkK - 1) / db::kChunkK;
-    pl.np = pick_parts(pl.nc);
+    pl.np = pl.nc >= 2 ? 2 : 1;                        // K parts (one half each; see below)
     pl.smem_bytes = 0;
     const int per_chunk = db::kChunkK / SB;           // blocks of a chunk: one vector of scales per row
     // one vector load per row for a chunk's scales when every chunk's scales start
@@ -1122,6 +1139,16 @@ cudaError_t launch_decode_band(int fmt, const GroupedArgs& a, cudaStream_t s, bo
     // group either way), so the choice never changes a result.
     const int64_t mmax = a.R < (int64_t)a.m_hi ? a.R : (int64_t)a.m_hi;      // no group exceeds this
     const bool one = mmax <= 8 || a.R < 4 * (int64_t)a.E;
+    // A row's bits are fixed by K (the sum of its two K halves), so the part count may
+    // follow the load: one part (a ring takes both halves, fewer part-sum hand-overs)
+    // when the call has units for every ring of the grid twice over, in the variants
+    // that can hold half 0 aside (NF4, 8 routed rows a pass); else two.
+    if (pl.np == 2 && fmt == FMT_NF4 && one) {
+        const int64_t rows_per_unit = fuse_swiglu ? db::kTileRows / 2 : db::kTileRows;
+        const int64_t unit_rows = fuse_swiglu ? a.N / 2 : a.N;
+        const int64_t units = (a.R < (int64_t)a.E ? a.R : (int64_t)a.E) * ((unit_rows + rows_per_unit - 1) / rows_per_unit);
+        if (units >= 2 * (int64_t)db::kQuads * device_sm_count()) pl.np = 1;
+    }
     if (fuse_swiglu) {
         // gate tile and up tile in one warp: two tiles a warp for both formats
         if (fmt == FMT_NF4) {
