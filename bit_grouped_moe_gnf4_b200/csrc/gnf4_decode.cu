@@ -93,7 +93,7 @@ __host__ __device__ constexpr uint32_t stage_stride() { return ST ? kStageBytes 
 template <bool ST>
 __host__ __device__ constexpr uint32_t ring_bytes() { return kStages * stage_stride<ST>(); }
 constexpr int kLutBytes = 256 * 256;           // byte b, lane l -> b*256 + l*4 (bytes 128..255 of each row hold the part slots)
-constexpr int kMaxTableRows = 1024;            // routed rows whose metadata the CTA stages in shared memory
+constexpr int kMaxTableRows = 1024;            // routed rows whose metadata a CTA stages in shared memory (at most)
 constexpr int kMaxSmem = 227 * 1024;
 
 // independent MMA chains per scale block (their sums are added in order afterwards)
@@ -107,6 +107,7 @@ struct Plan {
     int nblk;        // scale blocks per weight row
     int vec_scales;  // a chunk's scales of one row can be read with one vector load
     int smem_bytes;  // dynamic shared memory of the launch
+    int table_rows;  // routed rows whose metadata a CTA may stage (fewer when many experts fill the space)
 };
 
 // Scale storage of the band: f32 (NF4 absmax), bf16 (NF4 absmax stored as bf16),
@@ -379,9 +380,9 @@ __device__ __forceinline__ void chunk_math(const uint32_t (&rowa)[TPW], const ui
 
 // bytes of the shared memory other than the table and the rings: barriers and abort
 // flag, expert tables, scan scratch, row table (16-byte multiple)
-__host__ __device__ constexpr uint32_t other_bytes(int E) {
+__host__ __device__ constexpr uint32_t other_bytes(int E, int table_rows) {
     return (uint32_t)(((2 * kQuads * kStages * 8 + 16 + 8ull * (E + 1) + 8ull * E + 8ull * kMaxWarps + 4ull * E +
-                        4ull * E + 4ull * kMaxWarps + 12ull * kMaxTableRows) + 15) & ~15ull);
+                        4ull * E + 4ull * kMaxWarps + 12ull * table_rows) + 15) & ~15ull);
 }
 
 // Where the rings and the rest go, given the window address of the dynamic shared
@@ -392,7 +393,8 @@ __host__ __device__ constexpr uint32_t other_bytes(int E) {
 struct Layout {
     uint32_t lut, ring[kQuads], other;
 };
-__host__ __device__ inline bool make_layout(uint32_t base, uint32_t bytes, int E, uint32_t kRingBytes, Layout& L) {
+__host__ __device__ inline bool make_layout(uint32_t base, uint32_t bytes, int E, uint32_t kRingBytes, int table_rows,
+                                            Layout& L) {
     const uint32_t end = base + bytes;
     const uint32_t lut = (base + 0xFFFFu) & ~0xFFFFu;
     if (lut + kLutBytes > end) return false;
@@ -409,7 +411,7 @@ __host__ __device__ inline bool make_layout(uint32_t base, uint32_t bytes, int E
         L.ring[q] = b;
         hi = b + kRingBytes;
     }
-    const uint32_t ob = other_bytes(E);
+    const uint32_t ob = other_bytes(E, table_rows);
     const uint32_t a = (lo + 15u) & ~15u, b = (hi + 15u) & ~15u;
     if (a + ob <= lut) L.other = a;
     else if (b + ob <= end) L.other = b;
@@ -459,7 +461,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     const uint32_t smem_s = smem_addr(smem_raw);
     Layout lay;
     constexpr uint32_t kStride = stage_stride<ST>();    // bytes of one ring stage
-    if (!make_layout(smem_s, (uint32_t)pl.smem_bytes, p.E, ring_bytes<ST>(), lay)) {
+    if (!make_layout(smem_s, (uint32_t)pl.smem_bytes, p.E, ring_bytes<ST>(), pl.table_rows, lay)) {
         if (threadIdx.x == 0) atomicOr(&g_decode_error, 0x100u);
         return;
     }
@@ -474,8 +476,8 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
     int* s_m = s_e + p.E;
     int* s_wc = s_m + p.E;                          // [kMaxWarps]
     int* t_tok = s_wc + kMaxWarps;
-    float* t_wt = reinterpret_cast<float*>(t_tok + kMaxTableRows);
-    int* t_dst = reinterpret_cast<int*>(t_wt + kMaxTableRows);
+    float* t_wt = reinterpret_cast<float*>(t_tok + pl.table_rows);
+    int* t_dst = reinterpret_cast<int*>(t_wt + pl.table_rows);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -627,7 +629,7 @@ decode_band_kernel(const GroupedArgs p, const db::Plan pl, const __grid_constant
         const int a1 = find_active(U1 - 1);
         return s_r0[a1] + s_m[a1];
     }();
-    const bool table = (rhi - rlo) <= kMaxTableRows;
+    const bool table = (rhi - rlo) <= pl.table_rows;
     const bool m_have = table && rlo + tid < rhi;
     int m_tok = 0, m_dst = 0;
     float m_wt = 0.f;
@@ -1028,11 +1030,10 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn_db() {
     return fn;
 }
 
-template <int FMT, int SCL, int XH, int NG, int TPW, int FUSE, bool ST>
-static cudaError_t launch_db_st(const GroupedArgs& a, db::Plan& pl, cudaStream_t s) {
+// the dynamic shared memory starts after the per-block reserved bytes (this kernel has
+// no static shared memory): its window address, per device
+static uint32_t decode_smem_base() {
     const int dev = current_device();
-    // the dynamic shared memory starts after the per-block reserved bytes (this kernel
-    // has no static shared memory); size the launch so that the layout fits there
     static std::atomic<int> reserved[64];            // per device: reserved shared bytes + 1 (0 = unknown)
     int rsv = reserved[dev].load(std::memory_order_relaxed) - 1;
     if (rsv < 0) {
@@ -1042,15 +1043,22 @@ static cudaError_t launch_db_st(const GroupedArgs& a, db::Plan& pl, cudaStream_t
         }
         reserved[dev].store(rsv + 1, std::memory_order_relaxed);
     }
+    return (uint32_t)rsv;
+}
+
+// the smallest dynamic shared memory that holds the layout, or 0 if none does
+static uint32_t decode_smem_bytes(int E, uint32_t ring_bytes, int table_rows) {
     db::Layout lay;
-    uint32_t bytes = 0;
+    const uint32_t base = decode_smem_base();
     for (uint32_t b = 64 * 1024; b <= (uint32_t)db::kMaxSmem; b += 1024)
-        if (db::make_layout((uint32_t)rsv, b, a.E, db::ring_bytes<ST>(), lay)) {
-            bytes = b;
-            break;
-        }
-    if (bytes == 0) return cudaErrorInvalidConfiguration;
-    pl.smem_bytes = (int)bytes;
+        if (db::make_layout(base, b, E, ring_bytes, table_rows, lay)) return b;
+    return 0;
+}
+
+template <int FMT, int SCL, int XH, int NG, int TPW, int FUSE, bool ST>
+static cudaError_t launch_db_st(const GroupedArgs& a, db::Plan& pl, cudaStream_t s) {
+    const int dev = current_device();
+    const uint32_t bytes = (uint32_t)pl.smem_bytes;   // sized by the caller for this variant
     static std::atomic<bool> attr_done[64];          // per device: dynamic shared memory opted in
     if (!attr_done[dev].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(decode_band_kernel<FMT, SCL, XH, NG, TPW, FUSE, ST>,
@@ -1113,10 +1121,21 @@ static cudaError_t launch_db_st(const GroupedArgs& a, db::Plan& pl, cudaStream_t
 template <int FMT, int SCL, int XH, int NG, int TPW, int FUSE = 0>
 static cudaError_t launch_db(const GroupedArgs& a, db::Plan& pl, cudaStream_t s) {
     constexpr int SSZ = (SCL == db::SC_F32) ? 4 : (SCL == db::SC_BF16) ? 2 : 1;
-    const bool st = ((int64_t)pl.nblk * SSZ) % 16 == 0 && (reinterpret_cast<uintptr_t>(a.scales) & 15u) == 0 &&
-                    (int64_t)a.E * a.N < ((int64_t)1 << 31);
-    return st ? launch_db_st<FMT, SCL, XH, NG, TPW, FUSE, true>(a, pl, s)
-              : launch_db_st<FMT, SCL, XH, NG, TPW, FUSE, false>(a, pl, s);
+    const bool st_ok = ((int64_t)pl.nblk * SSZ) % 16 == 0 && (reinterpret_cast<uintptr_t>(a.scales) & 15u) == 0 &&
+                       (int64_t)a.E * a.N < ((int64_t)1 << 31);
+    // shared memory: the 9 KB stages of the scale boxes when they fit beside the per-expert
+    // tables, with the largest routing-row table that fits (a CTA whose rows do not fit reads
+    // them from global memory: the same results); else 8 KB stages, the same way
+    for (int st = st_ok ? 1 : 0; st >= 0; --st)
+        for (int rows = db::kMaxTableRows; rows >= 0; rows = rows > 64 ? rows / 2 : rows - 64) {
+            const uint32_t b = decode_smem_bytes(a.E, st ? db::ring_bytes<true>() : db::ring_bytes<false>(), rows);
+            if (b == 0) continue;
+            pl.table_rows = rows;
+            pl.smem_bytes = (int)b;
+            return st ? launch_db_st<FMT, SCL, XH, NG, TPW, FUSE, true>(a, pl, s)
+                      : launch_db_st<FMT, SCL, XH, NG, TPW, FUSE, false>(a, pl, s);
+        }
+    return cudaErrorInvalidConfiguration;
 }
 
 cudaError_t launch_decode_band(int fmt, const GroupedArgs& a, cudaStream_t s, bool fuse_swiglu) {
@@ -1126,6 +1145,7 @@ cudaError_t launch_decode_band(int fmt, const GroupedArgs& a, cudaStream_t s, bo
     pl.nc = (a.K + db::kChunkK - 1) / db::kChunkK;
     pl.np = pl.nc >= 2 ? 2 : 1;                        // K parts (one half each; see below)
     pl.smem_bytes = 0;
+    pl.table_rows = db::kMaxTableRows;
     const int per_chunk = db::kChunkK / SB;           // blocks of a chunk: one vector of scales per row
     // one vector load per row for a chunk's scales when every chunk's scales start
     // on a vector boundary (16 bytes of f32 x 4, 8 bytes of e8m0 x 8); else scalar loads

@@ -363,3 +363,25 @@ def test_default_mode_row_count_invariance():
     g.device_status()
     for r in rows0[1:]:
         assert np.array_equal(r, rows0[0])
+
+
+@pytest.mark.parametrize("E", [1600, 2048])
+@pytest.mark.parametrize("fmt", ["nf4", "mxfp4"])
+def test_many_experts_decode_band(E, fmt):
+    """The most experts a call allows (2048) and a count in between: the decode band's
+    per-expert tables then take most of its shared memory, and the host shrinks the routing
+    table and, past a point, the ring stages (scale boxes or not) to make room; every row
+    against the oracle."""
+    N, K = 64, 512
+    counts = np.zeros(E, np.int64)
+    rng = np.random.default_rng(E)
+    active = np.sort(rng.choice(E, 24, replace=False))
+    counts[active] = rng.integers(1, 12, len(active))
+    counts[E - 1] = 3                                   # the last expert too
+    active = np.nonzero(counts)[0]
+    Wd, Sd, Wh, Sh = build_stack(fmt, E, N, K, seed=E + 1, oracle_experts=active)
+    b = G.explicit_batch(counts, seed=E + 2)
+    x = synth.activations_bf16(E + 3, b.T, K)
+    out = run_gemm(fmt, x, Wd, Sd, b.offsets, b.row_token, b.row_weight, b.row_dest, flags=BANDS["decode"])
+    ref = O.grouped_rows_f64(fmt, x, Wh, Sh, b.offsets, b.row_token, b.row_weight, K, np.arange(b.R))
+    check_rows(out[b.row_dest], ref, f"{E} experts {fmt}")
