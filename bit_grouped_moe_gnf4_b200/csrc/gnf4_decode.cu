@@ -8,20 +8,24 @@
 // Work. A unit is (active expert, tile of 64 weight rows, pass), where a pass
 // covers up to 8*NG routed rows of the expert (larger groups take several
 // passes). Units are numbered expert by expert, tile-major, and every CTA of the
-// persistent grid (one per SM, 16 warps) takes an equal contiguous range. The 16
-// warps form 4 quads; warp w of a quad owns rows 16w .. 16w + 15 of a tile. The K
-// axis of a tile is cut into np parts (np depends on K alone); the quads form
-// 4/np groups of np quads, group gi takes the CTA's units gi, gi + 4/np, ..., and
-// quad p of the group computes part p of each of them.
+// persistent grid (one per SM) takes an equal contiguous range; it finds the
+// expert of its first unit by binary search. A CTA has 4 box rings ("quads") of
+// 4/TPW warps each (TPW 16-row tiles a warp: 8 warps for NF4, 16 for MXFP4). The
+// K axis of a tile is cut into np = 1 or 2 parts (the host's choice per call);
+// the quads form 4/np groups of np quads, group gi takes the CTA's units gi,
+// gi + 4/np, ..., and quad p of the group computes part p of each of them.
 //
 // Loads. The packed weights stream through the tensor memory accelerator: one
 // lane of each quad issues, per 256-K chunk, one 2-D box of 64 rows x 128 bytes
-// (8 KB, 128B-swizzled) into a 3-stage ring of the quad, so two chunks (64 KB a
-// CTA) are in flight while the quad reads the third. A full barrier per stage
-// carries the copy's byte count; an empty barrier per stage collects the four
-// warps' release before the stage is refilled. Block scales and activations are
-// small: each warp reads its rows' scales one chunk ahead into registers, and the
-// activations (shared by every tile of an expert) through L1.
+// (8 KB, 128B-swizzled) into a 3-stage ring of the quad, so two chunks are in
+// flight while the quad reads the third. When a row of block scales is TMA-able
+// (16-byte pitch multiple, aligned array) a second box brings the chunk's scales
+// of the same 64 rows into the stage; otherwise each warp loads its rows' scales
+// a chunk ahead into registers. A full barrier per stage carries the copies' byte
+// count; an empty barrier per stage collects the box's warps' release before the
+// stage is refilled. The activations (shared by every tile of an expert) come
+// through L1. The table below is built before the kernel's first global read, so
+// under a programmatic dependent launch it overlaps the previous kernel's tail.
 //
 // Decode. A lane-replicated table in shared memory maps each packed byte to its
 // two 16-bit values (entry b of lane l at b*256 + l*4: 32 lookups hit 32 banks).
@@ -38,13 +42,16 @@
 // 16t + 4s + {0,1,2,3} (NF4) or 8t + 4s + {..} (MXFP4) of step s inside the
 // block, the same for both operands, so each lane reads contiguous bytes.
 //
-// Order of the fp32 sums. Each part's sum runs over its blocks in K order; the
-// parts' sums are added in part order. np and the parts depend on K only, so a
-// row's bits never depend on the other rows of the call (row-count invariance)
-// nor on which warp or CTA computed it. With np > 1 the quads of a group hand
-// their part sums over shared memory (double-buffered, one named barrier per
-// unit) and each warp reduces a share of its rows, applies the routing weight,
-// rounds and scatters. Nothing but the output is written to global memory.
+// Order of the fp32 sums. A row's K sum is one chain over its blocks in K order
+// when K is a single chunk, and otherwise the sum of its two K halves (chunks
+// [0, nc/2) and [nc/2, nc), each a chain in K order), half 0 + half 1. With two
+// parts each quad of a group computes one half and the halves meet over shared
+// memory (double-buffered, one named barrier per unit), each warp reducing a
+// share of its rows; with one part a quad keeps half 0 aside and adds it at the
+// unit's end. So a row's bits depend on K alone, never on the other rows of the
+// call (row-count invariance), the part count, or which warp or CTA computed it.
+// The epilogue applies the routing weight, rounds and scatters; nothing but the
+// output is written to global memory.
 //
 // Waits. Every barrier wait is bounded: a wait that gives up records an error
 // for gnf4_device_status, raises the CTA's abort flag (every other wait then
