@@ -25,7 +25,10 @@
 //               fp32 sums from tensor memory, multiply by the block scale
 //               (fetched four blocks ahead)
 //               and add into fp32 running sums held in registers; at the end of
-//               a tile, weight, round to bf16 and store (scatter) the outputs
+//               a tile, weight and round, stage the tile's outputs in shared
+//               memory (two buffers), meet once on an mbarrier, and send each
+//               routed row's slice to its destination row with one bulk copy, so
+//               the warps go on to the next tile while the copies drain
 // The MMA (A from tensor memory, B from shared memory) chain of each scale block
 // (64 K for NF4, 32 K for MXFP4) goes to one of three tensor-memory accumulators,
 // so the scale is applied in fp32 outside the MMA while the tensor core fills
