@@ -183,10 +183,35 @@ def measured_peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+def _code_only(text):
+    """C++/CUDA source without comments and whitespace: what a kernel is made of."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        if text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif text[i] in "\"'":
+            q, j = text[i], i + 1
+            while j < n and text[j] != q:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            if not text[i].isspace():
+                out.append(text[i])
+            i += 1
+    return "".join(out)
+
+
 def kernel_source_hash(names):
+    """Hash of the kernel sources' code (comments and whitespace do not count)."""
     h = hashlib.sha256()
     for n in names:
-        h.update(open(os.path.join(ROOT, "bit_grouped_moe_gnf4_b200", "csrc", n), "rb").read())
+        text = open(os.path.join(ROOT, "bit_grouped_moe_gnf4_b200", "csrc", n), encoding="utf-8").read()
+        h.update(_code_only(text).encode())
     return h.hexdigest()[:16]
 
 
